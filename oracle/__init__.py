@@ -1,0 +1,133 @@
+"""fp64 CPU oracle for exact attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import this package.  The CUDA library never uses it, and the two share no code.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, IEEE binary64): for every requested
+query row it materialises the full score row ``s_j = scale * q.k_j`` over the admissible
+keys, takes its maximum ``m``, forms ``p_j = exp(s_j - m)``, ``l = sum_j p_j`` and
+returns ``O = sum_j p_j v_j / l`` and ``LSE = m + ln l``.  That is the attention formula
+``softmax(Q K^T / sqrt(d_k)) V`` of the page "FlashAttention (DE)", section
+"Problematik der Standard-Attention", which the pages say FlashAttention reproduces
+exactly.  This module only marshals arrays into that library.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+F64, BF16, E4M3 = 0, 1, 2
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        lib.oracle_attention_rows.restype = ctypes.c_int
+        lib.oracle_attention_rows.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int]
+        lib.oracle_decode_bf16.restype = ctypes.c_double
+        lib.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
+        lib.oracle_decode_e4m3.restype = ctypes.c_double
+        lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_max_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _as_numpy(x):
+    """CPU numpy view of a numpy array or CPU torch tensor (bf16 -> uint16 bits,
+    float8_e4m3fn -> uint8 bits)."""
+    if isinstance(x, np.ndarray):
+        return x
+    import torch  # only for tensors handed in by the caller
+    if x.dtype == torch.bfloat16:
+        x = x.view(torch.uint16) if hasattr(torch, "uint16") else x.view(torch.int16)
+    elif x.dtype == torch.float8_e4m3fn:
+        x = x.view(torch.uint8)
+    return x.detach().cpu().contiguous().numpy()
+
+
+def _elem_type(a: np.ndarray) -> int:
+    if a.dtype == np.float64:
+        return F64
+    if a.dtype in (np.uint16, np.int16):
+        return BF16
+    if a.dtype in (np.uint8, np.int8):
+        return E4M3
+    raise TypeError("oracle inputs must be float64, bf16 bits (uint16) or e4m3 bits "
+                    "(uint8); got %s" % a.dtype)
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def attention_rows(q, k, v, scale, causal=False, rows=None, descale_q=None,
+                   descale_k=None, descale_v=None, nthreads=0):
+    """Exact attention for selected query rows.
+
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] -- float64 values, bf16 bit patterns or
+    e4m3 bit patterns (all three of one kind).  rows: flattened row indices
+    ``(b*Hq + hq)*Nq + i`` or None for every row.  descale_*: per-(batch, head)
+    multipliers for e4m3 inputs.  Returns (o [nrows, d] float64, lse [nrows] float64).
+    """
+    qa, ka, va = (np.ascontiguousarray(_as_numpy(t)) for t in (q, k, v))
+    et = _elem_type(qa)
+    if _elem_type(ka) != et or _elem_type(va) != et:
+        raise TypeError("q, k and v must share one storage format")
+    B, Hq, Nq, d = qa.shape
+    Bk, Hkv, Nk, dk = ka.shape
+    if va.shape != ka.shape or Bk != B or dk != d:
+        raise ValueError("shape mismatch between q, k and v")
+    if rows is None:
+        nrows = B * Hq * Nq
+        rows_arr = None
+        rows_ptr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        nrows = rows_arr.size
+        rows_ptr = rows_arr.ctypes.data
+    o = np.empty((nrows, d), dtype=np.float64)
+    lse = np.empty((nrows,), dtype=np.float64)
+    ds = []
+    for arr in (descale_q, descale_k, descale_v):
+        ds.append(None if arr is None else
+                  np.ascontiguousarray(np.asarray(_as_numpy(arr), dtype=np.float64).reshape(-1)))
+    rc = _load().oracle_attention_rows(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, et,
+        None if ds[0] is None else ds[0].ctypes.data,
+        None if ds[1] is None else ds[1].ctypes.data,
+        None if ds[2] is None else ds[2].ctypes.data,
+        B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+        rows_ptr, nrows, o.ctypes.data, lse.ctypes.data, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_attention_rows failed with code %d" % rc)
+    return o, lse
+
+
+def attention(q, k, v, scale, causal=False, **kw):
+    """All rows: returns (o [B, Hq, Nq, d], lse [B, Hq, Nq]) in float64."""
+    qa = _as_numpy(q)
+    B, Hq, Nq, d = qa.shape
+    o, lse = attention_rows(q, k, v, scale, causal, rows=None, **kw)
+    return o.reshape(B, Hq, Nq, d), lse.reshape(B, Hq, Nq)
+
+
+def decode_bf16(bits: int) -> float:
+    return float(_load().oracle_decode_bf16(int(bits)))
+
+
+def decode_e4m3(code: int) -> float:
+    return float(_load().oracle_decode_e4m3(int(code)))

@@ -1,0 +1,131 @@
+"""Seeded synthetic workloads for the attention forward pass.
+
+This module only draws inputs.  It holds none of the attention arithmetic, so that both
+the CUDA library (through the tests and ``bench.py``) and the CPU oracle can be fed the
+same bytes.  Every tensor is drawn on the CPU from a ``torch.Generator`` seeded per
+workload, in a fixed order (Q, then K, then V, then -- fp8 only -- the outlier masks),
+and stored contiguous in [batch, heads, sequence, head_dim] order.
+
+The shapes are the five workloads the attention pages motivate: a tiny case, a
+GPT-2-small-shaped case (batch 16, 12 heads, 2048 tokens: the shape the "Flash
+Attention" page uses for its memory comparison in "Performance-Benchmarks"), a 16K-token
+long-context case (same page: 16K-token training), a grouped-query case (4 query heads
+per K/V head) and an fp8-e4m3 case with sparse large-magnitude entries (the outliers
+that the page "FlashAttention-3 (DE)" names as the risk of FP8 quantisation, section
+"Niedrige Praezision (FP8) mit reduziertem Quantisierungsfehler").  None of the pages
+benchmarks on a public dataset, so the values are i.i.d. standard normal.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional
+
+import torch
+
+E4M3_MAX = 448.0
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    in_dtype: str          # "bf16" or "e4m3"
+    out_dtype: str         # "bf16" or "f32"
+    seed: int
+    outlier_rate: float = 0.0
+    outlier_scale: float = 1.0
+
+    @property
+    def scale(self) -> float:
+        """Softmax scale 1/sqrt(d), rounded to fp32 (the value both sides receive)."""
+        return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32))
+
+    @property
+    def flops(self) -> float:
+        """Algorithmic FLOPs: 4*B*Hq*Nq*Nk*d, halved under the causal mask."""
+        f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def describe(self) -> Dict[str, object]:
+        return {"workload": self.name, "B": self.B, "Hq": self.Hq, "Hkv": self.Hkv,
+                "Nq": self.N, "Nk": self.N, "d": self.d, "causal": self.causal,
+                "in_dtype": self.in_dtype, "out_dtype": self.out_dtype,
+                "seed": self.seed}
+
+
+WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
+    Workload("tiny", 1, 2, 2, 256, 64, False, "bf16", "f32", 1001),
+    Workload("gpt2", 16, 12, 12, 2048, 64, False, "bf16", "bf16", 1002),
+    Workload("gpt2_causal", 16, 12, 12, 2048, 64, True, "bf16", "bf16", 1002),
+    Workload("long_causal", 1, 32, 32, 16384, 128, True, "bf16", "bf16", 1003),
+    Workload("long", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003),
+    Workload("gqa_causal", 4, 32, 8, 8192, 128, True, "bf16", "bf16", 1004),
+    Workload("fp8", 8, 16, 16, 4096, 128, False, "e4m3", "bf16", 1005, 1e-3, 50.0),
+]}
+
+
+@dataclasses.dataclass
+class Inputs:
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    descale_q: Optional[torch.Tensor] = None   # fp32 [B*Hq]   (e4m3 only)
+    descale_k: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
+    descale_v: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
+
+
+def _quantise_e4m3_per_head(x: torch.Tensor):
+    """Per-(batch, head) amax scaling into OCP e4m3: s = amax/448, code = e4m3(x/s).
+
+    Returns (codes as torch.float8_e4m3fn, descale s as fp32 [B*H]).  The cast is
+    torch's round-to-nearest-even; the clamp keeps x/s inside the finite range.
+    """
+    B, H = x.shape[:2]
+    amax = x.abs().amax(dim=(2, 3)).to(torch.float32)
+    s = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    y = (x / s[:, :, None, None]).clamp_(-E4M3_MAX, E4M3_MAX)
+    return y.to(torch.float8_e4m3fn).contiguous(), s.reshape(B * H).contiguous()
+
+
+def make_inputs(w: Workload, seed: Optional[int] = None, *, B: Optional[int] = None,
+                Hq: Optional[int] = None, Hkv: Optional[int] = None,
+                Nq: Optional[int] = None, Nk: Optional[int] = None,
+                d: Optional[int] = None) -> Inputs:
+    """Draw the inputs of workload ``w`` (shape overrides give smaller variants with the
+    same value distribution)."""
+    B = w.B if B is None else B
+    Hq = w.Hq if Hq is None else Hq
+    Hkv = w.Hkv if Hkv is None else Hkv
+    Nq = w.N if Nq is None else Nq
+    Nk = w.N if Nk is None else Nk
+    d = w.d if d is None else d
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    q32 = torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32)
+    k32 = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
+    v32 = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
+    if w.in_dtype == "bf16":
+        return Inputs(q32.to(torch.bfloat16), k32.to(torch.bfloat16), v32.to(torch.bfloat16))
+    if w.in_dtype != "e4m3":
+        raise ValueError(w.in_dtype)
+    for t in (q32, k32, v32):
+        if w.outlier_rate > 0:
+            mask = torch.rand(t.shape, generator=g) < w.outlier_rate
+            t[mask] *= w.outlier_scale
+    q8, dq = _quantise_e4m3_per_head(q32)
+    k8, dk = _quantise_e4m3_per_head(k32)
+    v8, dv = _quantise_e4m3_per_head(v32)
+    return Inputs(q8, k8, v8, dq, dk, dv)
+
+
+def random_bf16(shape, seed: int) -> torch.Tensor:
+    """Standard-normal bf16 tensor from a seeded generator (for ad-hoc test shapes)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
