@@ -1,0 +1,402 @@
+"""Throughput benchmark of the fused attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one ``fa_fwd`` call over the whole workload (scheduler, TMA loads, S = QK^T,
+masked online softmax with lazy rescaling, O += PV, epilogue).  The default workload is
+the long-context non-causal case (B=1, H=32, N=16384, d=128, bf16), whose Q/K/V (402 MB)
+exceed the 126 MB L2, so no flush is needed between steps.  Rank 0 prints one JSON line.
+
+With N > 1 (launched by torchrun) every rank runs its own copy of the workload on its own
+GPU with its own seed -- the (batch, head) units are independent, so the work shards with
+no exchange step and no collective on the data path (weak scaling); the only
+collectives are the timing barrier and the max over ranks of the elapsed time.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload
+(rank 0 only) and prints the same line with ``"impl": "reference"``.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s on 1 B200 and % of dense tensor peak (causal halved)"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_FP8_TFLOPS = 4500.0
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["exact_attention_101_b200/csrc/fa_fwd_kernel.cuh",
+                  "exact_attention_101_b200/csrc/sm100.cuh",
+                  "exact_attention_101_b200/csrc/fa_api.cu"]
+
+
+# ------------------------------------------------------------------ host-side helpers
+
+def rank_env():
+    """(rank, local_rank, world_size) from the torchrun environment (defaults 0, 0, 1)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def rank_seed(w, rank):
+    """Each rank draws its own batch: weak scaling over independent problems."""
+    return w.seed + 7919 * rank
+
+
+def max_over_ranks(value_ms, world_size, device=None):
+    """Max of a per-rank elapsed time over all ranks (the job is as slow as its slowest
+    rank).  Uses the default process group when world_size > 1."""
+    if world_size <= 1:
+        return float(value_ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload_name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(workload_name)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = str(gpu_index)
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, flag in zip(names, f[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_sample_rate(w, inp, target_s, seed=0):
+    """Time the fp64 oracle on a random sample of query rows of the workload.  Returns
+    (TFLOP/s, description, threads, rows, seconds)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    total_rows = w.B * w.Hq * w.N
+
+    def row_flops(rows):
+        i = rows % w.N
+        keys = (i + 1) if w.causal else np.full_like(i, w.N)
+        return float(4.0 * w.d * keys.sum())
+
+    kw = {}
+    if inp.descale_q is not None:
+        kw = dict(descale_q=inp.descale_q.double(), descale_k=inp.descale_k.double(),
+                  descale_v=inp.descale_v.double())
+    n = 16
+    while True:
+        rows = rng.integers(0, total_rows, size=n)
+        t0 = time.perf_counter()
+        oracle.attention_rows(inp.q, inp.k, inp.v, w.scale, w.causal, rows=rows, **kw)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or n >= total_rows:
+            break
+        n = int(min(total_rows, max(2 * n, n * target_s / max(dt, 1e-3) * 1.1)))
+    fl = row_flops(rows)
+    desc = ("%d random query rows (of %d) of workload %s, full key range per row, fp64"
+            % (n, total_rows, w.name))
+    return fl / dt / 1e12, desc, oracle.max_threads(), n, dt
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args):
+    import torch
+    import exact_attention_101_b200 as fa
+
+    rank, local_rank, world = rank_env()
+    w = workloads.WORKLOADS[args.workload]
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    inp = workloads.make_inputs(w, seed=rank_seed(w, rank))
+    host = [inp.q, inp.k, inp.v]
+    q, k, v = (t.to(dev) for t in host)
+    fp8 = inp.descale_q is not None
+    if fp8:
+        dq, dk, dv = (t.to(dev) for t in (inp.descale_q, inp.descale_k, inp.descale_v))
+    out_dtype = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    o = torch.empty((w.B, w.Hq, w.N, w.d), dtype=out_dtype, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if fp8:
+            fa.forward_fp8(q, k, v, dq, dk, dv, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        else:
+            fa.forward(q, k, v, causal=w.causal, scale=w.scale, out_dtype=out_dtype, out=o,
+                       lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    fa.check_device_error(stream)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    fa.check_device_error(stream)
+    elapsed_ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(elapsed_ms, world, dev)
+    ms_per_step = ms_max / args.steps
+    value = w.flops * world * args.steps / (ms_max / 1e3) / 1e12
+    # Dominant (only) kernel: one fa_fwd launch per step on `stream`, so its average
+    # launch duration is this rank's elapsed time / steps.
+    kernel_ms = elapsed_ms / args.steps
+    achieved = w.flops / (kernel_ms / 1e3) / 1e12
+
+    # End to end through the public API: pinned host inputs -> device, forward, O and LSE
+    # back to pinned host memory, every step inside the timed region.
+    e2e_steps = max(3, min(args.steps, 20))
+    hq_, hk_, hv_ = (t.pin_memory() for t in host)
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    if fp8:
+        hds = [t.pin_memory() for t in (inp.descale_q, inp.descale_k, inp.descale_v)]
+
+    def e2e_step():
+        q.copy_(hq_, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        if fp8:
+            for dst, src in zip((dq, dk, dv), hds):
+                dst.copy_(src, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    if fp8:
+        h2d += sum(t.numel() * t.element_size() for t in hds)
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    e2e = {"value": w.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    if fp8:
+        peak = peaks["bf16_tflops"] * 2.0   # fp8 dense = 2x bf16 dense (nominal ratio)
+        peak_note = "fp8 peak = measured bf16 burst x 2 (nominal fp8/bf16 ratio)"
+    else:
+        peak = peaks["bf16_tflops"]
+        peak_note = "measured cuBLAS bf16 burst (kernel timed alone)"
+    datasheet = DATASHEET_FP8_TFLOPS if fp8 else DATASHEET_BF16_TFLOPS
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        rate, desc, cores, _, _ = oracle_sample_rate(w, inp, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
+        "config": dict(w.describe(), l2="inputs larger than L2 (no flush)",
+                       parallelism="independent replicas of the workload per GPU"),
+        "frac_of_datasheet_peak": achieved / datasheet,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": profiled_traffic(w.name),
+                     "peak_source": "%s (%s)" % (peak_src, peak_note),
+                     "kernel": "fa_fwd_kernel"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line))
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank, _, world = rank_env()
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_inputs(w)
+    per_step = max(0.2, args.reference_budget_s / max(1, args.steps + args.warmup))
+    for i in range(args.warmup):
+        oracle_sample_rate(w, inp, per_step, seed=100 + i)
+    rates, descs, total_s = [], [], 0.0
+    cores = 1
+    for i in range(args.steps):
+        rate, desc, cores, _, dt = oracle_sample_rate(w, inp, per_step, seed=i)
+        rates.append(rate)
+        descs.append(desc)
+        total_s += dt
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(w.describe(), l2="n/a (CPU)",
+                       parallelism="independent replicas of the workload per GPU"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "per step: " + descs[-1]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="long", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU time spent timing the oracle for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-budget-s", type=float, default=120.0,
+                    help="total CPU time of the reference arm")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    _, _, world = rank_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus %d needs torchrun with %d processes" % (args.gpus, args.gpus))
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,163 @@
+"""B200-native fused exact attention forward: Python binding of ``libfa_b200.so``.
+
+The C ABI (``include/fa_b200.h``) is the product; this module only marshals arguments
+into it.  The functions ``fa_fwd``, ``fa_fwd_fp8``, ``fa_check_device_error`` and
+``fa_status_string`` have the names and argument order of the C entry points and take
+raw device pointers.  ``forward`` / ``forward_fp8`` are conveniences that take CUDA
+tensors (PyTorch provides device memory and streams only), allocate the outputs and
+raise on a non-zero status.  Every step of the attention runs in the CUDA kernels; there
+is no CPU or library fallback -- if the shared library is missing, importing a function
+that needs it raises.
+"""
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
+
+# Exported C symbols, in the order of include/fa_b200.h.
+C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_check_device_error", "fa_status_string", "fa_version")
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s failed: %s (status %d)" % (what, fa_status_string(status), status))
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libfa_b200.so not found at %s; build it with "
+                              "`python -m exact_attention_101_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.fa_fwd.restype = i
+        L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+        L.fa_fwd_fp8.restype = i
+        L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+        L.fa_check_device_error.restype = i
+        L.fa_check_device_error.argtypes = [vp]
+        L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_status_string.argtypes = [i]
+        L.fa_version.restype = i
+        L.fa_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------ raw C-ABI mirrors
+
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    """Raw ``fa_fwd``: pointers are ints (device addresses), stream an int handle."""
+    return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream)
+
+
+def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+               descale_q, descale_k, descale_v, stream) -> int:
+    """Raw ``fa_fwd_fp8``."""
+    return lib().fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                            descale_q, descale_k, descale_v, stream)
+
+
+def fa_check_device_error(stream) -> int:
+    return lib().fa_check_device_error(stream)
+
+
+def fa_status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def fa_version() -> int:
+    return lib().fa_version()
+
+
+# ------------------------------------------------------------------ tensor conveniences
+
+def _stream_handle(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check_inputs(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError("%s must be a CUDA tensor" % name)
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous [B, H, N, d]" % name)
+        if t.dim() != 4:
+            raise ValueError("%s must have 4 dimensions [B, H, N, d]" % name)
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError("shape mismatch: q %s, k %s, v %s" % (tuple(q.shape), tuple(k.shape),
+                                                               tuple(v.shape)))
+    return B, Hq, Hkv, Nq, Nk, d
+
+
+def forward(q, k, v, causal=False, scale=None, out_dtype=None, out=None, lse=None,
+            stream=None):
+    """Exact attention forward for bf16 CUDA tensors in [B, H, N, d] layout.
+
+    Returns ``(o, lse)``: o in ``out_dtype`` (torch.bfloat16 default, or torch.float32),
+    lse fp32 [B, Hq, Nq] (natural log).  ``scale`` defaults to 1/sqrt(d).
+    """
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _check_inputs(q, k, v)
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise ValueError("forward() takes bf16 q, k, v; use forward_fp8() for e4m3")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    dtype = FA_BF16_OUT_F32 if out_dtype == torch.float32 else FA_BF16
+    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), dtype, _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def forward_fp8(q, k, v, descale_q, descale_k, descale_v, causal=False, scale=None,
+                out=None, lse=None, stream=None):
+    """fp8-e4m3 attention forward with per-(batch, head) fp32 descales; bf16 output."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _check_inputs(q, k, v)
+    for t in (q, k, v):
+        if t.dtype != torch.float8_e4m3fn:
+            raise ValueError("forward_fp8() takes torch.float8_e4m3fn q, k, v")
+    for name, t, n in (("descale_q", descale_q, B * Hq), ("descale_k", descale_k, B * Hkv),
+                       ("descale_v", descale_v, B * Hkv)):
+        if not t.is_cuda or t.dtype != torch.float32 or t.numel() != n or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CUDA fp32 tensor of %d entries" % (name, n))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    st = fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                    B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), descale_q.data_ptr(),
+                    descale_k.data_ptr(), descale_v.data_ptr(), _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_fp8")
+    return out, lse
+
+
+def check_device_error(stream=None):
+    """Raise FaError if a bounded device-side wait gave up since the last check."""
+    st = fa_check_device_error(_stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "device")

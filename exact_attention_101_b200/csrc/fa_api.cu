@@ -1,0 +1,295 @@
+// fa_api.cu -- host side of the C ABI declared in include/fa_b200.h: argument
+// validation, TMA tensor-map encoding, kernel-instance selection and launch.
+//
+// Every call validates its arguments on the host before any CUDA call is made, so an
+// invalid request never reaches the GPU.  Buffers are then checked to be device (or
+// managed) memory of the current device whose allocation covers the bytes the shape
+// implies; only then are the three TMA descriptors encoded and one persistent kernel
+// launched on the caller's stream.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa_b200.h"
+#include "fa_fwd_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+using PFN_encodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                     const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                     const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+using PFN_addressRange = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+struct DriverFns {
+  PFN_encodeTiled encode = nullptr;
+  PFN_addressRange range = nullptr;
+  bool ok = false;
+};
+
+const DriverFns &driver_fns() {
+  static DriverFns fns;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.encode = reinterpret_cast<PFN_encodeTiled>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.range = reinterpret_cast<PFN_addressRange>(fn);
+    fns.ok = fns.encode && fns.range;
+  });
+  return fns;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0, minor = 0;
+  int max_smem_optin = 0;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev_info[kMaxDevices];
+bool g_dev_known[kMaxDevices] = {};
+
+fa_status device_info(int dev, DeviceInfo *out) {
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev_known[dev]) {
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return FA_ERR_CUDA;
+    g_dev_info[dev] = d;
+    g_dev_known[dev] = true;
+  }
+  *out = g_dev_info[dev];
+  return FA_OK;
+}
+
+// Device or managed memory of device `dev`, and the allocation holding `p` extends at
+// least `bytes` past it.
+bool buffer_ok(const void *p, size_t bytes, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return false;
+  if (a.type == cudaMemoryTypeDevice && a.device != dev) return false;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (driver_fns().range(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS)
+    return false;
+  const uint64_t end = static_cast<uint64_t>(reinterpret_cast<uintptr_t>(p)) + bytes;
+  return end <= static_cast<uint64_t>(base) + size;
+}
+
+// 3-D tensor map over a [heads, rows, d] tensor, box = [1, 128, box_inner], 128-byte
+// swizzle, out-of-bounds elements read as zero.
+bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_t rows,
+                 uint64_t heads) {
+  const uint64_t eb = fp8 ? 1 : 2;
+  cuuint64_t dims[3] = {d, rows, heads};
+  cuuint64_t strides[2] = {d * eb, rows * d * eb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = driver_fns().encode(
+      m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+      const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool CAUSAL, bool OUT_F32, bool FP8>
+fa_status launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                 const fa::FwdParams &p, int grid, int dev, cudaStream_t stream) {
+  using C = fa::TileCfg<D, FP8>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, OUT_F32, FP8>;
+  static std::once_flag attr_once[kMaxDevices];
+  static fa_status attr_st[kMaxDevices];
+  std::call_once(attr_once[dev], [&] {
+    attr_st[dev] = FA_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess) {
+      attr_st[dev] = FA_ERR_CUDA;
+      return;
+    }
+    // The warpgroups re-split the launch register pool with setmaxnreg; a build that
+    // launches with fewer registers per thread than the split assumes would wait forever
+    // in setmaxnreg.inc, so it is never launched.
+    cudaFuncAttributes fa_attr;
+    if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess) {
+      attr_st[dev] = FA_ERR_CUDA;
+      return;
+    }
+    if (fa_attr.numRegs * fa::NUM_THREADS < 256 * fa::SOFTMAX_REGS + 128 * fa::OTHER_REGS)
+      attr_st[dev] = FA_ERR_UNSUPPORTED;
+  });
+  if (attr_st[dev] != FA_OK) return attr_st[dev];
+  kern<<<grid, fa::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Pure host-side checks; no CUDA call.  Returns FA_OK or the error to report.
+fa_status check_args(const void *q, const void *k, const void *v, const void *o,
+                     const float *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                     float scale, int causal, bool fp8, const float *dq, const float *dk,
+                     const float *dv) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (fp8 && (!dq || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (fp8 && ((reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
+               reinterpret_cast<uintptr_t>(dv)) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  // Index ranges: work-unit and row counts must fit the kernel's 32-bit arithmetic.
+  const int64_t bh = static_cast<int64_t>(B) * Hq;
+  const int64_t units = bh * ((static_cast<int64_t>(Nq) + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS);
+  if (bh > INT32_MAX || static_cast<int64_t>(B) * Hkv > INT32_MAX || units > INT32_MAX)
+    return FA_ERR_INVALID_ARG;
+  if (Nk > INT32_MAX - 2 * fa::BN || Nq > INT32_MAX - 2 * fa::UNIT_ROWS) return FA_ERR_INVALID_ARG;
+  if (fp8 ? d != 128 : (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (causal && Nq != Nk) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     bool out_f32, bool fp8, const float *dq, const float *dk, const float *dv,
+                     cudaStream_t stream) {
+  fa_status st = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, fp8, dq, dk, dv);
+  if (st != FA_OK) return st;
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  DeviceInfo info;
+  st = device_info(dev, &info);
+  if (st != FA_OK) return st;
+  if (info.major != 10 || info.minor != 0) return FA_ERR_UNSUPPORTED;
+  if (!driver_fns().ok) return FA_ERR_CUDA;
+
+  const uint64_t eb = fp8 ? 1 : 2;
+  const uint64_t q_bytes = static_cast<uint64_t>(B) * Hq * Nq * d * eb;
+  const uint64_t kv_bytes = static_cast<uint64_t>(B) * Hkv * Nk * d * eb;
+  const uint64_t o_bytes = static_cast<uint64_t>(B) * Hq * Nq * d * (out_f32 ? 4 : 2);
+  const uint64_t lse_bytes = static_cast<uint64_t>(B) * Hq * Nq * 4;
+  if (!buffer_ok(q, q_bytes, dev) || !buffer_ok(k, kv_bytes, dev) || !buffer_ok(v, kv_bytes, dev) ||
+      !buffer_ok(o, o_bytes, dev) || !buffer_ok(lse, lse_bytes, dev))
+    return FA_ERR_INVALID_ARG;
+  if (fp8 && (!buffer_ok(dq, static_cast<size_t>(B) * Hq * 4, dev) ||
+              !buffer_ok(dk, static_cast<size_t>(B) * Hkv * 4, dev) ||
+              !buffer_ok(dv, static_cast<size_t>(B) * Hkv * 4, dev)))
+    return FA_ERR_INVALID_ARG;
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_tmap(&tq, q, fp8, d, Nq, static_cast<uint64_t>(B) * Hq) ||
+      !encode_tmap(&tk, k, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv) ||
+      !encode_tmap(&tv, v, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv))
+    return FA_ERR_INVALID_ARG;
+
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.descale_q = dq;
+  p.descale_k = dk;
+  p.descale_v = dv;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.num_qb = (Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  p.num_units = B * Hq * p.num_qb;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  const int grid = p.num_units < info.sms ? p.num_units : info.sms;
+
+  if (fp8) {
+    if (causal) return launch<128, true, false, true>(tq, tk, tv, p, grid, dev, stream);
+    return launch<128, false, false, true>(tq, tk, tv, p, grid, dev, stream);
+  }
+  if (d == 64) {
+    if (causal)
+      return out_f32 ? launch<64, true, true, false>(tq, tk, tv, p, grid, dev, stream)
+                     : launch<64, true, false, false>(tq, tk, tv, p, grid, dev, stream);
+    return out_f32 ? launch<64, false, true, false>(tq, tk, tv, p, grid, dev, stream)
+                   : launch<64, false, false, false>(tq, tk, tv, p, grid, dev, stream);
+  }
+  if (causal)
+    return out_f32 ? launch<128, true, true, false>(tq, tk, tv, p, grid, dev, stream)
+                   : launch<128, true, false, false>(tq, tk, tv, p, grid, dev, stream);
+  return out_f32 ? launch<128, false, true, false>(tq, tk, tv, p, grid, dev, stream)
+                 : launch<128, false, false, false>(tq, tk, tv, p, grid, dev, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                 int Hkv, int Nq, int Nk, int d, float scale, int causal, fa_dtype dtype,
+                 fa_stream_t stream) {
+  if (dtype != FA_BF16 && dtype != FA_BF16_OUT_F32) return FA_ERR_INVALID_ARG;
+  return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                    dtype == FA_BF16_OUT_F32, false, nullptr, nullptr, nullptr,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     const float *descale_q, const float *descale_k, const float *descale_v,
+                     fa_stream_t stream) {
+  return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, false, true,
+                    descale_q, descale_k, descale_v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_check_device_error(fa_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, fa::g_fa_error, sizeof(word)) != cudaSuccess) return FA_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_fa_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+const char *fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "success";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

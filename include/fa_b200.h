@@ -1,0 +1,124 @@
+/*
+ * fa_b200.h -- C ABI of the B200 (sm_100a) fused exact-attention forward library.
+ *
+ * The library computes, for every batch b, query head hq and query row i,
+ *
+ *     O[b,hq,i,:] = sum_j softmax_j( scale * q_i . k_j  [+ causal mask] ) * v_j
+ *     LSE[b,hq,i] = ln sum_j exp( scale * q_i . k_j )          (admissible j only)
+ *
+ * i.e. softmax(Q K^T / sqrt(d_k)) V from the page "FlashAttention (DE)", section
+ * "Problematik der Standard-Attention", with the scale passed explicitly, plus the
+ * per-row natural-log normaliser.  The N x N score matrix never reaches device memory:
+ * Q/K/V are tiled through shared memory and tensor memory and an online softmax keeps a
+ * running maximum and sum per row (same page, sections "Tiling und blockweise
+ * Verarbeitung", "Online-Softmax-Berechnung" and "Zusammenfassen von Operationen in
+ * einem CUDA-Kernel").  The result is exact up to floating-point rounding, as the
+ * pages state for FlashAttention.
+ *
+ * Layout (all tensors contiguous, row-major, device memory of the current device):
+ *   q : [B, Hq,  Nq, d]      k, v : [B, Hkv, Nk, d]
+ *   o : [B, Hq,  Nq, d]      lse  : [B, Hq,  Nq]  (fp32)
+ * Grouped-query / multi-query attention: Hq must be a multiple of Hkv and query head hq
+ * reads K/V head hq / (Hq / Hkv) (consecutive query heads share a K/V head).
+ * Causal masking admits key j for query i iff j <= i and requires Nq == Nk.
+ *
+ * Ownership: the caller allocates and owns every buffer.  The library allocates no
+ * device memory in these calls and keeps no pointer after a call returns.
+ *
+ * Execution: every call validates its arguments on the host first; on a validation error
+ * it returns without touching the GPU.  Otherwise it enqueues one kernel on `stream`
+ * and returns immediately (asynchronous).  A device-side wait that gave up (see
+ * fa_check_device_error) is reported by the next fa_check_device_error call.
+ *
+ * Thread safety: calls from several host threads are allowed.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; 0 means the legacy default stream. */
+typedef struct CUstream_st *fa_stream_t;
+
+typedef enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, bad size, bad scale, buffer
+                                too small for the given shape or not device memory */
+    FA_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement: head
+                                dim not 64/128, causal with Nq != Nk, GPU not sm_100 */
+    FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, attribute) */
+    FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (see below) */
+} fa_status;
+
+typedef enum fa_dtype {
+    FA_BF16 = 0,          /* q, k, v bf16 -> o bf16, lse fp32 */
+    FA_BF16_OUT_F32 = 1,  /* q, k, v bf16 -> o fp32, lse fp32 */
+    FA_E4M3 = 2           /* q, k, v OCP fp8 e4m3 -> o bf16, lse fp32; use fa_fwd_fp8 */
+} fa_dtype;
+
+/*
+ * Fused attention forward, bf16 inputs, fp32 accumulation.
+ *
+ *   q, k, v  device pointers to bf16 tensors in the layout above (16-byte aligned)
+ *   o        device pointer, bf16 (FA_BF16) or fp32 (FA_BF16_OUT_F32), [B,Hq,Nq,d]
+ *   lse      device pointer, fp32 [B,Hq,Nq]: LSE = ln sum_j exp(scale * q_i . k_j)
+ *   B, Hq, Hkv, Nq, Nk   >= 1; Hq % Hkv == 0
+ *   d        head dimension, 64 or 128
+ *   scale    softmax scale (> 0, finite); callers normally pass 1/sqrt(d)
+ *   causal   0 or 1
+ *   dtype    FA_BF16 or FA_BF16_OUT_F32 (FA_E4M3 is rejected: use fa_fwd_fp8)
+ *   stream   CUDA stream of the current device
+ *
+ * Returns FA_OK once the kernel is enqueued; FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED
+ * with nothing enqueued; FA_ERR_CUDA if the launch failed.
+ */
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                 fa_dtype dtype, fa_stream_t stream);
+
+/*
+ * Fused attention forward, fp8 (OCP e4m3) inputs with per-(batch, head) scales, fp32
+ * accumulation, bf16 output.  FP8 on the tensor cores is the low-precision variant the
+ * page "FlashAttention-3 (DE)" describes (section "Neue Hardwarefaehigkeiten der
+ * Hopper-GPU (H100)", FP8 format).
+ *
+ * The real values are q = descale_q[b*Hq+hq] * e4m3(q8), k = descale_k[b*Hkv+hk] *
+ * e4m3(k8), v = descale_v[b*Hkv+hk] * e4m3(v8).  The descale arrays are fp32 device
+ * arrays of B*Hq, B*Hkv and B*Hkv entries.  The kernel rounds the softmax numerators P
+ * to e4m3 before the P.V product (values in [0, 256]).
+ *
+ *   d must be 128.  Other arguments as for fa_fwd; o is bf16 [B,Hq,Nq,d].
+ */
+fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                     int causal, const float *descale_q, const float *descale_k,
+                     const float *descale_v, fa_stream_t stream);
+
+/*
+ * Device-side failure report.  Every wait inside the kernels (on a shared-memory
+ * mbarrier filled by a TMA copy or a tensor-core commit) is bounded in time; a wait
+ * that runs out sets a device error word, makes the other warps of the CTA stop, drains
+ * the CTA's copies in flight, frees its tensor memory and returns.  The outputs of such
+ * a call are undefined.
+ *
+ * fa_check_device_error synchronises `stream`, reads and clears the error word of the
+ * current device and returns FA_ERR_TIMEOUT if it was set (FA_ERR_CUDA if the
+ * synchronisation itself failed), else FA_OK.
+ */
+fa_status fa_check_device_error(fa_stream_t stream);
+
+/* Static English description of a status code. */
+const char *fa_status_string(fa_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

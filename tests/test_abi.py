@@ -1,0 +1,96 @@
+"""The C-ABI library: it loads without a GPU, exports every entry point the header
+declares, keeps the oracle out of the product, and rejects invalid arguments on the host
+before any CUDA call (so these checks run on a CPU-only machine)."""
+import os
+import re
+
+import pytest
+
+import exact_attention_101_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa_b200.h")
+
+A = 0x10000          # a 16-byte-aligned fake address: never dereferenced by these calls
+OK_ARGS = dict(B=1, Hq=4, Hkv=2, Nq=256, Nk=256, d=128, scale=0.088, causal=0)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_builds_and_loads():
+    from exact_attention_101_b200 import build
+    assert os.path.exists(build.build())
+    assert fa.fa_version() == 100
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert set(names) == set(fa.C_SYMBOLS)
+    L = fa.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_product_does_not_reference_the_oracle():
+    L = fa.lib()
+    for sym in ("oracle_attention_rows", "oracle_decode_bf16"):
+        with pytest.raises(AttributeError):
+            getattr(L, sym)
+    pkg = os.path.join(ROOT, "exact_attention_101_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
+                assert "attn_oracle" not in src and "liboracle" not in src, f
+
+
+def call(**kw):
+    a = dict(OK_ARGS)
+    a.update(kw)
+    ptrs = dict(q=A, k=A, v=A, o=A, lse=A)
+    for p in list(ptrs):
+        if p in a:
+            ptrs[p] = a.pop(p)
+    dtype = a.pop("dtype", fa.FA_BF16)
+    return fa.fa_fwd(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["lse"], a["B"], a["Hq"],
+                     a["Hkv"], a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"], dtype, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=0), dict(k=0), dict(v=0), dict(o=0), dict(lse=0),
+    dict(q=A + 8), dict(o=A + 4), dict(lse=A + 2),
+    dict(B=0), dict(Hq=0), dict(Hkv=0), dict(Nq=0), dict(Nk=0), dict(d=0), dict(Nk=-5),
+    dict(Hq=3, Hkv=2), dict(causal=2), dict(scale=0.0), dict(scale=-1.0),
+    dict(scale=float("nan")), dict(scale=float("inf")), dict(dtype=fa.FA_E4M3), dict(dtype=7),
+    dict(B=1 << 20, Hq=1 << 12, Hkv=1 << 12),
+])
+def test_invalid_arguments(kw):
+    assert call(**kw) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d=96), dict(d=256), dict(d=32), dict(causal=1, Nq=256, Nk=512),
+])
+def test_unsupported_configurations(kw):
+    assert call(**kw) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_fp8_entry_validation():
+    args = (A, A, A, A, A, 1, 2, 2, 128, 128)
+    # missing descales
+    assert fa.fa_fwd_fp8(*args, 128, 0.1, 0, 0, A, A, None) == fa.FA_ERR_INVALID_ARG
+    # misaligned descale
+    assert fa.fa_fwd_fp8(*args, 128, 0.1, 0, A + 2, A, A, None) == fa.FA_ERR_INVALID_ARG
+    # fp8 supports d = 128 only
+    assert fa.fa_fwd_fp8(*args, 64, 0.1, 0, A, A, A, None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_status_strings():
+    for s in range(5):
+        assert fa.fa_status_string(s)
+    assert fa.fa_status_string(99) == "unknown status"
