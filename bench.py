@@ -201,7 +201,7 @@ def run_ours(args):
     import exact_attention_101_b200 as fa
 
     rank, local_rank, world = rank_env()
-    w = workloads.WORKLOADS[args.workload]
+    w = select_workload(args)
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
@@ -263,7 +263,7 @@ def run_ours(args):
 
     # End to end through the public API: pinned host inputs -> device, forward, O and LSE
     # back to pinned host memory, every step inside the timed region.
-    e2e_steps = max(3, min(args.steps, 20))
+    e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 20))
     hq_, hk_, hv_ = (t.pin_memory() for t in host)
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
@@ -281,23 +281,25 @@ def run_ours(args):
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
+    e2e = None
+    if e2e_steps:
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    h2d = sum(t.numel() * t.element_size() for t in host)
-    if fp8:
-        h2d += sum(t.numel() * t.element_size() for t in hds)
-    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-    e2e = {"value": w.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        h2d = sum(t.numel() * t.element_size() for t in host)
+        if fp8:
+            h2d += sum(t.numel() * t.element_size() for t in hds)
+        d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+        e2e = {"value": w.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     if world > 1:
         import torch.distributed as dist
@@ -333,7 +335,7 @@ def run_ours(args):
                      "kernel": "fa_fwd_kernel"},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps + 1 + e2e_steps,
         "clocks": clk,
     }
     print(json.dumps(line))
@@ -341,11 +343,25 @@ def run_ours(args):
 
 # ------------------------------------------------------------------ reference arm
 
+def select_workload(args):
+    """The named workload, optionally with fewer heads (a smaller case of the same
+    kernel for profiling); the query/KV head ratio is kept."""
+    import dataclasses
+    w = workloads.WORKLOADS[args.workload]
+    if args.heads:
+        g = w.Hq // w.Hkv
+        if args.heads % g:
+            raise SystemExit("--heads must be a multiple of %d for %s" % (g, w.name))
+        w = dataclasses.replace(w, name="%s_h%d" % (w.name, args.heads), Hq=args.heads,
+                                Hkv=args.heads // g)
+    return w
+
+
 def run_reference(args):
     rank, _, world = rank_env()
     if rank != 0:
         return
-    w = workloads.WORKLOADS[args.workload]
+    w = select_workload(args)
     inp = workloads.make_inputs(w)
     per_step = max(0.2, args.reference_budget_s / max(1, args.steps + args.warmup))
     for i in range(args.warmup):
@@ -383,6 +399,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="CPU time spent timing the oracle for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the number of query heads (smaller profiling case)")
     ap.add_argument("--reference-budget-s", type=float, default=120.0,
                     help="total CPU time of the reference arm")
     args = ap.parse_args(argv)

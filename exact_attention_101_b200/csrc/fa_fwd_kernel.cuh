@@ -396,7 +396,8 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
     // Last admissible key for this row (keys beyond Nk never count).
     const int key_lim = CAUSAL ? min(row, p.Nk - 1) : p.Nk - 1;
     float m_used = NEG_INF;  // running maximum in use, base-2 scaled domain
-    float l = 0.f;           // running sum of the numerators fed to the P V product
+    float l = 0.f;           // running sum of the numerators as rounded for the P V product
+    float l_exact = 0.f;     // running sum of the unrounded numerators (for the LSE)
 
     for (int j = 0; j < nx; ++j) {
       bool ok = wait_phase(bar.s_full(x), sph, abort_flag, ERR_WAIT_SOFTMAX);
@@ -449,12 +450,14 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       }
       if (resc) {
         l *= alpha;
+        l_exact *= alpha;
         m_used = xmax;
       }
       const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
 
       // Numerators p = 2^(s*sl2 - m_used), packed for the P V product.
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      float le[4] = {0.f, 0.f, 0.f, 0.f};
       if (!FP8) {
         uint32_t pk[4][16];
 #pragma unroll
@@ -466,8 +469,10 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
             const uint32_t pp = ptx::pack_bf16x2(p0, p1);
             const int col = c * 8 + e / 2;
             pk[col / 16][col % 16] = pp;
-            // l sums the same rounded values the tensor core multiplies with V.
+            // l sums the same rounded values the tensor core multiplies with V, so that O
+            // stays a convex combination of value rows; l_exact keeps the LSE accurate.
             ls[(e / 2) & 3] += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
+            le[(e / 2) & 3] += p0 + p1;
           }
 #pragma unroll
         for (int c = 0; c < 4; ++c) ptx::tmem_st16(t_p + c * 16, pk[c]);
@@ -483,18 +488,23 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
             const float p3 = ptx::ex2(fmaf(__uint_as_float(sr[c][e + 3]), sl2, neg_m));
             const int col = c * 4 + e / 4;
             pk[col / 16][col % 16] = ptx::pack_e4m3x4(p0, p1, p2, p3);
-            ls[(e / 4) & 3] += (p0 + p1) + (p2 + p3);
+            le[(e / 4) & 3] += (p0 + p1) + (p2 + p3);
           }
 #pragma unroll
         for (int c = 0; c < 2; ++c) ptx::tmem_st16(t_p + c * 16, pk[c]);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l_exact += (le[0] + le[1]) + (le[2] + le[3]);
+      if (FP8)
+        l = l_exact;
+      else
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.p_full(x));
     }
 
-    // Epilogue: O = O_acc / l (times the V descale for fp8), LSE = ln 2 * (m_used + log2 l).
+    // Epilogue: O = O_acc / l (times the V descale for fp8),
+    // LSE = ln 2 * (m_used + log2 l_exact).
     {
       bool ok = wait_phase(bar.o_full(x), unit_it & 1u, abort_flag, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;
@@ -536,7 +546,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
           }
         }
       }
-      if (valid) p.lse[orow] = (m_used + log2f(l)) * 0.69314718055994530942f;
+      if (valid) p.lse[orow] = (m_used + log2f(l_exact)) * 0.69314718055994530942f;
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.o_empty(x));
     }
