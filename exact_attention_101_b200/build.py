@@ -37,8 +37,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if all(os.path.getmtime(f) <= t for f in DEPS):
             return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [_nvcc()] + NVCC_FLAGS + ["-I", os.path.join(ROOT, "include"), "-I", CSRC,
-                                     "-o", tmp] + SOURCES
+    extra = os.environ.get("FA_NVCC_EXTRA", "").split()  # e.g. tuning -D overrides
+    cmd = [_nvcc()] + NVCC_FLAGS + extra + ["-I", os.path.join(ROOT, "include"), "-I", CSRC,
+                                             "-o", tmp] + SOURCES
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)

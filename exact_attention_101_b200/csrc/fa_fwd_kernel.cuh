@@ -14,7 +14,7 @@
 //
 //   warps 0-3  softmax + epilogue for Q tile 0 (one thread per query row)
 //   warps 4-7  softmax + epilogue for Q tile 1
-//   warp  8    tensor-memory allocator and single-thread tcgen05.mma issuer
+//   warp  8    tensor-memory allocator and tcgen05.mma issuer (warp-wide, elected lane)
 //   warp  9    single-thread TMA producer
 //   warps 10-11 idle (they complete the third warpgroup)
 //
@@ -66,12 +66,19 @@ constexpr int NUM_THREADS = 384;
 constexpr int MMA_WARP = 8;
 constexpr int TMA_WARP = 9;
 constexpr int LAUNCH_REGS = 168;    // 65536 / 384, rounded down to a multiple of 8
-constexpr int SOFTMAX_REGS = 200;
-constexpr int OTHER_REGS = 104;
+constexpr int SOFTMAX_REGS = 208;
+constexpr int OTHER_REGS = 88;
 static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch pool");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units: p <= 256
+#ifndef FA_EXP2_POLY_PAIRS
+#define FA_EXP2_POLY_PAIRS 0
+#endif
+// Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial on unmasked
+// tiles; the rest use the MUFU unit.
+constexpr int EXP2_POLY_PAIRS = FA_EXP2_POLY_PAIRS;
+static_assert(EXP2_POLY_PAIRS >= 0 && EXP2_POLY_PAIRS <= 8, "pairs per 16-column chunk");
 
 // Error bits written to the device error word when a bounded wait runs out.
 constexpr uint32_t ERR_WAIT_SOFTMAX = 1u << 0;
@@ -134,14 +141,14 @@ struct Unit {
   int n1;   // key tiles visited by Q tile 1 (>= n0)
 };
 
-// Work list: units of the last query block first (the longest under the causal mask),
-// heads in order inside a block so that query heads sharing a K/V head run side by side.
+// Work list: head-major, so that the CTAs running at the same time share the K/V of a
+// few heads in L2 (and query heads that share a K/V head are neighbours); inside a head
+// the query blocks run last-first, i.e. longest-first under the causal mask.
 template <bool CAUSAL>
 __device__ __forceinline__ Unit decode_unit(const FwdParams &p, int u) {
-  const int BH = p.B * p.Hq;
-  const int qb = p.num_qb - 1 - u / BH;
+  const int qb = p.num_qb - 1 - u % p.num_qb;
   Unit w;
-  w.bh = u % BH;
+  w.bh = u / p.num_qb;
   const int b = w.bh / p.Hq, hq = w.bh % p.Hq;
   w.bhk = b * p.Hkv + hq / p.group;
   w.r0 = qb * UNIT_ROWS;
@@ -258,117 +265,214 @@ drain:
 
 // ---------------------------------------------------------------------------- MMA issuer
 
+// The start-address field of a descriptor is bits [0,14) of (address >> 4); shared
+// memory addresses stay below 2^18, so advancing a descriptor by b bytes is adding b >> 4.
+// The issue loops below are fully unrolled with compile-time offsets and run on the whole
+// MMA warp (one elected lane issues): the tensor core then gets a new 128x128x16 MMA every
+// 64 cycles, which a loop with per-step descriptor arithmetic in one thread cannot sustain.
 template <int D, bool FP8>
-__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_saddr, uint32_t k_saddr) {
+__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
   using C = TileCfg<D, FP8>;
 #pragma unroll
   for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
-    const uint32_t kb = kk * C::MMA_K * C::ELEM;  // byte offset along the head dim
-    const uint32_t off = (kb / 128) * C::BOX_BYTES + (kb % 128);
-    const uint64_t a = ptx::smem_desc_sw128(q_saddr + off, 16, 1024);
-    const uint64_t b = ptx::smem_desc_sw128(k_saddr + off, 16, 1024);
+    constexpr uint32_t step = C::MMA_K * C::ELEM;  // bytes along the head dim per MMA
+    const uint32_t kb = kk * step;
+    const uint32_t off = ((kb / 128) * C::BOX_BYTES + (kb % 128)) >> 4;
     if (FP8)
-      ptx::mma_f8_ss(tmem_s, a, b, C::IDESC_S, kk > 0);
+      ptx::mma_f8_ss_elect(tmem_s, q_desc + off, k_desc + off, C::IDESC_S, kk > 0 ? 1u : 0u);
     else
-      ptx::mma_bf16_ss(tmem_s, a, b, C::IDESC_S, kk > 0);
+      ptx::mma_bf16_ss_elect(tmem_s, q_desc + off, k_desc + off, C::IDESC_S, kk > 0 ? 1u : 0u);
   }
 }
 
 template <int D, bool FP8>
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_saddr,
-                                         bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t v_desc,
+                                         uint32_t accumulate) {
   using C = TileCfg<D, FP8>;
+  // V is [keys x D] with D contiguous: MN-major B operand.  MMA_K key rows of 128 bytes
+  // per step; successive 128-byte D chunks are one TMA box apart (the LBO of v_desc).
 #pragma unroll
   for (int kk = 0; kk < C::PV_KSTEPS; ++kk) {
-    // V is [keys x D] with D contiguous: MN-major B operand.  MMA_K key rows of 128 bytes
-    // per step; successive 128-byte D chunks are one TMA box apart.
-    const uint64_t b = ptx::smem_desc_sw128(v_saddr + kk * C::MMA_K * 128, C::BOX_BYTES, 1024);
+    const uint32_t off = (kk * C::MMA_K * 128) >> 4;
     const uint32_t a = tmem_p + kk * 8;  // 8 TMEM columns hold MMA_K packed P values
+    const uint32_t acc = kk > 0 ? 1u : accumulate;
     if (FP8)
-      ptx::mma_f8_ts(tmem_o, a, b, C::IDESC_O, (accumulate || kk > 0) ? 1u : 0u);
+      ptx::mma_f8_ts_elect(tmem_o, a, v_desc + off, C::IDESC_O, acc);
     else
-      ptx::mma_bf16_ts(tmem_o, a, b, C::IDESC_O, (accumulate || kk > 0) ? 1u : 0u);
+      ptx::mma_bf16_ts_elect(tmem_o, a, v_desc + off, C::IDESC_O, acc);
   }
 }
 
+// Runs on all 32 lanes of the MMA warp; waits are polled by every lane and made
+// warp-uniform, MMAs and commits are issued by one elected lane.
 template <int D, bool CAUSAL, bool FP8>
 __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
                          const Bars<TileCfg<D, FP8>::NSLOT> &bar, uint32_t drain_bar,
                          volatile uint32_t *abort_flag) {
   using C = TileCfg<D, FP8>;
-  const uint32_t q_s[2] = {smem + C::Q_OFF, smem + C::Q_OFF + C::TILE_BYTES};
+  const uint64_t q_d[2] = {ptx::smem_desc_sw128(smem + C::Q_OFF, 16, 1024),
+                           ptx::smem_desc_sw128(smem + C::Q_OFF + C::TILE_BYTES, 16, 1024)};
+  const uint64_t k_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, 16, 1024);
+  const uint64_t v_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, C::BOX_BYTES, 1024);
+  constexpr uint32_t SLOT_STEP = C::TILE_BYTES >> 4;
   const uint32_t t_s[2] = {tmem + C::S_COL0, tmem + C::S_COL1};
   const uint32_t t_p[2] = {tmem + C::S_COL0 + C::P_OFF, tmem + C::S_COL1 + C::P_OFF};
   const uint32_t t_o[2] = {tmem + C::O_COL0, tmem + C::O_COL1};
   uint32_t kv_base = 0;
   uint32_t pph[2] = {0u, 0u};
   uint32_t unit_it = 0;
-  auto slot_addr = [&](uint32_t idx) { return smem + C::RING_OFF + (idx % C::NSLOT) * C::TILE_BYTES; };
-  auto wait_slot = [&](uint32_t idx) {
-    return wait_phase(bar.slot_full(idx % C::NSLOT), (idx / C::NSLOT) & 1u, abort_flag, ERR_WAIT_MMA);
+  auto wait = [&](uint32_t b, uint32_t parity) {
+    const bool ok = wait_phase(b, parity, abort_flag, ERR_WAIT_MMA);
+    return __all_sync(0xffffffffu, ok);
   };
+  auto wait_slot = [&](uint32_t idx) {
+    return wait(bar.slot_full(idx % C::NSLOT), (idx / C::NSLOT) & 1u);
+  };
+  auto kdesc = [&](uint32_t idx) { return k_d0 + (idx % C::NSLOT) * SLOT_STEP; };
+  auto vdesc = [&](uint32_t idx) { return v_d0 + (idx % C::NSLOT) * SLOT_STEP; };
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++unit_it) {
     const Unit w = decode_unit<CAUSAL>(p, u);
-    if (!wait_phase(bar.q_full(), unit_it & 1u, abort_flag, ERR_WAIT_MMA)) break;
+    if (!wait(bar.q_full(), unit_it & 1u)) break;
     if (!wait_slot(kv_base)) break;
     ptx::tc_fence_after();
-    issue_s<D, FP8>(t_s[0], q_s[0], slot_addr(kv_base));
-    ptx::mma_commit(bar.s_full(0));
-    issue_s<D, FP8>(t_s[1], q_s[1], slot_addr(kv_base));
-    ptx::mma_commit(bar.s_full(1));
-    ptx::mma_commit(bar.slot_empty(kv_base % C::NSLOT));
-    if (w.n1 == 1) ptx::mma_commit(bar.q_empty());
+    issue_s<D, FP8>(t_s[0], q_d[0], kdesc(kv_base));
+    ptx::mma_commit_elect(bar.s_full(0));
+    issue_s<D, FP8>(t_s[1], q_d[1], kdesc(kv_base));
+    ptx::mma_commit_elect(bar.s_full(1));
+    ptx::mma_commit_elect(bar.slot_empty(kv_base % C::NSLOT));
+    if (w.n1 == 1) ptx::mma_commit_elect(bar.q_empty());
     bool ok = true;
     for (int j = 0; j < w.n1 && ok; ++j) {
       const uint32_t vi = kv_base + 2 * j + 1;  // V_j
       const uint32_t ki = kv_base + 2 * j + 2;  // K_{j+1}
       const bool next = j + 1 < w.n1;
+      const uint32_t acc = j > 0 ? 1u : 0u;
       if (!wait_slot(vi)) { ok = false; break; }
       if (j < w.n0) {
-        if (!wait_phase(bar.p_full(0), pph[0], abort_flag, ERR_WAIT_MMA)) { ok = false; break; }
+        if (!wait(bar.p_full(0), pph[0])) { ok = false; break; }
         pph[0] ^= 1u;
-        if (j == 0 && !wait_phase(bar.o_empty(0), (unit_it & 1u) ^ 1u, abort_flag, ERR_WAIT_MMA)) {
-          ok = false;
-          break;
-        }
+        if (j == 0 && !wait(bar.o_empty(0), (unit_it & 1u) ^ 1u)) { ok = false; break; }
         ptx::tc_fence_after();
-        issue_pv<D, FP8>(t_o[0], t_p[0], slot_addr(vi), j > 0);
-        if (j == w.n0 - 1) ptx::mma_commit(bar.o_full(0));
+        issue_pv<D, FP8>(t_o[0], t_p[0], vdesc(vi), acc);
+        if (j == w.n0 - 1) ptx::mma_commit_elect(bar.o_full(0));
         if (j + 1 < w.n0) {
           if (!wait_slot(ki)) { ok = false; break; }
           ptx::tc_fence_after();
-          issue_s<D, FP8>(t_s[0], q_s[0], slot_addr(ki));
-          ptx::mma_commit(bar.s_full(0));
+          issue_s<D, FP8>(t_s[0], q_d[0], kdesc(ki));
+          ptx::mma_commit_elect(bar.s_full(0));
         }
       }
-      if (!wait_phase(bar.p_full(1), pph[1], abort_flag, ERR_WAIT_MMA)) { ok = false; break; }
+      if (!wait(bar.p_full(1), pph[1])) { ok = false; break; }
       pph[1] ^= 1u;
-      if (j == 0 && !wait_phase(bar.o_empty(1), (unit_it & 1u) ^ 1u, abort_flag, ERR_WAIT_MMA)) {
-        ok = false;
-        break;
-      }
+      if (j == 0 && !wait(bar.o_empty(1), (unit_it & 1u) ^ 1u)) { ok = false; break; }
       ptx::tc_fence_after();
-      issue_pv<D, FP8>(t_o[1], t_p[1], slot_addr(vi), j > 0);
-      ptx::mma_commit(bar.slot_empty(vi % C::NSLOT));
-      if (j == w.n1 - 1) ptx::mma_commit(bar.o_full(1));
+      issue_pv<D, FP8>(t_o[1], t_p[1], vdesc(vi), acc);
+      ptx::mma_commit_elect(bar.slot_empty(vi % C::NSLOT));
+      if (j == w.n1 - 1) ptx::mma_commit_elect(bar.o_full(1));
       if (next) {
         if (!wait_slot(ki)) { ok = false; break; }
         ptx::tc_fence_after();
-        issue_s<D, FP8>(t_s[1], q_s[1], slot_addr(ki));
-        ptx::mma_commit(bar.s_full(1));
-        ptx::mma_commit(bar.slot_empty(ki % C::NSLOT));
-        if (j + 1 == w.n1 - 1) ptx::mma_commit(bar.q_empty());
+        issue_s<D, FP8>(t_s[1], q_d[1], kdesc(ki));
+        ptx::mma_commit_elect(bar.s_full(1));
+        ptx::mma_commit_elect(bar.slot_empty(ki % C::NSLOT));
+        if (j + 1 == w.n1 - 1) ptx::mma_commit_elect(bar.q_empty());
       }
     }
     if (!ok) break;
     kv_base += 2 * w.n1;
   }
-  // Wait until every MMA issued by this thread has finished before TMEM is freed.
-  ptx::mma_commit(drain_bar);
+  // Wait until every MMA issued by this warp has finished before TMEM is freed.
+  ptx::mma_commit_elect(drain_bar);
   drain_wait(drain_bar, 0);
 }
 
 // ---------------------------------------------------------------------------- softmax
+
+// Software 2^x for a pair of arguments on the FMA pipe: j = round(x) through the
+// 1.5*2^23 addition trick, f = x - j in [-1/2, 1/2], 2^f from the minimax cubic fitted by
+// gen_exp2_poly.py (max relative error 7.5e-5, below bf16 and e4m3 rounding), and 2^j
+// applied by adding j to the exponent field.  Arguments are clamped at -126 so that the
+// exponent stays in range (the result is then below 2^-125, i.e. nothing next to the row
+// maximum's term >= 1).  This is the FMA-unit exponential of the page "FlashAttention 4:
+// Praxisleitfaden ...", section "Software-Exponentialfunktionen ueber CUDA-Kerne".
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
+  const float MAGIC = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = ptx::f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = ptx::f2_add(x, ptx::f2_pack(MAGIC, MAGIC));
+  const uint64_t jf = ptx::f2_add(t, ptx::f2_pack(-MAGIC, -MAGIC));
+  const uint64_t f = ptx::f2_fma(jf, ptx::f2_pack(-1.f, -1.f), x);
+  uint64_t q = ptx::f2_fma(f, ptx::f2_pack(5.517166853e-02f, 5.517166853e-02f),
+                           ptx::f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  q = ptx::f2_fma(q, f, ptx::f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  q = ptx::f2_fma(q, f, ptx::f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float t0, t1, q0, q1;
+  ptx::f2_unpack(t, t0, t1);
+  ptx::f2_unpack(q, q0, q1);
+  // low mantissa bits of t hold j (two's complement); shifting them into the exponent
+  // field and adding multiplies q by 2^j.
+  y0 = __uint_as_float(__float_as_uint(t0) * (1u << 23) + __float_as_uint(q0));
+  y1 = __uint_as_float(__float_as_uint(t1) * (1u << 23) + __float_as_uint(q1));
+}
+
+// One score row tile (128 columns, in sr) -> numerators in TMEM at t_p.  Adds the sum of
+// the numerators as rounded for the tensor core (bf16 only) to lr and of the unrounded
+// numerators to le.  NPOLY of every 8 column pairs use the polynomial exponential.
+template <bool FP8, int NPOLY>
+__device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[8][16], float sl2,
+                                                   float neg_m, uint32_t t_p, float &lr,
+                                                   float &le) {
+  const uint64_t scale2 = ptx::f2_pack(sl2, sl2);
+  const uint64_t bias2 = ptx::f2_pack(neg_m, neg_m);
+  uint64_t acc_r[2] = {0ull, 0ull};  // packed (0.f, 0.f)
+  uint64_t acc_e[2] = {0ull, 0ull};
+  uint32_t pk[FP8 ? 2 : 4][16];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float pv[16];
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const uint64_t xx = ptx::f2_fma(
+          ptx::f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, bias2);
+      float x0, x1;
+      ptx::f2_unpack(xx, x0, x1);
+      if ((e / 2) < NPOLY) {
+        exp2_poly_pair(x0, x1, pv[e], pv[e + 1]);
+      } else {
+        pv[e] = ptx::ex2(x0);
+        pv[e + 1] = ptx::ex2(x1);
+      }
+      acc_e[(e / 2) & 1] = ptx::f2_add(acc_e[(e / 2) & 1], ptx::f2_pack(pv[e], pv[e + 1]));
+    }
+    if (!FP8) {
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        const uint32_t pp = ptx::pack_bf16x2(pv[e], pv[e + 1]);
+        const int col = c * 8 + e / 2;
+        pk[col / 16][col % 16] = pp;
+        // sum of the rounded values the tensor core multiplies with V, so that O stays a
+        // convex combination of value rows
+        acc_r[(e / 2) & 1] = ptx::f2_add(
+            acc_r[(e / 2) & 1],
+            ptx::f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u)));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        const int col = c * 4 + e / 4;
+        pk[col / 16][col % 16] = ptx::pack_e4m3x4(pv[e], pv[e + 1], pv[e + 2], pv[e + 3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < (FP8 ? 2 : 4); ++c) ptx::tmem_st16(t_p + c * 16, pk[c]);
+  float a0, a1, b0, b1;
+  ptx::f2_unpack(ptx::f2_add(acc_e[0], acc_e[1]), a0, a1);
+  le += a0 + a1;
+  if (!FP8) {
+    ptx::f2_unpack(ptx::f2_add(acc_r[0], acc_r[1]), b0, b1);
+    lr += b0 + b1;
+  }
+}
 
 template <int D, bool CAUSAL, bool OUT_F32, bool FP8>
 __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
@@ -422,13 +526,20 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
           for (int e = 0; e < 16; ++e)
             if (c * 16 + e > lim) sr[c][e] = __float_as_uint(NEG_INF);
       }
-      // Row maximum (4 independent chains).
-      float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+      // Row maximum: 8 independent chains of three-input maxima.
+      float mx[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+      for (int c = 0; c < 8; ++c) {
+        float m = ptx::max3(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]),
+                            __uint_as_float(sr[c][2]));
 #pragma unroll
-        for (int e = 0; e < 16; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(sr[c][e]));
-      const float xmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+        for (int e = 3; e < 15; e += 2)
+          m = ptx::max3(m, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+        mx[c] = fmaxf(m, __uint_as_float(sr[c][15]));
+      }
+      const float xmax =
+          ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]),
+                    fmaxf(mx[6], mx[7])) * sl2;
 
       // Lazy rescale: move m_used only when the new maximum is far above it.
       const bool resc = xmax > m_used + RESCALE_THRESHOLD;
@@ -455,49 +566,19 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       }
       const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
 
-      // Numerators p = 2^(s*sl2 - m_used), packed for the P V product.
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      float le[4] = {0.f, 0.f, 0.f, 0.f};
-      if (!FP8) {
-        uint32_t pk[4][16];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[c][e]), sl2, neg_m));
-            const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m));
-            const uint32_t pp = ptx::pack_bf16x2(p0, p1);
-            const int col = c * 8 + e / 2;
-            pk[col / 16][col % 16] = pp;
-            // l sums the same rounded values the tensor core multiplies with V, so that O
-            // stays a convex combination of value rows; l_exact keeps the LSE accurate.
-            ls[(e / 2) & 3] += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
-            le[(e / 2) & 3] += p0 + p1;
-          }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_st16(t_p + c * 16, pk[c]);
-      } else {
-        uint32_t pk[2][16];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-#pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[c][e]), sl2, neg_m));
-            const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m));
-            const float p2 = ptx::ex2(fmaf(__uint_as_float(sr[c][e + 2]), sl2, neg_m));
-            const float p3 = ptx::ex2(fmaf(__uint_as_float(sr[c][e + 3]), sl2, neg_m));
-            const int col = c * 4 + e / 4;
-            pk[col / 16][col % 16] = ptx::pack_e4m3x4(p0, p1, p2, p3);
-            le[(e / 4) & 3] += (p0 + p1) + (p2 + p3);
-          }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) ptx::tmem_st16(t_p + c * 16, pk[c]);
-      }
-      l_exact += (le[0] + le[1]) + (le[2] + le[3]);
+      // Numerators p = 2^(s*sl2 - m_used), packed for the P V product.  Tiles without
+      // masked entries send EXP2_POLY_PAIRS of every 8 column pairs to the FMA-pipe
+      // polynomial and the rest to the MUFU unit.
+      float lr = 0.f, le = 0.f;
+      if (need_mask)
+        softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, lr, le);
+      else
+        softmax_numerators<FP8, EXP2_POLY_PAIRS>(sr, sl2, neg_m, t_p, lr, le);
+      l_exact += le;
       if (FP8)
         l = l_exact;
       else
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l += lr;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.p_full(x));
@@ -607,7 +688,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp < 8) {
     softmax_role<D, CAUSAL, OUT_F32, FP8>(p, tmem, bar, abort_flag);
   } else if (warp == MMA_WARP) {
-    if (lane == 0) mma_role<D, CAUSAL, FP8>(p, smem, tmem, bar, drain_bar, abort_flag);
+    mma_role<D, CAUSAL, FP8>(p, smem, tmem, bar, drain_bar, abort_flag);
     __syncwarp();
   } else if (warp == TMA_WARP) {
     if (lane == 0) load_role<D, CAUSAL, FP8>(&tmQ, &tmK, &tmV, p, smem, bar, abort_flag);
