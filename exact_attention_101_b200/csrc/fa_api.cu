@@ -99,14 +99,14 @@ bool buffer_ok(const void *p, size_t bytes, int dev) {
   return end <= static_cast<uint64_t>(base) + size;
 }
 
-// 3-D tensor map over a [heads, rows, d] tensor, box = [1, 128, box_inner], 128-byte
-// swizzle, out-of-bounds elements read as zero.
+// 3-D tensor map over a [heads, rows, d] tensor, box = [1, box_rows, 128 bytes of d],
+// 128-byte swizzle, out-of-bounds elements read as zero.
 bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_t rows,
-                 uint64_t heads) {
+                 uint64_t heads, uint32_t box_rows) {
   const uint64_t eb = fp8 ? 1 : 2;
   cuuint64_t dims[3] = {d, rows, heads};
   cuuint64_t strides[2] = {d * eb, rows * d * eb};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 128, 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = driver_fns().encode(
       m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
@@ -205,9 +205,9 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
     return FA_ERR_INVALID_ARG;
 
   CUtensorMap tq, tk, tv;
-  if (!encode_tmap(&tq, q, fp8, d, Nq, static_cast<uint64_t>(B) * Hq) ||
-      !encode_tmap(&tk, k, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv) ||
-      !encode_tmap(&tv, v, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv))
+  if (!encode_tmap(&tq, q, fp8, d, Nq, static_cast<uint64_t>(B) * Hq, fa::BM) ||
+      !encode_tmap(&tk, k, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::BN) ||
+      !encode_tmap(&tv, v, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::BN))
     return FA_ERR_INVALID_ARG;
 
   fa::FwdParams p;

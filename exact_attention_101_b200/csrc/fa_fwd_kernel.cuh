@@ -2,50 +2,63 @@
 //
 // One persistent CTA per SM walks a static list of work units.  A unit is 256 query
 // rows (two 128-row Q tiles) of one (batch, query head); the two tiles share every K/V
-// tile that is streamed through shared memory, and their softmax work alternates with
-// the tensor core's work on the other tile.  The method is the IO-aware tiled attention
-// of the page "FlashAttention (DE)" (sections "Tiling und blockweise Verarbeitung",
-// "Online-Softmax-Berechnung", "Zusammenfassen von Operationen in einem CUDA-Kernel"):
-// S = Q K^T, the mask, the online softmax and O += P V all happen on chip; only O and
-// the per-row log-sum-exp are written.  The warp roles follow the idea of a
+// tile that is streamed through shared memory.  The method is the IO-aware tiled
+// attention of the page "FlashAttention (DE)" (sections "Tiling und blockweise
+// Verarbeitung", "Online-Softmax-Berechnung", "Zusammenfassen von Operationen in einem
+// CUDA-Kernel"): S = Q K^T, the mask, the online softmax and O += P V all happen on chip;
+// only O and the per-row log-sum-exp are written.  The warp roles follow the idea of a
 // warp-specialised pipeline (page "FlashAttention 4: Praxisleitfaden ...", section "Was
 // ist neu in FlashAttention 4?": loading, MMA, softmax, rescaling, epilogue), mapped
 // onto sm_100a as follows:
 //
-//   warps 0-3  softmax + epilogue for Q tile 0 (one thread per query row)
-//   warps 4-7  softmax + epilogue for Q tile 1
-//   warp  8    tensor-memory allocator and tcgen05.mma issuer (warp-wide, elected lane)
-//   warp  9    single-thread TMA producer
-//   warps 10-11 idle (they complete the third warpgroup)
+//   warps 0-3   softmax + epilogue for Q tile 0 (one thread per query row)
+//   warps 4-7   softmax + epilogue for Q tile 1
+//   warp  8     tensor-memory allocator; tcgen05.mma issuer for Q tile 0
+//   warp  9     TMA producer (one lane)
+//   warp  10    tcgen05.mma issuer for Q tile 1
+//   warp  11    idle (it completes the third warpgroup)
 //
-// Registers: the kernel is launched with LAUNCH_REGS per thread (384 threads); the
-// third warpgroup gives registers back (setmaxnreg.dec to OTHER_REGS) and the two
-// softmax warpgroups take them (setmaxnreg.inc to SOFTMAX_REGS), so that a whole score
-// row (128 fp32 values) stays in registers.  256*SOFTMAX_REGS + 128*OTHER_REGS equals
-// the launch pool 384*LAUNCH_REGS; the host refuses to launch a build whose register
-// count would make that sum exceed the pool.
+// Key tiles are BN = 64 keys, and every Q tile has TWO score buffers in tensor memory:
+// while the softmax warps of a tile turn S(j) into P(j), the tensor core already
+// computes S(j+1) (and S(j+2) as soon as P(j) has been consumed).  So a tile's softmax
+// never waits for its own P.V product, and the two tiles' softmax warps -- one of each per
+// SM sub-partition -- can both be busy at once.  This matters on B200 because, at head
+// dim 128, the exponentials of one score tile take the SFU as long as the tensor core
+// takes for that tile's two products.
 //
-// Tensor memory (512 columns x 128 lanes x 32 bit):
-//   [  0,128) S0 (fp32 scores of tile 0); P0 (bf16/e4m3 numerators) aliases [64,128)
-//   [128,256) S1; P1 aliases [192,256)
-//   [256,256+D) O0 accumulator, [256+D, 256+2D) O1 accumulator
+// Tensor memory (512 columns x 128 lanes x 32 bit), BN = 64:
+//   S(x, b) at x*128 + b*64, 64 fp32 columns (tile x, buffer b); the numerators P of
+//   that buffer (bf16 pairs or e4m3 quads packed in 32-bit columns) overwrite its upper
+//   32 columns; O_x accumulator at 256 + x*D.
 //
-// Shared memory: Q0, Q1 tiles and a ring of NSLOT K/V tile slots, all in the 128-byte
-// swizzled layout that TMA writes and the tensor core reads; plus the mbarriers.
+// Registers: the kernel is launched with LAUNCH_REGS per thread (384 threads); the third
+// warpgroup gives registers back (setmaxnreg.dec to OTHER_REGS) and the two softmax
+// warpgroups take them (setmaxnreg.inc to SOFTMAX_REGS).  256*SOFTMAX_REGS +
+// 128*OTHER_REGS stays within the launch pool 384*LAUNCH_REGS; the host refuses to launch
+// a build whose register count would make that sum exceed the pool.
+//
+// Shared memory: Q0, Q1 (128-row tiles) and a ring of NSLOT 64-row K/V tiles, all in the
+// 128-byte swizzled layout that TMA writes and the tensor core reads; the mbarriers.
 //
 // Synchronisation (all mbarriers):
 //   q_full / q_empty        Q tiles of a unit loaded / no longer read by an MMA
 //   slot_full / slot_empty  ring slot loaded (TMA tx bytes) / released by an MMA commit
-//   s_full[x]               S_x of the current key tile is in TMEM
-//   p_full[x]               P_x written to TMEM by the 128 softmax threads of tile x
+//   s_full[x][b]            S(x, b) computed
+//   p_full[x][b]            P(x, b) written by the 128 softmax threads of tile x
+//   pv_done[x]              one P.V product of tile x finished (for the rare rescale)
 //   o_full[x] / o_empty[x]  O_x final for the unit / read out by the epilogue
+//
+// MMA order of tile x inside a unit (j = key tile): S(x, 0), S(x, 1), then for every j
+// PV(x, j), S(x, j+2).  S(x, j+2) reuses the buffer of P(x, j) and is issued after
+// PV(x, j) by the same thread: tcgen05 operations from one thread run in issue order, so
+// the product reads P before the next scores overwrite it.
 //
 // Softmax details.  Scores are moved into the base-2 domain with one FFMA,
 // x = s * (scale * log2 e), and p = 2^(x - m_used).  m_used is only raised when a key
 // tile's row maximum exceeds it by more than RESCALE_THRESHOLD (lazy rescaling, page
 // "FlashAttention 4: Praxisleitfaden ...", section "Intelligenteres Online-Softmax-
-// Rescaling in FA4"), so p <= 2^RESCALE_THRESHOLD and the accumulator O and the sum l
-// are multiplied by 2^(m_old - m_new) only then.  The causal mask is applied only on key
+// Rescaling in FA4"), so p <= 2^RESCALE_THRESHOLD and the accumulator O and the sums are
+// multiplied by 2^(m_old - m_new) only then.  The causal mask is applied only on key
 // tiles that cross the diagonal; tiles entirely above it are never loaded.
 #pragma once
 
@@ -60,14 +73,18 @@ namespace fa {
 // ---------------------------------------------------------------------------- config
 
 constexpr int BM = 128;               // query rows per Q tile (MMA M)
-constexpr int BN = 128;               // keys per K/V tile (MMA N of S = Q K^T)
+constexpr int BN = 64;                // keys per K/V tile (MMA N of S = Q K^T)
 constexpr int UNIT_ROWS = 2 * BM;     // query rows per work unit
 constexpr int NUM_THREADS = 384;
 constexpr int MMA_WARP = 8;
 constexpr int TMA_WARP = 9;
 constexpr int LAUNCH_REGS = 168;    // 65536 / 384, rounded down to a multiple of 8
-constexpr int SOFTMAX_REGS = 208;
-constexpr int OTHER_REGS = 88;
+#ifndef FA_SOFTMAX_REGS
+#define FA_SOFTMAX_REGS 184
+#endif
+constexpr int SOFTMAX_REGS = FA_SOFTMAX_REGS;
+constexpr int OTHER_REGS = (NUM_THREADS * LAUNCH_REGS - 256 * SOFTMAX_REGS) / 128 / 8 * 8;
+static_assert(OTHER_REGS >= 64, "register split leaves too few for the MMA/TMA warps");
 static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch pool");
 constexpr uint32_t TMEM_COLS = 512;
@@ -96,9 +113,12 @@ struct TileCfg {
   static_assert(ROW_BYTES % 128 == 0, "tile rows must be whole 128-byte swizzle rows");
   static constexpr int NBOX = ROW_BYTES / 128;       // 128-byte-wide TMA boxes per row
   static constexpr int BOX_ELEMS = 128 / ELEM;       // elements per box row
-  static constexpr int BOX_BYTES = 128 * 128;        // 128 rows x 128 bytes
-  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
-  static constexpr int NSLOT = TILE_BYTES == 32768 ? 4 : 8;
+  static constexpr int Q_BOX_BYTES = BM * 128;       // 128 rows x 128 bytes
+  static constexpr int KV_BOX_BYTES = BN * 128;      // 64 rows x 128 bytes
+  static constexpr int Q_TILE_BYTES = NBOX * Q_BOX_BYTES;
+  static constexpr int KV_TILE_BYTES = NBOX * KV_BOX_BYTES;
+  static constexpr int NSLOT = 131072 / KV_TILE_BYTES;  // 128 KB ring: 8 or 16 slots
+  static_assert((NSLOT & (NSLOT - 1)) == 0, "ring size must be a power of two");
   static constexpr int MMA_K = FP8 ? 32 : 16;        // K extent of one MMA instruction
   static constexpr int S_KSTEPS = D / MMA_K;         // MMAs per S = Q K^T
   static constexpr int PV_KSTEPS = BN / MMA_K;       // MMAs per O += P V
@@ -106,19 +126,21 @@ struct TileCfg {
   static constexpr uint32_t IDESC_S = ptx::make_idesc(AB_FORMAT, BM, BN, 0);
   static constexpr uint32_t IDESC_O = ptx::make_idesc(AB_FORMAT, BM, D, 1);
   // TMEM column map.
-  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
-  static constexpr uint32_t P_OFF = 64;
+  static constexpr uint32_t P_OFF = 32;                  // P inside a 64-column S buffer
   static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
   static_assert(256 + 2 * D <= (int)TMEM_COLS, "TMEM budget");
   // Shared memory map (offsets from a 1024-aligned base).
   static constexpr int Q_OFF = 0;
-  static constexpr int RING_OFF = 2 * TILE_BYTES;
-  static constexpr int BAR_OFF = RING_OFF + NSLOT * TILE_BYTES;
-  static constexpr int NUM_BARS = 2 * NSLOT + 11;   // + drain barrier
+  static constexpr int RING_OFF = 2 * Q_TILE_BYTES;
+  static constexpr int BAR_OFF = RING_OFF + NSLOT * KV_TILE_BYTES;
+  static constexpr int NUM_BARS = 2 * NSLOT + 18;
   static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
+
+// TMEM column of score buffer b of Q tile x.
+__host__ __device__ constexpr uint32_t s_col(int x, int b) { return x * 128 + b * 64; }
 
 struct FwdParams {
   void *o;
@@ -168,7 +190,7 @@ __device__ unsigned int g_fa_error = 0;
 // Bounded wait on an mbarrier phase.  Returns false if another warp of the CTA aborted or
 // if this wait ran out (then it raises the CTA abort flag and the device error word).
 __device__ __forceinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity,
-                                             volatile uint32_t *abort_flag, uint32_t who) {
+                                                volatile uint32_t *abort_flag, uint32_t who) {
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1; it < WAIT_MAX_ITERS; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
@@ -207,10 +229,12 @@ struct Bars {
   __device__ uint32_t slot_empty(int s) const { return base + 8u * (NSLOT + s); }
   __device__ uint32_t q_full() const { return base + 8u * (2 * NSLOT + 0); }
   __device__ uint32_t q_empty() const { return base + 8u * (2 * NSLOT + 1); }
-  __device__ uint32_t s_full(int x) const { return base + 8u * (2 * NSLOT + 2 + x); }
-  __device__ uint32_t p_full(int x) const { return base + 8u * (2 * NSLOT + 4 + x); }
-  __device__ uint32_t o_full(int x) const { return base + 8u * (2 * NSLOT + 6 + x); }
-  __device__ uint32_t o_empty(int x) const { return base + 8u * (2 * NSLOT + 8 + x); }
+  __device__ uint32_t s_full(int x, int b) const { return base + 8u * (2 * NSLOT + 2 + 2 * x + b); }
+  __device__ uint32_t p_full(int x, int b) const { return base + 8u * (2 * NSLOT + 6 + 2 * x + b); }
+  __device__ uint32_t pv_done(int x) const { return base + 8u * (2 * NSLOT + 10 + x); }
+  __device__ uint32_t o_full(int x) const { return base + 8u * (2 * NSLOT + 12 + x); }
+  __device__ uint32_t o_empty(int x) const { return base + 8u * (2 * NSLOT + 14 + x); }
+  __device__ uint32_t drain(int x) const { return base + 8u * (2 * NSLOT + 16 + x); }
 };
 
 // ---------------------------------------------------------------------------- producer
@@ -228,12 +252,12 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
     const Unit w = decode_unit<CAUSAL>(p, u);
     if (!wait_phase(bar.q_empty(), (q_issued & 1u) ^ 1u, abort_flag, ERR_WAIT_LOAD)) goto drain;
-    ptx::mbar_arrive_expect_tx(bar.q_full(), 2 * C::TILE_BYTES);
+    ptx::mbar_arrive_expect_tx(bar.q_full(), 2 * C::Q_TILE_BYTES);
 #pragma unroll
     for (int x = 0; x < 2; ++x)
 #pragma unroll
       for (int bx = 0; bx < C::NBOX; ++bx)
-        ptx::tma_load_3d(smem + C::Q_OFF + x * C::TILE_BYTES + bx * C::BOX_BYTES, tmQ,
+        ptx::tma_load_3d(smem + C::Q_OFF + x * C::Q_TILE_BYTES + bx * C::Q_BOX_BYTES, tmQ,
                          bar.q_full(), bx * C::BOX_ELEMS, w.r0 + x * BM, w.bh);
     ++q_issued;
     for (int j = 0; j < w.n1; ++j) {
@@ -242,10 +266,10 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
         const int s = issued % C::NSLOT;
         const uint32_t ph = (issued / C::NSLOT) & 1u;
         if (!wait_phase(bar.slot_empty(s), ph ^ 1u, abort_flag, ERR_WAIT_LOAD)) goto drain;
-        ptx::mbar_arrive_expect_tx(bar.slot_full(s), C::TILE_BYTES);
+        ptx::mbar_arrive_expect_tx(bar.slot_full(s), C::KV_TILE_BYTES);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
-          ptx::tma_load_3d(smem + C::RING_OFF + s * C::TILE_BYTES + bx * C::BOX_BYTES,
+          ptx::tma_load_3d(smem + C::RING_OFF + s * C::KV_TILE_BYTES + bx * C::KV_BOX_BYTES,
                            t ? tmV : tmK, bar.slot_full(s), bx * C::BOX_ELEMS, j * BN, w.bhk);
         ++issued;
       }
@@ -268,8 +292,8 @@ drain:
 // The start-address field of a descriptor is bits [0,14) of (address >> 4); shared
 // memory addresses stay below 2^18, so advancing a descriptor by b bytes is adding b >> 4.
 // The issue loops below are fully unrolled with compile-time offsets and run on the whole
-// MMA warp (one elected lane issues): the tensor core then gets a new 128x128x16 MMA every
-// 64 cycles, which a loop with per-step descriptor arithmetic in one thread cannot sustain.
+// MMA warp (one elected lane issues): the tensor core then gets a new MMA every few
+// cycles, which a loop with per-step descriptor arithmetic in one thread cannot sustain.
 template <int D, bool FP8>
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
   using C = TileCfg<D, FP8>;
@@ -277,11 +301,12 @@ __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t q_desc, uint64
   for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
     constexpr uint32_t step = C::MMA_K * C::ELEM;  // bytes along the head dim per MMA
     const uint32_t kb = kk * step;
-    const uint32_t off = ((kb / 128) * C::BOX_BYTES + (kb % 128)) >> 4;
+    const uint32_t qoff = ((kb / 128) * C::Q_BOX_BYTES + (kb % 128)) >> 4;
+    const uint32_t koff = ((kb / 128) * C::KV_BOX_BYTES + (kb % 128)) >> 4;
     if (FP8)
-      ptx::mma_f8_ss_elect(tmem_s, q_desc + off, k_desc + off, C::IDESC_S, kk > 0 ? 1u : 0u);
+      ptx::mma_f8_ss_elect(tmem_s, q_desc + qoff, k_desc + koff, C::IDESC_S, kk > 0 ? 1u : 0u);
     else
-      ptx::mma_bf16_ss_elect(tmem_s, q_desc + off, k_desc + off, C::IDESC_S, kk > 0 ? 1u : 0u);
+      ptx::mma_bf16_ss_elect(tmem_s, q_desc + qoff, k_desc + koff, C::IDESC_S, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -303,23 +328,26 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint6
   }
 }
 
-// Runs on all 32 lanes of the MMA warp; waits are polled by every lane and made
-// warp-uniform, MMAs and commits are issued by one elected lane.
+// One MMA warp per Q tile x (warp 8 for tile 0, warp 10 for tile 1), so that each tile's
+// chain P(x, j) -> PV(x, j) -> S(x, j+2) waits only for its own softmax warps while the
+// other warp keeps the tensor core busy.  Runs on all 32 lanes of the warp; waits are
+// polled by every lane and made warp-uniform, MMAs and commits are issued by one elected
+// lane.  K/V ring slots and the Q tiles are shared by the two tiles: each is released by
+// two arrivals, one per tile.  Key tiles that only tile 1 visits (causal) get tile 0's
+// arrival from tile 1's warp as a plain arrive; it happens only after the slot's load has
+// landed, so it can never complete the slot's previous phase early.
 template <int D, bool CAUSAL, bool FP8>
 __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
-                         const Bars<TileCfg<D, FP8>::NSLOT> &bar, uint32_t drain_bar,
+                         const Bars<TileCfg<D, FP8>::NSLOT> &bar, const int x,
                          volatile uint32_t *abort_flag) {
   using C = TileCfg<D, FP8>;
-  const uint64_t q_d[2] = {ptx::smem_desc_sw128(smem + C::Q_OFF, 16, 1024),
-                           ptx::smem_desc_sw128(smem + C::Q_OFF + C::TILE_BYTES, 16, 1024)};
+  const uint64_t q_d = ptx::smem_desc_sw128(smem + C::Q_OFF + x * C::Q_TILE_BYTES, 16, 1024);
   const uint64_t k_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, 16, 1024);
-  const uint64_t v_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, C::BOX_BYTES, 1024);
-  constexpr uint32_t SLOT_STEP = C::TILE_BYTES >> 4;
-  const uint32_t t_s[2] = {tmem + C::S_COL0, tmem + C::S_COL1};
-  const uint32_t t_p[2] = {tmem + C::S_COL0 + C::P_OFF, tmem + C::S_COL1 + C::P_OFF};
-  const uint32_t t_o[2] = {tmem + C::O_COL0, tmem + C::O_COL1};
+  const uint64_t v_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, C::KV_BOX_BYTES, 1024);
+  constexpr uint32_t SLOT_STEP = C::KV_TILE_BYTES >> 4;
+  const uint32_t t_o = tmem + (x ? C::O_COL1 : C::O_COL0);
   uint32_t kv_base = 0;
-  uint32_t pph[2] = {0u, 0u};
+  uint32_t pph = 0;  // phase bits of p_full(x, b), bit b
   uint32_t unit_it = 0;
   auto wait = [&](uint32_t b, uint32_t parity) {
     const bool ok = wait_phase(b, parity, abort_flag, ERR_WAIT_MMA);
@@ -328,62 +356,53 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
   auto wait_slot = [&](uint32_t idx) {
     return wait(bar.slot_full(idx % C::NSLOT), (idx / C::NSLOT) & 1u);
   };
-  auto kdesc = [&](uint32_t idx) { return k_d0 + (idx % C::NSLOT) * SLOT_STEP; };
-  auto vdesc = [&](uint32_t idx) { return v_d0 + (idx % C::NSLOT) * SLOT_STEP; };
+  // Release ring slot idx for this tile (and for tile 0 if tile 0 does not visit it).
+  auto release = [&](uint32_t idx, bool also_tile0) {
+    ptx::mma_commit_elect(bar.slot_empty(idx % C::NSLOT));
+    if (also_tile0) ptx::mbar_arrive_elect(bar.slot_empty(idx % C::NSLOT));
+  };
+  auto scores = [&](const Unit &w, int nx, int j, uint32_t ki) {
+    issue_s<D, FP8>(tmem + s_col(x, j & 1), q_d, k_d0 + (ki % C::NSLOT) * SLOT_STEP);
+    ptx::mma_commit_elect(bar.s_full(x, j & 1));
+    release(ki, x == 1 && j >= w.n0);
+    if (j == nx - 1) ptx::mma_commit_elect(bar.q_empty());
+  };
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++unit_it) {
     const Unit w = decode_unit<CAUSAL>(p, u);
+    const int nx = x ? w.n1 : w.n0;
     if (!wait(bar.q_full(), unit_it & 1u)) break;
-    if (!wait_slot(kv_base)) break;
-    ptx::tc_fence_after();
-    issue_s<D, FP8>(t_s[0], q_d[0], kdesc(kv_base));
-    ptx::mma_commit_elect(bar.s_full(0));
-    issue_s<D, FP8>(t_s[1], q_d[1], kdesc(kv_base));
-    ptx::mma_commit_elect(bar.s_full(1));
-    ptx::mma_commit_elect(bar.slot_empty(kv_base % C::NSLOT));
-    if (w.n1 == 1) ptx::mma_commit_elect(bar.q_empty());
     bool ok = true;
-    for (int j = 0; j < w.n1 && ok; ++j) {
-      const uint32_t vi = kv_base + 2 * j + 1;  // V_j
-      const uint32_t ki = kv_base + 2 * j + 2;  // K_{j+1}
-      const bool next = j + 1 < w.n1;
-      const uint32_t acc = j > 0 ? 1u : 0u;
-      if (!wait_slot(vi)) { ok = false; break; }
-      if (j < w.n0) {
-        if (!wait(bar.p_full(0), pph[0])) { ok = false; break; }
-        pph[0] ^= 1u;
-        if (j == 0 && !wait(bar.o_empty(0), (unit_it & 1u) ^ 1u)) { ok = false; break; }
-        ptx::tc_fence_after();
-        issue_pv<D, FP8>(t_o[0], t_p[0], vdesc(vi), acc);
-        if (j == w.n0 - 1) ptx::mma_commit_elect(bar.o_full(0));
-        if (j + 1 < w.n0) {
-          if (!wait_slot(ki)) { ok = false; break; }
-          ptx::tc_fence_after();
-          issue_s<D, FP8>(t_s[0], q_d[0], kdesc(ki));
-          ptx::mma_commit_elect(bar.s_full(0));
-        }
-      }
-      if (!wait(bar.p_full(1), pph[1])) { ok = false; break; }
-      pph[1] ^= 1u;
-      if (j == 0 && !wait(bar.o_empty(1), (unit_it & 1u) ^ 1u)) { ok = false; break; }
+    for (int j = 0; j < 2 && j < nx; ++j) {
+      if (!wait_slot(kv_base + 2 * j)) { ok = false; break; }
       ptx::tc_fence_after();
-      issue_pv<D, FP8>(t_o[1], t_p[1], vdesc(vi), acc);
-      ptx::mma_commit_elect(bar.slot_empty(vi % C::NSLOT));
-      if (j == w.n1 - 1) ptx::mma_commit_elect(bar.o_full(1));
-      if (next) {
+      scores(w, nx, j, kv_base + 2 * j);
+    }
+    for (int j = 0; j < nx && ok; ++j) {
+      const int b = j & 1;
+      const uint32_t vi = kv_base + 2 * j + 1;    // V_j
+      if (!wait_slot(vi)) { ok = false; break; }
+      if (!wait(bar.p_full(x, b), (pph >> b) & 1u)) { ok = false; break; }
+      pph ^= 1u << b;
+      if (j == 0 && !wait(bar.o_empty(x), (unit_it & 1u) ^ 1u)) { ok = false; break; }
+      ptx::tc_fence_after();
+      issue_pv<D, FP8>(t_o, tmem + s_col(x, b) + C::P_OFF, v_d0 + (vi % C::NSLOT) * SLOT_STEP,
+                       j > 0 ? 1u : 0u);
+      ptx::mma_commit_elect(bar.pv_done(x));
+      release(vi, x == 1 && j >= w.n0);
+      if (j == nx - 1) ptx::mma_commit_elect(bar.o_full(x));
+      if (j + 2 < nx) {
+        const uint32_t ki = kv_base + 2 * (j + 2);  // K_{j+2}
         if (!wait_slot(ki)) { ok = false; break; }
         ptx::tc_fence_after();
-        issue_s<D, FP8>(t_s[1], q_d[1], kdesc(ki));
-        ptx::mma_commit_elect(bar.s_full(1));
-        ptx::mma_commit_elect(bar.slot_empty(ki % C::NSLOT));
-        if (j + 1 == w.n1 - 1) ptx::mma_commit_elect(bar.q_empty());
+        scores(w, nx, j + 2, ki);
       }
     }
     if (!ok) break;
     kv_base += 2 * w.n1;
   }
   // Wait until every MMA issued by this warp has finished before TMEM is freed.
-  ptx::mma_commit_elect(drain_bar);
-  drain_wait(drain_bar, 0);
+  ptx::mma_commit_elect(bar.drain(x));
+  drain_wait(bar.drain(x), 0);
 }
 
 // ---------------------------------------------------------------------------- softmax
@@ -414,28 +433,32 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, fl
   y1 = __uint_as_float(__float_as_uint(t1) * (1u << 23) + __float_as_uint(q1));
 }
 
-// One score row tile (128 columns, in sr) -> numerators in TMEM at t_p.  Adds the sum of
-// the numerators as rounded for the tensor core (bf16 only) to lr and of the unrounded
+// One 64-column score row (sr) -> numerators in TMEM at t_p.  Adds the sum of the
+// numerators as rounded for the tensor core (bf16 only) to lr and of the unrounded
 // numerators to le.  NPOLY of every 8 column pairs use the polynomial exponential.
+// Numerators are packed and stored to TMEM 32 columns at a time (64 for e4m3).
 template <bool FP8, int NPOLY>
-__device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[8][16], float sl2,
+__device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], float sl2,
                                                    float neg_m, uint32_t t_p, float &lr,
                                                    float &le) {
   const uint64_t scale2 = ptx::f2_pack(sl2, sl2);
   const uint64_t bias2 = ptx::f2_pack(neg_m, neg_m);
   uint64_t acc_r[2] = {0ull, 0ull};  // packed (0.f, 0.f)
   uint64_t acc_e[2] = {0ull, 0ull};
-  uint32_t pk[FP8 ? 2 : 4][16];
+  constexpr int SCOLS = FP8 ? 64 : 32;  // score columns per 16-column TMEM store
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    float pv[16];
+  for (int q = 0; q < 64 / SCOLS; ++q) {
+    uint32_t pk[16];
+    float pv[SCOLS];
 #pragma unroll
-    for (int e = 0; e < 16; e += 2) {
-      const uint64_t xx = ptx::f2_fma(
-          ptx::f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, bias2);
+    for (int e = 0; e < SCOLS; e += 2) {
+      const int col = q * SCOLS + e;
+      const uint64_t xx = ptx::f2_fma(ptx::f2_pack(__uint_as_float(sr[col / 16][col % 16]),
+                                                   __uint_as_float(sr[col / 16][col % 16 + 1])),
+                                      scale2, bias2);
       float x0, x1;
       ptx::f2_unpack(xx, x0, x1);
-      if ((e / 2) < NPOLY) {
+      if (((col % 16) / 2) < NPOLY) {
         exp2_poly_pair(x0, x1, pv[e], pv[e + 1]);
       } else {
         pv[e] = ptx::ex2(x0);
@@ -445,10 +468,9 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[8][16], 
     }
     if (!FP8) {
 #pragma unroll
-      for (int e = 0; e < 16; e += 2) {
+      for (int e = 0; e < SCOLS; e += 2) {
         const uint32_t pp = ptx::pack_bf16x2(pv[e], pv[e + 1]);
-        const int col = c * 8 + e / 2;
-        pk[col / 16][col % 16] = pp;
+        pk[e / 2] = pp;
         // sum of the rounded values the tensor core multiplies with V, so that O stays a
         // convex combination of value rows
         acc_r[(e / 2) & 1] = ptx::f2_add(
@@ -457,14 +479,11 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[8][16], 
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < 16; e += 4) {
-        const int col = c * 4 + e / 4;
-        pk[col / 16][col % 16] = ptx::pack_e4m3x4(pv[e], pv[e + 1], pv[e + 2], pv[e + 3]);
-      }
+      for (int e = 0; e < SCOLS; e += 4)
+        pk[e / 4] = ptx::pack_e4m3x4(pv[e], pv[e + 1], pv[e + 2], pv[e + 3]);
     }
+    ptx::tmem_st16(t_p + q * 16, pk);
   }
-#pragma unroll
-  for (int c = 0; c < (FP8 ? 2 : 4); ++c) ptx::tmem_st16(t_p + c * 16, pk[c]);
   float a0, a1, b0, b1;
   ptx::f2_unpack(ptx::f2_add(acc_e[0], acc_e[1]), a0, a1);
   le += a0 + a1;
@@ -474,6 +493,10 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[8][16], 
   }
 }
 
+// Softmax warps: warpgroup x (warps 4x..4x+3) handles Q tile x, one thread per query row
+// (TMEM lane).  Every 64-key score tile is loaded whole into registers, masked if it
+// crosses the diagonal or the end of the keys, turned into numerators in place, and the
+// row statistics are carried from tile to tile.
 template <int D, bool CAUSAL, bool OUT_F32, bool FP8>
 __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
                              volatile uint32_t *abort_flag) {
@@ -483,11 +506,10 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
   const int wq = warp % 4;             // TMEM lane quarter of this warp
   const int row_in_tile = wq * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-  const uint32_t t_s = tmem + lane_base + (x ? C::S_COL1 : C::S_COL0);
-  const uint32_t t_p = t_s + C::P_OFF;
   const uint32_t t_o = tmem + lane_base + (x ? C::O_COL1 : C::O_COL0);
   const float NEG_INF = -__int_as_float(0x7f800000);
-  uint32_t sph = 0;
+  uint32_t sph = 0;      // phase bits of s_full(x, b), bit b
+  uint32_t pv_base = 0;  // P.V products of this tile in earlier units
   uint32_t unit_it = 0;
 
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++unit_it) {
@@ -504,32 +526,34 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
     float l_exact = 0.f;     // running sum of the unrounded numerators (for the LSE)
 
     for (int j = 0; j < nx; ++j) {
-      bool ok = wait_phase(bar.s_full(x), sph, abort_flag, ERR_WAIT_SOFTMAX);
+      const int b = j & 1;
+      bool ok = wait_phase(bar.s_full(x, b), (sph >> b) & 1u, abort_flag, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;
-      sph ^= 1u;
+      sph ^= 1u << b;
       ptx::tc_fence_after();
 
-      uint32_t sr[8][16];
+      const uint32_t t_s = tmem + lane_base + s_col(x, b);
+      uint32_t sr[4][16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) ptx::tmem_ld16(t_s + c * 16, sr[c]);
+      for (int c = 0; c < 4; ++c) ptx::tmem_ld16(t_s + c * 16, sr[c]);
       ptx::tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 8; ++c) ptx::reg_fence16(sr[c]);
+      for (int c = 0; c < 4; ++c) ptx::reg_fence16(sr[c]);
 
       const int kv0 = j * BN;
       const bool need_mask = (CAUSAL && kv0 + BN - 1 > tile_row0) || (kv0 + BN > p.Nk);
       if (need_mask) {
         const int lim = key_lim - kv0;  // column c is admissible iff c <= lim
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             if (c * 16 + e > lim) sr[c][e] = __float_as_uint(NEG_INF);
       }
-      // Row maximum: 8 independent chains of three-input maxima.
-      float mx[8];
+      // Row maximum: 4 independent chains of three-input maxima.
+      float mx[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         float m = ptx::max3(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]),
                             __uint_as_float(sr[c][2]));
 #pragma unroll
@@ -537,16 +561,18 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
           m = ptx::max3(m, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
         mx[c] = fmaxf(m, __uint_as_float(sr[c][15]));
       }
-      const float xmax =
-          ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]),
-                    fmaxf(mx[6], mx[7])) * sl2;
+      const float xmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
 
       // Lazy rescale: move m_used only when the new maximum is far above it.
       const bool resc = xmax > m_used + RESCALE_THRESHOLD;
       const float alpha = resc ? ptx::ex2(m_used - xmax) : 1.f;  // 0 on the first tile
       if (__any_sync(0xffffffffu, resc && j > 0)) {
-        // O_x is quiescent here: the commit that signalled S_x(j) covers the MMA that
-        // accumulated P_x(j-1) V(j-1), and P_x(j) V(j) waits for p_full below.
+        // The accumulator must be quiescent: wait for P(j-1) V(j-1) of this tile (the
+        // earlier products are covered by the commit that signalled S(j)); P(j) V(j) waits
+        // for p_full below.
+        ok = wait_phase(bar.pv_done(x), (pv_base + j - 1) & 1u, abort_flag, ERR_WAIT_SOFTMAX);
+        if (!__all_sync(0xffffffffu, ok)) return;
+        ptx::tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 16; ++c) {
           uint32_t o[16];
@@ -557,7 +583,6 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
           for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           ptx::tmem_st16(t_o + c * 16, o);
         }
-        ptx::tmem_wait_st();
       }
       if (resc) {
         l *= alpha;
@@ -570,6 +595,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       // masked entries send EXP2_POLY_PAIRS of every 8 column pairs to the FMA-pipe
       // polynomial and the rest to the MUFU unit.
       float lr = 0.f, le = 0.f;
+      const uint32_t t_p = t_s + C::P_OFF;
       if (need_mask)
         softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, lr, le);
       else
@@ -581,8 +607,9 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
         l += lr;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar.p_full(x));
+      ptx::mbar_arrive(bar.p_full(x, b));
     }
+    pv_base += nx;
 
     // Epilogue: O = O_acc / l (times the V descale for fp8),
     // LSE = ln 2 * (m_used + log2 l_exact).
@@ -596,12 +623,12 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       const size_t orow = static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[16], b[16];
+        uint32_t a[16], bb[16];
         ptx::tmem_ld16(t_o + c * 32, a);
-        ptx::tmem_ld16(t_o + c * 32 + 16, b);
+        ptx::tmem_ld16(t_o + c * 32 + 16, bb);
         ptx::tmem_wait_ld();
         ptx::reg_fence16(a);
-        ptx::reg_fence16(b);
+        ptx::reg_fence16(bb);
         if (valid) {
           if (OUT_F32) {
             float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + c * 32);
@@ -611,8 +638,8 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
                                    __uint_as_float(a[4 * v + 2]) * inv, __uint_as_float(a[4 * v + 3]) * inv);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
-              dst[4 + v] = make_float4(__uint_as_float(b[4 * v]) * inv, __uint_as_float(b[4 * v + 1]) * inv,
-                                       __uint_as_float(b[4 * v + 2]) * inv, __uint_as_float(b[4 * v + 3]) * inv);
+              dst[4 + v] = make_float4(__uint_as_float(bb[4 * v]) * inv, __uint_as_float(bb[4 * v + 1]) * inv,
+                                       __uint_as_float(bb[4 * v + 2]) * inv, __uint_as_float(bb[4 * v + 3]) * inv);
           } else {
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + c * 32);
             uint32_t h[16];
@@ -621,7 +648,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
               h[e] = ptx::pack_bf16x2(__uint_as_float(a[2 * e]) * inv, __uint_as_float(a[2 * e + 1]) * inv);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              h[8 + e] = ptx::pack_bf16x2(__uint_as_float(b[2 * e]) * inv, __uint_as_float(b[2 * e + 1]) * inv);
+              h[8 + e] = ptx::pack_bf16x2(__uint_as_float(bb[2 * e]) * inv, __uint_as_float(bb[2 * e + 1]) * inv);
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
           }
@@ -646,7 +673,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t smem = (raw + 1023u) & ~1023u;  // 1024-aligned for 128-byte swizzle
   uint8_t *smem_gen = smem_raw + (smem - raw);
   const Bars<C::NSLOT> bar{smem + C::BAR_OFF};
-  const uint32_t drain_bar = smem + C::BAR_OFF + 8u * (C::NUM_BARS - 1);
   uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + C::CTL_OFF);
   volatile uint32_t *tmem_slot = ctl;
   volatile uint32_t *abort_flag = ctl + 1;
@@ -657,17 +683,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
       ptx::mbar_init(bar.slot_full(s), 1);
-      ptx::mbar_init(bar.slot_empty(s), 1);
+      ptx::mbar_init(bar.slot_empty(s), 2);   // one arrival per Q tile
     }
     ptx::mbar_init(bar.q_full(), 1);
-    ptx::mbar_init(bar.q_empty(), 1);
+    ptx::mbar_init(bar.q_empty(), 2);
     for (int x = 0; x < 2; ++x) {
-      ptx::mbar_init(bar.s_full(x), 1);
-      ptx::mbar_init(bar.p_full(x), BM);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(bar.s_full(x, b), 1);
+        ptx::mbar_init(bar.p_full(x, b), BM);
+      }
+      ptx::mbar_init(bar.pv_done(x), 1);
       ptx::mbar_init(bar.o_full(x), 1);
       ptx::mbar_init(bar.o_empty(x), BM);
     }
-    ptx::mbar_init(drain_bar, 1);
+    ptx::mbar_init(bar.drain(0), 1);
+    ptx::mbar_init(bar.drain(1), 1);
     *abort_flag = 0u;
     ptx::fence_mbar_init();
   }
@@ -687,8 +717,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp < 8) {
     softmax_role<D, CAUSAL, OUT_F32, FP8>(p, tmem, bar, abort_flag);
-  } else if (warp == MMA_WARP) {
-    mma_role<D, CAUSAL, FP8>(p, smem, tmem, bar, drain_bar, abort_flag);
+  } else if (warp == MMA_WARP || warp == MMA_WARP + 2) {
+    mma_role<D, CAUSAL, FP8>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, abort_flag);
     __syncwarp();
   } else if (warp == TMA_WARP) {
     if (lane == 0) load_role<D, CAUSAL, FP8>(&tmQ, &tmK, &tmV, p, smem, bar, abort_flag);

@@ -258,6 +258,15 @@ __device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
       : "memory");
 }
 
+// Plain (immediate) arrive on `bar` by one elected lane of the warp.
+__device__ __forceinline__ void mbar_arrive_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread has
 // completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
