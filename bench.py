@@ -162,36 +162,59 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def oracle_sample_rate(w, inp, target_s, seed=0):
-    """Time the fp64 oracle on a random sample of query rows of the workload.  Returns
-    (TFLOP/s, description, threads, rows, seconds)."""
+def _oracle_kwargs(inp):
+    if inp.descale_q is None:
+        return {}
+    return dict(descale_q=inp.descale_q.double(), descale_k=inp.descale_k.double(),
+                descale_v=inp.descale_v.double())
+
+
+def _row_flops(w, rows):
+    i = rows % w.N
+    keys = (i + 1) if w.causal else (i * 0 + w.N)
+    return float(4.0 * w.d * keys.sum())
+
+
+def oracle_calibrate(w, inp, target_s, seed=0):
+    """Number of random query rows the fp64 oracle processes in about target_s seconds."""
     import numpy as np
     import oracle
     rng = np.random.default_rng(seed)
     total_rows = w.B * w.Hq * w.N
-
-    def row_flops(rows):
-        i = rows % w.N
-        keys = (i + 1) if w.causal else np.full_like(i, w.N)
-        return float(4.0 * w.d * keys.sum())
-
-    kw = {}
-    if inp.descale_q is not None:
-        kw = dict(descale_q=inp.descale_q.double(), descale_k=inp.descale_k.double(),
-                  descale_v=inp.descale_v.double())
     n = 16
     while True:
         rows = rng.integers(0, total_rows, size=n)
         t0 = time.perf_counter()
-        oracle.attention_rows(inp.q, inp.k, inp.v, w.scale, w.causal, rows=rows, **kw)
+        oracle.attention_rows(inp.q, inp.k, inp.v, w.scale, w.causal, rows=rows,
+                              **_oracle_kwargs(inp))
         dt = time.perf_counter() - t0
-        if dt >= target_s or n >= total_rows:
-            break
-        n = int(min(total_rows, max(2 * n, n * target_s / max(dt, 1e-3) * 1.1)))
-    fl = row_flops(rows)
-    desc = ("%d random query rows (of %d) of workload %s, full key range per row, fp64"
-            % (n, total_rows, w.name))
-    return fl / dt / 1e12, desc, oracle.max_threads(), n, dt
+        if dt >= 0.5 * target_s or n >= total_rows:
+            return int(min(total_rows, max(16, n * target_s / max(dt, 1e-4))))
+        n = int(min(total_rows, 4 * n))
+
+
+def oracle_timed_sample(w, inp, n_rows, seed=0):
+    """Time the fp64 oracle on n_rows random query rows of the workload.  Returns
+    (TFLOP/s, description, threads, seconds)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    total_rows = w.B * w.Hq * w.N
+    rows = rng.integers(0, total_rows, size=n_rows)
+    t0 = time.perf_counter()
+    oracle.attention_rows(inp.q, inp.k, inp.v, w.scale, w.causal, rows=rows,
+                          **_oracle_kwargs(inp))
+    dt = time.perf_counter() - t0
+    desc = ("%d random query rows (of %d) of workload %s, each over its full admissible key "
+            "range, fp64" % (n_rows, total_rows, w.name))
+    return _row_flops(w, rows) / dt / 1e12, desc, oracle.max_threads(), dt
+
+
+def oracle_sample_rate(w, inp, target_s, seed=0):
+    """Calibrate, then time one sample of about target_s seconds."""
+    n = oracle_calibrate(w, inp, target_s, seed)
+    rate, desc, cores, dt = oracle_timed_sample(w, inp, n, seed + 1)
+    return rate, desc, cores, n, dt
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -363,13 +386,14 @@ def run_reference(args):
         return
     w = select_workload(args)
     inp = workloads.make_inputs(w)
-    per_step = max(0.2, args.reference_budget_s / max(1, args.steps + args.warmup))
+    per_step = max(0.05, args.reference_budget_s / max(1, args.steps + args.warmup))
+    n_rows = oracle_calibrate(w, inp, per_step)
     for i in range(args.warmup):
-        oracle_sample_rate(w, inp, per_step, seed=100 + i)
+        oracle_timed_sample(w, inp, n_rows, seed=100 + i)
     rates, descs, total_s = [], [], 0.0
     cores = 1
     for i in range(args.steps):
-        rate, desc, cores, _, dt = oracle_sample_rate(w, inp, per_step, seed=i)
+        rate, desc, cores, dt = oracle_timed_sample(w, inp, n_rows, seed=i)
         rates.append(rate)
         descs.append(desc)
         total_s += dt

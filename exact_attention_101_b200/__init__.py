@@ -20,7 +20,8 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
-C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_check_device_error", "fa_status_string", "fa_version")
+C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_check_device_error", "fa_selftest_bounded_wait",
+             "fa_status_string", "fa_version")
 
 _lib = None
 
@@ -46,6 +47,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
         L.fa_check_device_error.restype = i
         L.fa_check_device_error.argtypes = [vp]
+        L.fa_selftest_bounded_wait.restype = i
+        L.fa_selftest_bounded_wait.argtypes = [i, vp]
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_status_string.argtypes = [i]
         L.fa_version.restype = i
@@ -70,6 +73,12 @@ def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
 
 def fa_check_device_error(stream) -> int:
     return lib().fa_check_device_error(stream)
+
+
+def fa_selftest_bounded_wait(timeout_us, stream) -> int:
+    """Raw ``fa_selftest_bounded_wait``: a wait that nothing completes runs out after
+    timeout_us; the next fa_check_device_error reports FA_ERR_TIMEOUT."""
+    return lib().fa_selftest_bounded_wait(int(timeout_us), stream)
 
 
 def fa_status_string(status: int) -> str:

@@ -279,6 +279,13 @@ fa_status fa_check_device_error(fa_stream_t stream) {
   return FA_OK;
 }
 
+fa_status fa_selftest_bounded_wait(int timeout_us, fa_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return FA_ERR_INVALID_ARG;
+  fa::fa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 const char *fa_status_string(fa_status s) {
   switch (s) {
     case FA_OK: return "success";

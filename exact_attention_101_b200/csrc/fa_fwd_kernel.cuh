@@ -102,6 +102,7 @@ constexpr uint32_t ERR_WAIT_SOFTMAX = 1u << 0;
 constexpr uint32_t ERR_WAIT_MMA = 1u << 1;
 constexpr uint32_t ERR_WAIT_LOAD = 1u << 2;
 constexpr uint32_t ERR_WAIT_DRAIN = 1u << 3;
+constexpr uint32_t ERR_WAIT_SELFTEST = 1u << 4;
 
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait
 constexpr uint32_t WAIT_MAX_ITERS = 1u << 28;
@@ -190,13 +191,14 @@ __device__ unsigned int g_fa_error = 0;
 // Bounded wait on an mbarrier phase.  Returns false if another warp of the CTA aborted or
 // if this wait ran out (then it raises the CTA abort flag and the device error word).
 __device__ __forceinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity,
-                                                volatile uint32_t *abort_flag, uint32_t who) {
+                                                volatile uint32_t *abort_flag, uint32_t who,
+                                                uint64_t limit_ns = WAIT_LIMIT_NS) {
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1; it < WAIT_MAX_ITERS; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (ptx::globaltimer_ns() - t0 > WAIT_LIMIT_NS) break;
+      if (ptx::globaltimer_ns() - t0 > limit_ns) break;
     }
   }
   *abort_flag = 1u;
@@ -731,6 +733,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
   }
+}
+
+// Self-test of the bounded wait: one warp waits on the first phase of an mbarrier that
+// nothing ever arrives on, with a limit of limit_ns.  The wait runs out, raises
+// ERR_WAIT_SELFTEST in the device error word and the kernel returns normally.
+__global__ void __launch_bounds__(32, 1) fa_selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_word;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_addr(&bar), 1);
+    abort_word = 0u;
+    ptx::fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = wait_phase_slow(ptx::smem_addr(&bar), 0u, &abort_word, ERR_WAIT_SELFTEST,
+                                  limit_ns);
+  __syncwarp();
+  (void)ok;
 }
 
 }  // namespace fa

@@ -111,6 +111,16 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
  */
 fa_status fa_check_device_error(fa_stream_t stream);
 
+/*
+ * Self-test of the failure path above, without faulting anything: launches one warp that
+ * waits on a shared-memory mbarrier nothing ever arrives on, with a limit of timeout_us
+ * microseconds (1 .. 1000000).  The wait runs out, the kernel records the time-out in the
+ * device error word and returns; the next fa_check_device_error(stream) reports
+ * FA_ERR_TIMEOUT and clears the word.  Returns FA_OK once launched, FA_ERR_INVALID_ARG
+ * for an out-of-range timeout, FA_ERR_CUDA if the launch failed.
+ */
+fa_status fa_selftest_bounded_wait(int timeout_us, fa_stream_t stream);
+
 /* Static English description of a status code. */
 const char *fa_status_string(fa_status s);
 

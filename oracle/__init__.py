@@ -23,26 +23,29 @@ F64, BF16, E4M3 = 0, 1, 2
 _lib = None
 
 
+def _bind(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    lib.oracle_attention_rows.restype = ctypes.c_int
+    lib.oracle_attention_rows.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int]
+    lib.oracle_decode_bf16.restype = ctypes.c_double
+    lib.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
+    lib.oracle_decode_e4m3.restype = ctypes.c_double
+    lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
+    lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_max_threads.argtypes = []
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        path = _build.build()
-        lib = ctypes.CDLL(path)
-        lib.oracle_attention_rows.restype = ctypes.c_int
-        lib.oracle_attention_rows.argtypes = [
-            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
-            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-            ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
-            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
-            ctypes.c_int]
-        lib.oracle_decode_bf16.restype = ctypes.c_double
-        lib.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
-        lib.oracle_decode_e4m3.restype = ctypes.c_double
-        lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
-        lib.oracle_max_threads.restype = ctypes.c_int
-        lib.oracle_max_threads.argtypes = []
-        _lib = lib
+        _lib = _bind(ctypes.CDLL(_build.build()))
     return _lib
 
 
@@ -75,7 +78,7 @@ def max_threads() -> int:
 
 
 def attention_rows(q, k, v, scale, causal=False, rows=None, descale_q=None,
-                   descale_k=None, descale_v=None, nthreads=0):
+                   descale_k=None, descale_v=None, nthreads=0, _library=None):
     """Exact attention for selected query rows.
 
     q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] -- float64 values, bf16 bit patterns or
@@ -105,7 +108,7 @@ def attention_rows(q, k, v, scale, causal=False, rows=None, descale_q=None,
     for arr in (descale_q, descale_k, descale_v):
         ds.append(None if arr is None else
                   np.ascontiguousarray(np.asarray(_as_numpy(arr), dtype=np.float64).reshape(-1)))
-    rc = _load().oracle_attention_rows(
+    rc = (_library or _load()).oracle_attention_rows(
         qa.ctypes.data, ka.ctypes.data, va.ctypes.data, et,
         None if ds[0] is None else ds[0].ctypes.data,
         None if ds[1] is None else ds[1].ctypes.data,
@@ -125,9 +128,15 @@ def attention(q, k, v, scale, causal=False, **kw):
     return o.reshape(B, Hq, Nq, d), lse.reshape(B, Hq, Nq)
 
 
-def decode_bf16(bits: int) -> float:
-    return float(_load().oracle_decode_bf16(int(bits)))
+def decode_bf16(bits: int, _library=None) -> float:
+    return float((_library or _load()).oracle_decode_bf16(int(bits)))
 
 
-def decode_e4m3(code: int) -> float:
-    return float(_load().oracle_decode_e4m3(int(code)))
+def decode_e4m3(code: int, _library=None) -> float:
+    return float((_library or _load()).oracle_decode_e4m3(int(code)))
+
+
+def load_library(path):
+    """Load another build of the oracle source (the tests use this to check that their
+    pins catch deliberately broken copies)."""
+    return _bind(ctypes.CDLL(path))

@@ -94,3 +94,8 @@ def test_status_strings():
     for s in range(5):
         assert fa.fa_status_string(s)
     assert fa.fa_status_string(99) == "unknown status"
+
+
+def test_selftest_rejects_out_of_range_timeout():
+    assert fa.fa_selftest_bounded_wait(0, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_selftest_bounded_wait(2000000, None) == fa.FA_ERR_INVALID_ARG
