@@ -3,13 +3,16 @@
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
 may import this package.  The CUDA library never uses it, and the two share no code.
 
-The arithmetic lives in ``attn_oracle.c`` (plain C, IEEE binary64): for every requested
+The attention arithmetic lives in ``attn_oracle.c`` (plain C, IEEE binary64): for every requested
 query row it materialises the full score row ``s_j = scale * q.k_j`` over the admissible
 keys, takes its maximum ``m``, forms ``p_j = exp(s_j - m)``, ``l = sum_j p_j`` and
 returns ``O = sum_j p_j v_j / l`` and ``LSE = m + ln l``.  That is the attention formula
 ``softmax(Q K^T / sqrt(d_k)) V`` of the page "FlashAttention (DE)", section
 "Problematik der Standard-Attention", which the pages say FlashAttention reproduces
-exactly.  This module only marshals arrays into that library.
+exactly.  ``quant_oracle.c`` holds the per-head e4m3 quantisation with the random-sign
+Hadamard rotation of the page "FlashAttention-3 (DE)", section "Niedrige Praezision
+(FP8) mit reduziertem Quantisierungsfehler".  This module only marshals arrays into that
+library.
 """
 import ctypes
 import os
@@ -39,6 +42,14 @@ def _bind(lib):
     lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
     lib.oracle_max_threads.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
+    lib.oracle_hadamard.restype = ctypes.c_int
+    lib.oracle_hadamard.argtypes = [ctypes.c_int64, ctypes.c_void_p]
+    lib.oracle_encode_e4m3.restype = ctypes.c_uint8
+    lib.oracle_encode_e4m3.argtypes = [ctypes.c_double]
+    lib.oracle_quantize_e4m3.restype = ctypes.c_int
+    lib.oracle_quantize_e4m3.argtypes = [
+        ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return lib
 
 
@@ -134,6 +145,45 @@ def decode_bf16(bits: int, _library=None) -> float:
 
 def decode_e4m3(code: int, _library=None) -> float:
     return float((_library or _load()).oracle_decode_e4m3(int(code)))
+
+
+def hadamard(d: int, _library=None) -> np.ndarray:
+    """Sylvester's Hadamard matrix of order d (a power of two) as float64 [d, d]."""
+    out = np.empty((d, d), dtype=np.float64)
+    if (_library or _load()).oracle_hadamard(int(d), out.ctypes.data) != 0:
+        raise ValueError("d must be a power of two >= 1, got %r" % (d,))
+    return out
+
+
+def encode_e4m3(value: float, _library=None) -> int:
+    """Nearest finite OCP e4m3 code (ties to even, saturating at 448)."""
+    return int((_library or _load()).oracle_encode_e4m3(float(value)))
+
+
+def quantize_e4m3(x, signs=None, nthreads=0, _library=None):
+    """Per-(batch, head) e4m3 quantisation of x [B, H, N, d] (float64 or bf16 bits),
+    after the rotation y = x diag(signs) H / sqrt(d) when ``signs`` (d values of +1/-1)
+    is given.  Returns (codes uint8 [B, H, N, d], descale float64 [B*H],
+    y float64 [B, H, N, d])."""
+    xa = np.ascontiguousarray(_as_numpy(x))
+    et = _elem_type(xa)
+    if et == E4M3:
+        raise TypeError("quantize_e4m3 takes float64 or bf16 input")
+    B, H, N, d = xa.shape
+    sa = None
+    if signs is not None:
+        sa = np.ascontiguousarray(np.asarray(_as_numpy(signs)).astype(np.int8).reshape(-1))
+        if sa.size != d:
+            raise ValueError("signs must have d entries")
+    codes = np.empty(xa.shape, dtype=np.uint8)
+    descale = np.empty((B * H,), dtype=np.float64)
+    y = np.empty(xa.shape, dtype=np.float64)
+    rc = (_library or _load()).oracle_quantize_e4m3(
+        xa.ctypes.data, et, None if sa is None else sa.ctypes.data, B * H, N, d,
+        codes.ctypes.data, descale.ctypes.data, y.ctypes.data, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_quantize_e4m3 failed with code %d" % rc)
+    return codes, descale, y
 
 
 def load_library(path):

@@ -1,6 +1,7 @@
 """Build the fp64 CPU oracle (test infrastructure) as a shared library.
 
-Compiles ``attn_oracle.c`` with gcc and OpenMP into ``oracle/liboracle.so``.  Only the
+Compiles ``attn_oracle.c`` (attention) and ``quant_oracle.c`` (fp8 quantisation with
+incoherent processing) with gcc and OpenMP into ``oracle/liboracle.so``.  Only the
 tests, the smoke check and the CPU-baseline leg of ``bench.py`` load that library.
 """
 import os
@@ -8,18 +9,25 @@ import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "attn_oracle.c")
+QUANT_SRC = os.path.join(HERE, "quant_oracle.c")
+SOURCES = (SRC, QUANT_SRC)
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+def compile_library(out: str, sources, opt: str = "-O2") -> None:
+    """gcc the given oracle sources into the shared library ``out``."""
+    cmd = ["gcc", opt, "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra",
+           "-o", out] + list(sources) + ["-lm"]
+    subprocess.run(cmd, check=True)
+
+
 def build(force: bool = False) -> str:
-    """Compile the oracle if the library is missing or older than its source."""
+    """Compile the oracle if the library is missing or older than one of its sources."""
     if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
+            and all(os.path.getmtime(LIB) >= os.path.getmtime(s) for s in SOURCES)):
         return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
-           "-Wall", "-Wextra", "-o", tmp, SRC, "-lm"]
-    subprocess.run(cmd, check=True)
+    compile_library(tmp, SOURCES)
     os.replace(tmp, LIB)
     return LIB
 

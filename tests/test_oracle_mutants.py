@@ -1,19 +1,20 @@
 """The pins are not vacuous: each plausible mistake, planted in a copy of the oracle's C
-source (a dropped term, a wrong sign or index, a transposed operand, a wrong log base, a
-mis-decoded format), makes at least one pin fail, while the real oracle passes them all.
-The mistakes are planted on the CPU only, in temporary builds."""
+sources (a dropped term, a wrong sign or index, a transposed operand, a wrong log base, a
+mis-decoded format, a wrong rounding tie rule or scale), makes at least one pin fail,
+while the real oracle passes them all.  The mistakes are planted on the CPU only, in
+temporary builds."""
 import math
 import os
-import subprocess
 
 import numpy as np
 import pytest
+import scipy.linalg
 import torch
 
 import oracle
 from oracle import build as oracle_build
 
-SRC = oracle_build.SRC
+SOURCES = oracle_build.SOURCES
 
 
 def rnd(shape, seed, scale=1.0):
@@ -85,7 +86,54 @@ def pin_e4m3_descales(lib):
     assert np.abs(o1 - o2).max() < 1e-12 and np.abs(l1 - l2).max() < 1e-12
 
 
-PINS = [pin_sdpa, pin_bruteforce_lse, pin_gqa, pin_decoders, pin_e4m3_descales]
+def _signs(d, seed):
+    return np.where(np.random.default_rng(seed).random(d) < 0.5, -1, 1).astype(np.int8)
+
+
+def pin_hadamard_scipy(lib):
+    assert np.array_equal(oracle.hadamard(16, _library=lib), scipy.linalg.hadamard(16))
+
+
+def pin_encoder_torch(lib):
+    vals = torch.arange(0, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    probes = np.concatenate([vals, (vals[:-1] + vals[1:]) / 2, [500.0]]).astype(np.float32)
+    probes = np.concatenate([probes[:-1], -probes[:-1]])
+    ref = torch.from_numpy(probes).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = [oracle.encode_e4m3(float(v), _library=lib) for v in probes]
+    assert np.array_equal(got, ref) and oracle.encode_e4m3(500.0, _library=lib) == 0x7E
+
+
+def pin_rotation_basis_and_norm(lib):
+    d, s = 32, _signs(32, 20)
+    h = scipy.linalg.hadamard(d)
+    x = np.zeros((1, 1, 2, d))
+    x[0, 0, 0, 5] = 1.0
+    x[0, 0, 1] = np.random.default_rng(21).standard_normal(d)
+    _, _, y = oracle.quantize_e4m3(x, s, _library=lib)
+    assert np.allclose(y[0, 0, 0], s[5] * h[5] / math.sqrt(d), atol=1e-15, rtol=0)
+    assert abs(np.linalg.norm(y[0, 0, 1]) - np.linalg.norm(x[0, 0, 1])) < 1e-12
+
+
+def pin_quantise_rounding_bound(lib):
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal((1, 2, 8, 32))
+    x[0, 0, 3, 4] = 40.0
+    x[0, 1] *= -3.0
+    x[0, 1, 2, 7] = -60.0
+    codes, descale, y = oracle.quantize_e4m3(x, _signs(32, 23), _library=lib)
+    u = y / descale.reshape(1, 2, 1, 1)
+    deq = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    half = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(u), 2.0 ** -6))) - 4)
+    assert (np.abs(deq - u) <= half * (1 + 1e-12)).all()
+    assert np.allclose(descale, np.abs(y).reshape(2, -1).max(axis=1) / 448.0, rtol=1e-15)
+    assert (np.abs(deq).reshape(2, -1).max(axis=1) == 448.0).all()
+    z, dz, _ = oracle.quantize_e4m3(np.zeros((1, 1, 2, 32)), None, _library=lib)
+    assert dz[0] == 1.0 and not z.any()
+
+
+PINS = [pin_sdpa, pin_bruteforce_lse, pin_gqa, pin_decoders, pin_e4m3_descales,
+        pin_hadamard_scipy, pin_encoder_torch, pin_rotation_basis_and_norm,
+        pin_quantise_rounding_bound]
 
 MUTANTS = {
     "scale_dropped": ("srow[j] = scale * dot;", "srow[j] = dot;"),
@@ -107,17 +155,36 @@ MUTANTS = {
     "bf16_shift": ("uint32_t u = ((uint32_t)h) << 16;", "uint32_t u = ((uint32_t)h) << 15;"),
     "descale_mixup": ("const double dv = descale_v ? descale_v[bhk] : 1.0;",
                       "const double dv = descale_k ? descale_k[bhk] : 1.0;"),
+    # quantisation oracle
+    "hadamard_lower_right_sign": ("out[(i + n) * d + (j + n)] = -h;",
+                                  "out[(i + n) * d + (j + n)] = h;"),
+    "rotation_norm_dropped": ("y[i * d + j] = acc / sqrt((double)d);", "y[i * d + j] = acc;"),
+    "rotation_signs_ignored": ("* (double)signs[t] *", "*"),
+    "rotation_wrong_operand": ("acc += load_x(x, elem_type, base + i * d + t)",
+                               "acc += load_x(x, elem_type, base + i * d + j)"),
+    "ties_to_odd": ("(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
+    "amax_signed": ("if (fabs(y[e]) > amax) amax = fabs(y[e]);", "if (y[e] > amax) amax = y[e];"),
+    "descale_inverted": ("descale[s] = amax > 0.0 ? amax / E4M3_MAX_FINITE : 1.0;",
+                         "descale[s] = amax > 0.0 ? E4M3_MAX_FINITE / amax : 1.0;"),
+    "zero_slice_descale": ("descale[s] = amax > 0.0 ? amax / E4M3_MAX_FINITE : 1.0;",
+                           "descale[s] = amax > 0.0 ? amax / E4M3_MAX_FINITE : 0.0;"),
+    "code_scale_wrong": ("oracle_encode_e4m3(y[e] * E4M3_MAX_FINITE / amax)",
+                         "oracle_encode_e4m3(y[e] * 240.0 / amax)"),
 }
 
 
 def _build_mutant(tmp_path, name, old, new):
-    src = open(SRC).read()
-    assert src.count(old) == 1, "mutation anchor not found: %s" % name
-    path = tmp_path / (name + ".c")
-    path.write_text(src.replace(old, new))
+    hits = [src for src in SOURCES if open(src).read().count(old) == 1]
+    assert len(hits) == 1 and sum(open(src).read().count(old) for src in SOURCES) == 1, \
+        "mutation anchor not found exactly once: %s" % name
+    sources = []
+    for src in SOURCES:
+        text = open(src).read()
+        path = tmp_path / os.path.basename(src)
+        path.write_text(text.replace(old, new) if src == hits[0] else text)
+        sources.append(str(path))
     lib = tmp_path / ("lib" + name + ".so")
-    subprocess.run(["gcc", "-O1", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", str(lib),
-                    str(path), "-lm"], check=True)
+    oracle_build.compile_library(str(lib), sources, opt="-O1")
     return oracle.load_library(str(lib))
 
 
