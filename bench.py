@@ -207,6 +207,9 @@ def oracle_timed_sample(w, inp, n_rows, seed=0):
     dt = time.perf_counter() - t0
     desc = ("%d random query rows (of %d) of workload %s, each over its full admissible key "
             "range, fp64" % (n_rows, total_rows, w.name))
+    if w.rotate:
+        desc += (" (attention over the bf16 source values; the oracle's quantisation, about "
+                 "%.1f%% of its work at this shape, is not timed)" % (100.0 * w.d / w.N / 2))
     return _row_flops(w, rows) / dt / 1e12, desc, oracle.max_threads(), dt
 
 
@@ -241,16 +244,43 @@ def run_ours(args):
     inp = workloads.make_inputs(w, seed=rank_seed(w, rank))
     host = [inp.q, inp.k, inp.v]
     q, k, v = (t.to(dev) for t in host)
-    fp8 = inp.descale_q is not None
-    if fp8:
+    fp8 = inp.descale_q is not None or w.rotate
+    if inp.descale_q is not None:
         dq, dk, dv = (t.to(dev) for t in (inp.descale_q, inp.descale_k, inp.descale_v))
     out_dtype = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
     o = torch.empty((w.B, w.Hq, w.N, w.d), dtype=out_dtype, device=dev)
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # Incoherent-processing workloads quantise their bf16 Q, K (rotated) and V on the GPU
+    # every step, then run the fp8 kernel: 3 quantisation kernels + 1 attention kernel.
+    launches_per_step = 4 if w.rotate else 1
+    split = None
+    if w.rotate:
+        host.append(inp.signs)
+        signs = inp.signs.to(dev)
+        q8, k8, v8 = (torch.empty(t.shape, dtype=torch.float8_e4m3fn, device=dev)
+                      for t in (q, k, v))
+        dq = torch.empty((w.B * w.Hq,), dtype=torch.float32, device=dev)
+        dk = torch.empty((w.B * w.Hkv,), dtype=torch.float32, device=dev)
+        dv = torch.empty((w.B * w.Hkv,), dtype=torch.float32, device=dev)
+        split = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                 for _ in range(args.steps)]
 
-    def step():
-        if fp8:
+    def step(i=None):
+        ev = split[i] if (split is not None and i is not None) else None
+        if w.rotate:
+            if ev:
+                ev[0].record(stream)
+            fa.quantize_e4m3(q, signs, out=q8, descale=dq)
+            fa.quantize_e4m3(k, signs, out=k8, descale=dk)
+            fa.quantize_e4m3(v, None, out=v8, descale=dv)
+            if ev:
+                ev[1].record(stream)
+            fa.forward_fp8(q8, k8, v8, dq, dk, dv, causal=w.causal, scale=w.scale, out=o,
+                           lse=lse)
+            if ev:
+                ev[2].record(stream)
+        elif fp8:
             fa.forward_fp8(q, k, v, dq, dk, dv, causal=w.causal, scale=w.scale, out=o, lse=lse)
         else:
             fa.forward(q, k, v, causal=w.causal, scale=w.scale, out_dtype=out_dtype, out=o,
@@ -268,8 +298,8 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for _ in range(args.steps):
-        step()
+    for i in range(args.steps):
+        step(i)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -279,25 +309,44 @@ def run_ours(args):
     ms_max = max_over_ranks(elapsed_ms, world, dev)
     ms_per_step = ms_max / args.steps
     value = w.flops * world * args.steps / (ms_max / 1e3) / 1e12
-    # Dominant (only) kernel: one fa_fwd launch per step on `stream`, so its average
-    # launch duration is this rank's elapsed time / steps.
-    kernel_ms = elapsed_ms / args.steps
+    # Dominant kernel: the attention kernel, launched once per step on `stream`.  Alone in
+    # the step, its average launch duration is this rank's elapsed time / steps; after the
+    # quantisation kernels, events recorded around it inside the timed loop give it.
+    quant = None
+    if split is None:
+        kernel_ms = elapsed_ms / args.steps
+    else:
+        kernel_ms = sum(e[1].elapsed_time(e[2]) for e in split) / args.steps
+        quant_ms = sum(e[0].elapsed_time(e[1]) for e in split) / args.steps
+        # Algorithmic bytes of quantising Q, K and V: read bf16 once, write e4m3 codes and
+        # one fp32 descale per (batch, head).
+        elems = sum(t.numel() for t in (q, k, v))
+        qbytes = 3.0 * elems + 4.0 * (dq.numel() + dk.numel() + dv.numel())
+        quant = {"kernel": "fa_quant_kernel x 3 (Q and K rotated, V plain)",
+                 "bound": "hbm", "ms_per_step": quant_ms,
+                 "achieved": qbytes / (quant_ms / 1e3) / 1e9, "unit": "GB/s",
+                 "algorithmic_bytes": qbytes}
     achieved = w.flops / (kernel_ms / 1e3) / 1e12
 
     # End to end through the public API: pinned host inputs -> device, forward, O and LSE
     # back to pinned host memory, every step inside the timed region.
     e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 20))
-    hq_, hk_, hv_ = (t.pin_memory() for t in host)
+    hq_, hk_, hv_ = (t.pin_memory() for t in host[:3])
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    if fp8:
+    hds = []
+    if w.rotate:
+        hs_ = inp.signs.pin_memory()
+    elif fp8:
         hds = [t.pin_memory() for t in (inp.descale_q, inp.descale_k, inp.descale_v)]
 
     def e2e_step():
         q.copy_(hq_, non_blocking=True)
         k.copy_(hk_, non_blocking=True)
         v.copy_(hv_, non_blocking=True)
-        if fp8:
+        if w.rotate:
+            signs.copy_(hs_, non_blocking=True)
+        elif fp8:
             for dst, src in zip((dq, dk, dv), hds):
                 dst.copy_(src, non_blocking=True)
         step()
@@ -318,8 +367,7 @@ def run_ours(args):
         barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d = sum(t.numel() * t.element_size() for t in host)
-        if fp8:
-            h2d += sum(t.numel() * t.element_size() for t in hds)
+        h2d += sum(t.numel() * t.element_size() for t in hds)
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
         e2e = {"value": w.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
@@ -331,6 +379,9 @@ def run_ours(args):
         return
 
     peaks, peak_src = load_peaks()
+    if quant is not None:
+        quant["peak"] = peaks["hbm_gbs"]
+        quant["frac"] = quant["achieved"] / quant["peak"]
     if fp8:
         peak = peaks["bf16_tflops"] * 2.0   # fp8 dense = 2x bf16 dense (nominal ratio)
         peak_note = "fp8 peak = measured bf16 burst x 2 (nominal fp8/bf16 ratio)"
@@ -358,9 +409,11 @@ def run_ours(args):
                      "kernel": "fa_fwd_kernel"},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps + 1 + e2e_steps,
+        "gpu_launches": launches_per_step * (args.steps + e2e_steps),
         "clocks": clk,
     }
+    if quant is not None:
+        line["quantise"] = quant
     print(json.dumps(line))
 
 

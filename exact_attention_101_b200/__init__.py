@@ -1,11 +1,11 @@
 """B200-native fused exact attention forward: Python binding of ``libfa_b200.so``.
 
 The C ABI (``include/fa_b200.h``) is the product; this module only marshals arguments
-into it.  The functions ``fa_fwd``, ``fa_fwd_fp8``, ``fa_check_device_error`` and
-``fa_status_string`` have the names and argument order of the C entry points and take
-raw device pointers.  ``forward`` / ``forward_fp8`` are conveniences that take CUDA
-tensors (PyTorch provides device memory and streams only), allocate the outputs and
-raise on a non-zero status.  Every step of the attention runs in the CUDA kernels; there
+into it.  The functions ``fa_fwd``, ``fa_fwd_fp8``, ``fa_quantize_e4m3``,
+``fa_check_device_error`` and ``fa_status_string`` have the names and argument order of
+the C entry points and take raw device pointers.  ``forward`` / ``forward_fp8`` /
+``quantize_e4m3`` are conveniences that take CUDA tensors (PyTorch provides device
+memory and streams only), allocate the outputs and raise on a non-zero status.  Every step of the attention runs in the CUDA kernels; there
 is no CPU or library fallback -- if the shared library is missing, importing a function
 that needs it raises.
 """
@@ -20,8 +20,8 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
-C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_check_device_error", "fa_selftest_bounded_wait",
-             "fa_status_string", "fa_version")
+C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_quantize_e4m3", "fa_check_device_error",
+             "fa_selftest_bounded_wait", "fa_status_string", "fa_version")
 
 _lib = None
 
@@ -45,6 +45,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
         L.fa_fwd_fp8.restype = i
         L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+        L.fa_quantize_e4m3.restype = i
+        L.fa_quantize_e4m3.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.fa_check_device_error.restype = i
         L.fa_check_device_error.argtypes = [vp]
         L.fa_selftest_bounded_wait.restype = i
@@ -69,6 +71,11 @@ def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
     """Raw ``fa_fwd_fp8``."""
     return lib().fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
                             descale_q, descale_k, descale_v, stream)
+
+
+def fa_quantize_e4m3(x, signs, x8, descale, B, H, N, d, stream) -> int:
+    """Raw ``fa_quantize_e4m3`` (signs may be 0 / None for no rotation)."""
+    return lib().fa_quantize_e4m3(x, signs, x8, descale, B, H, N, d, stream)
 
 
 def fa_check_device_error(stream) -> int:
@@ -163,6 +170,30 @@ def forward_fp8(q, k, v, descale_q, descale_k, descale_v, causal=False, scale=No
     if st != FA_OK:
         raise FaError(st, "fa_fwd_fp8")
     return out, lse
+
+
+def quantize_e4m3(x, signs=None, out=None, descale=None, stream=None):
+    """Per-(batch, head) e4m3 quantisation of a bf16 CUDA tensor x [B, H, N, 128], after
+    the random-sign Hadamard rotation when ``signs`` (int8 CUDA tensor of 128 entries,
+    +1 / -1) is given.  Returns ``(codes, descale)``: torch.float8_e4m3fn [B, H, N, 128]
+    and fp32 [B*H], ready for ``forward_fp8``."""
+    import torch
+    if not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 4 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor [B, H, N, d]")
+    B, H, N, d = x.shape
+    if signs is not None and (not signs.is_cuda or signs.dtype != torch.int8 or
+                              signs.numel() != d or not signs.is_contiguous()):
+        raise ValueError("signs must be a contiguous int8 CUDA tensor of d entries")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float8_e4m3fn, device=x.device)
+    if descale is None:
+        descale = torch.empty((B * H,), dtype=torch.float32, device=x.device)
+    st = fa_quantize_e4m3(x.data_ptr(), None if signs is None else signs.data_ptr(),
+                          out.data_ptr(), descale.data_ptr(), B, H, N, d,
+                          _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_quantize_e4m3")
+    return out, descale
 
 
 def check_device_error(stream=None):

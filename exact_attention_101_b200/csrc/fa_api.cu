@@ -16,6 +16,7 @@
 
 #include "fa_b200.h"
 #include "fa_fwd_kernel.cuh"
+#include "fa_quant.cuh"
 
 namespace {
 
@@ -245,6 +246,52 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
                  : launch<128, false, false, false>(tq, tk, tv, p, grid, dev, stream);
 }
 
+template <bool ROTATE>
+fa_status quant_launch(const fa::quant::QuantParams &qp, long long slices, cudaStream_t stream) {
+  const long long grid = slices * fa::quant::CLUSTER;
+  if (grid > INT32_MAX) return FA_ERR_INVALID_ARG;
+  fa::quant::fa_quant_kernel<ROTATE>
+      <<<static_cast<unsigned>(grid), fa::quant::THREADS, 0, stream>>>(qp);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status quantize_common(const void *x, const int8_t *signs, void *x8, float *descale, int B,
+                          int H, int N, int d, cudaStream_t stream) {
+  if (!x || !x8 || !descale) return FA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || (reinterpret_cast<uintptr_t>(descale) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (d != fa::quant::D) return FA_ERR_UNSUPPORTED;
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  DeviceInfo info;
+  fa_status st = device_info(dev, &info);
+  if (st != FA_OK) return st;
+  if (info.major != 10 || info.minor != 0) return FA_ERR_UNSUPPORTED;
+  if (!driver_fns().ok) return FA_ERR_CUDA;
+
+  const uint64_t slices = static_cast<uint64_t>(B) * H;
+  const uint64_t elems = slices * N * d;
+  if (!buffer_ok(x, elems * 2, dev) || !buffer_ok(x8, elems, dev) ||
+      !buffer_ok(descale, slices * 4, dev) || (signs && !buffer_ok(signs, d, dev)))
+    return FA_ERR_INVALID_ARG;
+
+  fa::quant::QuantParams qp;
+  qp.x = static_cast<const uint16_t *>(x);
+  qp.signs = signs;
+  qp.codes = static_cast<uint8_t *>(x8);
+  qp.descale = descale;
+  qp.rows = N;
+  const long long s = static_cast<long long>(slices);
+  if (signs) {
+    qp.norm_over_max = static_cast<float>(1.0 / (448.0 * std::sqrt(static_cast<double>(d))));
+    return quant_launch<true>(qp, s, stream);
+  }
+  qp.norm_over_max = static_cast<float>(1.0 / 448.0);
+  return quant_launch<false>(qp, s, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -264,6 +311,12 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
                      fa_stream_t stream) {
   return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, false, true,
                     descale_q, descale_k, descale_v, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_quantize_e4m3(const void *x, const int8_t *signs, void *x8, float *descale, int B,
+                           int H, int N, int d, fa_stream_t stream) {
+  return quantize_common(x, signs, x8, descale, B, H, N, d,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_check_device_error(fa_stream_t stream) {

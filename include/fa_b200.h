@@ -99,6 +99,36 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
                      const float *descale_v, fa_stream_t stream);
 
 /*
+ * Per-(batch, head) fp8-e4m3 quantisation of a bf16 tensor, optionally with incoherent
+ * processing: the page "FlashAttention-3 (DE)", section "Niedrige Praezision (FP8) mit
+ * reduziertem Quantisierungsfehler", multiplies the query and key vectors by a random
+ * orthogonal (Hadamard) matrix before quantising them to FP8.  The matrix spreads large
+ * entries over all coordinates and, being orthogonal, leaves Q K^T unchanged, so codes
+ * made from rotated Q and K can be passed straight to fa_fwd_fp8.  Rotate Q and K with
+ * the same signs; quantise V without rotation.
+ *
+ *   x        device pointer, bf16 [B, H, N, d] (16-byte aligned, finite values)
+ *   signs    device pointer to d int8 entries, or NULL for no rotation.  An entry < 0
+ *            stands for -1, any other for +1.  With signs every row is replaced by
+ *            y = x diag(s) H / sqrt(d), H the Sylvester-Hadamard matrix of order d
+ *            (H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]).
+ *   x8       device pointer, e4m3 codes [B, H, N, d] (16-byte aligned); must not overlap
+ *            x, signs or descale
+ *   descale  device pointer, fp32 [B*H]: per slice amax = max |y|, descale = amax / 448,
+ *            code = e4m3(y / descale) rounded to nearest even, so y ~ descale * e4m3(code).
+ *            A slice of zeros gets descale 1 and zero codes.
+ *   B, H, N  >= 1
+ *   d        128 (the head dimension of fa_fwd_fp8)
+ *
+ * The call enqueues a memset of descale (used as the amax accumulator) and three kernels
+ * on `stream`.  Returns FA_OK once enqueued; FA_ERR_INVALID_ARG (null, misaligned or
+ * undersized buffer, bad size) or FA_ERR_UNSUPPORTED (d != 128, GPU not sm_100) with
+ * nothing enqueued; FA_ERR_CUDA if a launch failed.
+ */
+fa_status fa_quantize_e4m3(const void *x, const int8_t *signs, void *x8, float *descale,
+                           int B, int H, int N, int d, fa_stream_t stream);
+
+/*
  * Device-side failure report.  Every wait inside the kernels (on a shared-memory
  * mbarrier filled by a TMA copy or a tensor-core commit) is bounded in time; a wait
  * that runs out sets a device error word, makes the other warps of the CTA stop, drains

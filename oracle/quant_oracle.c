@@ -88,7 +88,8 @@ static double load_x(const void *x, int elem_type, int64_t idx) {
  * descale = 1 and every code 0 when amax == 0.
  *
  * Outputs: codes [S, N, d] (may be NULL), descale [S] (may be NULL), y_out [S, N, d] in
- * fp64 (may be NULL).  Returns 0, -1 on invalid arguments, -2 on allocation failure.
+ * fp64 (may be NULL).  nthreads > 0 sets the OpenMP thread count, 0 keeps the default.
+ * Returns 0, -1 on invalid arguments, -2 on allocation failure.
  */
 int oracle_quantize_e4m3(const void *x, int elem_type, const int8_t *signs, int64_t S,
                          int64_t N, int64_t d, uint8_t *codes, double *descale,
@@ -97,6 +98,11 @@ int oracle_quantize_e4m3(const void *x, int elem_type, const int8_t *signs, int6
         (elem_type != ORACLE_QF64 && elem_type != ORACLE_QBF16))
         return -1;
     if (signs != NULL && (d & (d - 1)) != 0) return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
     double *H = NULL;
     if (signs != NULL) {
         for (int64_t t = 0; t < d; ++t)
@@ -112,7 +118,7 @@ int oracle_quantize_e4m3(const void *x, int elem_type, const int8_t *signs, int6
     }
     for (int64_t s = 0; s < S; ++s) {
         const int64_t base = s * N * d;
-#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+#pragma omp parallel for schedule(static)
         for (int64_t i = 0; i < N; ++i) {
             for (int64_t j = 0; j < d; ++j) {
                 if (H == NULL) {
@@ -131,7 +137,7 @@ int oracle_quantize_e4m3(const void *x, int elem_type, const int8_t *signs, int6
             if (fabs(y[e]) > amax) amax = fabs(y[e]);
         if (descale != NULL) descale[s] = amax > 0.0 ? amax / E4M3_MAX_FINITE : 1.0;
         if (codes != NULL) {
-#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+#pragma omp parallel for schedule(static)
             for (int64_t e = 0; e < N * d; ++e)
                 codes[base + e] = amax > 0.0 ? oracle_encode_e4m3(y[e] * E4M3_MAX_FINITE / amax)
                                              : 0;

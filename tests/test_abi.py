@@ -99,3 +99,19 @@ def test_status_strings():
 def test_selftest_rejects_out_of_range_timeout():
     assert fa.fa_selftest_bounded_wait(0, None) == fa.FA_ERR_INVALID_ARG
     assert fa.fa_selftest_bounded_wait(2000000, None) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [
+    dict(x=0), dict(x8=0), dict(descale=0), dict(x=A + 8), dict(x8=A + 4), dict(descale=A + 2),
+    dict(B=0), dict(H=0), dict(N=0), dict(d=0), dict(N=-1),
+])
+def test_quantize_invalid_arguments(kw):
+    a = dict(x=A, signs=A, x8=A, descale=A, B=1, H=2, N=64, d=128)
+    a.update(kw)
+    assert fa.fa_quantize_e4m3(a["x"], a["signs"], a["x8"], a["descale"], a["B"], a["H"],
+                               a["N"], a["d"], None) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_quantize_supports_head_dim_128_only(d):
+    assert fa.fa_quantize_e4m3(A, None, A, A, 1, 2, 64, d, None) == fa.FA_ERR_UNSUPPORTED

@@ -14,6 +14,11 @@ per K/V head) and an fp8-e4m3 case with sparse large-magnitude entries (the outl
 that the page "FlashAttention-3 (DE)" names as the risk of FP8 quantisation, section
 "Niedrige Praezision (FP8) mit reduziertem Quantisierungsfehler").  None of the pages
 benchmarks on a public dataset, so the values are i.i.d. standard normal.
+
+Two more workloads feed the incoherent processing of that section (``rotate=True``):
+bf16 Q/K/V with the fp8 case's outliers, or with a few outlier channels shared by Q and
+K, that the library quantises itself after a random-sign Hadamard rotation of Q and K.
+Their sign vector is drawn here, after the values, and passed to the library as input.
 """
 from __future__ import annotations
 
@@ -40,6 +45,10 @@ class Workload:
     seed: int
     outlier_rate: float = 0.0
     outlier_scale: float = 1.0
+    outlier_kind: str = "entry"   # "entry": i.i.d. entries of Q, K, V; "channel": whole
+    #                               channels of Q and K (outlier_channels of them)
+    outlier_channels: int = 0
+    rotate: bool = False          # bf16 source quantised on the GPU with Hadamard rotation
 
     @property
     def scale(self) -> float:
@@ -53,10 +62,13 @@ class Workload:
         return f / 2 if self.causal else f
 
     def describe(self) -> Dict[str, object]:
-        return {"workload": self.name, "B": self.B, "Hq": self.Hq, "Hkv": self.Hkv,
-                "Nq": self.N, "Nk": self.N, "d": self.d, "causal": self.causal,
-                "in_dtype": self.in_dtype, "out_dtype": self.out_dtype,
-                "seed": self.seed}
+        out = {"workload": self.name, "B": self.B, "Hq": self.Hq, "Hkv": self.Hkv,
+               "Nq": self.N, "Nk": self.N, "d": self.d, "causal": self.causal,
+               "in_dtype": self.in_dtype, "out_dtype": self.out_dtype,
+               "seed": self.seed}
+        if self.rotate:
+            out["quantise"] = "e4m3 per head on the GPU, Q and K after random-sign Hadamard"
+        return out
 
 
 WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
@@ -67,6 +79,10 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("long", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003),
     Workload("gqa_causal", 4, 32, 8, 8192, 128, True, "bf16", "bf16", 1004),
     Workload("fp8", 8, 16, 16, 4096, 128, False, "e4m3", "bf16", 1005, 1e-3, 50.0),
+    Workload("fp8_incoherent", 8, 16, 16, 4096, 128, False, "bf16", "bf16", 1006, 1e-3, 50.0,
+             rotate=True),
+    Workload("fp8_incoherent_channels", 8, 16, 16, 4096, 128, False, "bf16", "bf16", 1007,
+             1.0, 10.0, outlier_kind="channel", outlier_channels=4, rotate=True),
 ]}
 
 
@@ -78,6 +94,7 @@ class Inputs:
     descale_q: Optional[torch.Tensor] = None   # fp32 [B*Hq]   (e4m3 only)
     descale_k: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
     descale_v: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
+    signs: Optional[torch.Tensor] = None       # int8 [d] of +-1 (rotate workloads only)
 
 
 def _quantise_e4m3_per_head(x: torch.Tensor):
@@ -110,14 +127,21 @@ def make_inputs(w: Workload, seed: Optional[int] = None, *, B: Optional[int] = N
     q32 = torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32)
     k32 = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
     v32 = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
-    if w.in_dtype == "bf16":
-        return Inputs(q32.to(torch.bfloat16), k32.to(torch.bfloat16), v32.to(torch.bfloat16))
-    if w.in_dtype != "e4m3":
-        raise ValueError(w.in_dtype)
-    for t in (q32, k32, v32):
-        if w.outlier_rate > 0:
+    if w.outlier_kind == "channel":
+        channels = torch.randperm(d, generator=g)[:w.outlier_channels]
+        q32[..., channels] *= w.outlier_scale
+        k32[..., channels] *= w.outlier_scale
+    elif w.outlier_rate > 0:
+        for t in (q32, k32, v32):
             mask = torch.rand(t.shape, generator=g) < w.outlier_rate
             t[mask] *= w.outlier_scale
+    if w.in_dtype == "bf16":
+        inp = Inputs(q32.to(torch.bfloat16), k32.to(torch.bfloat16), v32.to(torch.bfloat16))
+        if w.rotate:
+            inp.signs = torch.where(torch.rand(d, generator=g) < 0.5, -1, 1).to(torch.int8)
+        return inp
+    if w.in_dtype != "e4m3":
+        raise ValueError(w.in_dtype)
     q8, dq = _quantise_e4m3_per_head(q32)
     k8, dk = _quantise_e4m3_per_head(k32)
     v8, dv = _quantise_e4m3_per_head(v32)
