@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
 
 #include <cuda.h>
@@ -246,8 +247,84 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
                  : launch<128, false, false, false>(tq, tk, tv, p, grid, dev, stream);
 }
 
+// Shared-memory quantisation kernel: the smallest power-of-two cluster (<= 8 CTAs) that
+// keeps a CTA at <= MAX_SMEM_ROWS rows.  Returns false if the slice is longer than that.
+bool quant_smem_shape(int N, int *cs, int *cta_rows) {
+  int c = 1;
+  auto rows_for = [&](int cc) { return ((N + cc - 1) / cc + 7) / 8 * 8; };
+  while (c < fa::quant::MAX_CLUSTER && rows_for(c) > fa::quant::MAX_SMEM_ROWS) c *= 2;
+  *cs = c;
+  *cta_rows = rows_for(c);
+  return *cta_rows <= fa::quant::MAX_SMEM_ROWS;
+}
+
+// Whether a cluster of `cs` CTAs with `smem` bytes of dynamic shared memory each can be
+// resident on this device (asked once per device, kernel and shape).
 template <bool ROTATE>
-fa_status quant_launch(const fa::quant::QuantParams &qp, long long slices, cudaStream_t stream) {
+bool quant_smem_fits(int dev, int cs, int smem, int grid) {
+  static std::mutex mu;
+  static std::map<long long, bool> known;
+  auto kern = fa::quant::fa_quant_smem_kernel<ROTATE>;
+  static std::once_flag attr_once[kMaxDevices];
+  static bool attr_ok[kMaxDevices];
+  std::call_once(attr_once[dev], [&] {
+    attr_ok[dev] =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::quant::MAX_SMEM_ROWS * fa::quant::ROW_BYTES) == cudaSuccess;
+  });
+  if (!attr_ok[dev]) {
+    cudaGetLastError();
+    return false;
+  }
+  const long long key = (static_cast<long long>(dev) << 40) | (static_cast<long long>(cs) << 32) | smem;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = known.find(key);
+  if (it != known.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = cs;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(fa::quant::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  const bool ok =
+      cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0;
+  if (!ok) cudaGetLastError();
+  known[key] = ok;
+  return ok;
+}
+
+template <bool ROTATE>
+fa_status quant_launch(fa::quant::QuantParams qp, long long slices, int dev,
+                       cudaStream_t stream) {
+  int cs = 1, cta_rows = 0;
+  if (quant_smem_shape(qp.rows, &cs, &cta_rows)) {
+    const long long grid = slices * cs;
+    const int smem = cta_rows * fa::quant::ROW_BYTES;
+    if (grid <= INT32_MAX && quant_smem_fits<ROTATE>(dev, cs, smem, static_cast<int>(grid))) {
+      qp.cta_rows = cta_rows;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = cs;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+      cfg.blockDim = dim3(fa::quant::THREADS, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = stream;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, fa::quant::fa_quant_smem_kernel<ROTATE>, qp) != cudaSuccess)
+        return FA_ERR_CUDA;
+      return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
+  }
   const long long grid = slices * fa::quant::CLUSTER;
   if (grid > INT32_MAX) return FA_ERR_INVALID_ARG;
   fa::quant::fa_quant_kernel<ROTATE>
@@ -283,13 +360,14 @@ fa_status quantize_common(const void *x, const int8_t *signs, void *x8, float *d
   qp.codes = static_cast<uint8_t *>(x8);
   qp.descale = descale;
   qp.rows = N;
+  qp.cta_rows = 0;
   const long long s = static_cast<long long>(slices);
   if (signs) {
     qp.norm_over_max = static_cast<float>(1.0 / (448.0 * std::sqrt(static_cast<double>(d))));
-    return quant_launch<true>(qp, s, stream);
+    return quant_launch<true>(qp, s, dev, stream);
   }
   qp.norm_over_max = static_cast<float>(1.0 / 448.0);
-  return quant_launch<false>(qp, s, stream);
+  return quant_launch<false>(qp, s, dev, stream);
 }
 
 }  // namespace

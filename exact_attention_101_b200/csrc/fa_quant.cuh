@@ -15,14 +15,19 @@
 // y = z / sqrt(d)), so it only enters the descale.  Without rotation z = x and the
 // descale is amax / 448.
 //
-// HBM-bound: a row is 256 bytes of bf16 in and 128 bytes of codes out.  One kernel does
-// the whole job: a cluster of CLUSTER CTAs owns one slice, each CTA an eighth of its rows.
-// Pass 1 computes the CTA's amax; the cluster combines the CTAs' values through
-// distributed shared memory; pass 2 re-reads the same rows -- from L2, since only a few
-// tens of MB stream through the GPU in between -- and writes the codes.  So HBM sees one
-// read of the input and one write of the codes.
-//
-// Thread layout: four threads per row, 8 rows per warp.  The row's 16-byte chunks c =
+// HBM-bound: a row is 256 bytes of bf16 in and 128 bytes of codes out, and the slice
+// amax must be known before the first code is written.  A cluster of CTAs owns one slice
+// (the amax is combined through distributed shared memory), each CTA a contiguous share of
+// its rows:
+//  * fa_quant_smem_kernel (slices up to 2048 rows): the CTA copies its whole share (at
+//    most 256 rows, 64 KB) into shared memory with bulk asynchronous copies (64-row
+//    chunks, one mbarrier each, all in flight at once), computes its amax from there, and
+//    after the cluster exchange rounds the same rows from shared memory.  HBM sees one
+//    read and one write.
+//  * fa_quant_kernel (longer slices): pass 2 re-reads the rows from global memory
+//    (partly from L2).  Measured on B200, it beats holding longer slices on chip in
+//    clusters of 16 CTAs (which the GPU keeps fewer of in flight).
+//// Thread layout: four threads per row, 8 rows per warp.  The row's 16-byte chunks c =
 // 0..15 (8 bf16 each) are dealt round-robin: thread p holds chunks 4 i + p, i = 0..3, so
 // each load instruction of a warp reads 64 contiguous bytes of each of 8 rows.  Element
 // t = 32 i + 8 p + e (e = 0..7) is kept at position q = 8 i + e of the thread.  The
@@ -36,6 +41,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "fa_fwd_kernel.cuh"  // device error word
 #include "sm100.cuh"
 
 namespace fa {
@@ -45,8 +51,14 @@ constexpr int D = 128;
 constexpr int UNIT_ROWS = 8;          // rows per warp-level unit (4 threads per row)
 constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
-constexpr int CLUSTER = 8;            // CTAs per slice
+constexpr int CLUSTER = 8;            // CTAs per slice of the global-memory kernel
+constexpr int MAX_CLUSTER = 8;        // CTAs per slice of the shared-memory kernel
+constexpr int ROW_BYTES = D * 2;
+constexpr int CHUNK_ROWS = 64;        // rows per bulk copy
+constexpr int MAX_SMEM_ROWS = 256;    // rows a CTA holds on chip (64 KB)
+constexpr int MAX_CHUNKS = MAX_SMEM_ROWS / CHUNK_ROWS;
 constexpr float E4M3_MAX = 448.0f;
+constexpr uint32_t ERR_WAIT_QUANT = 1u << 5;
 
 struct QuantParams {
   const uint16_t *x;                  // bf16 bits [S, N, D]
@@ -54,6 +66,7 @@ struct QuantParams {
   uint8_t *codes;                     // e4m3 [S, N, D]
   float *descale;                     // [S]
   int rows;                           // N
+  int cta_rows;                       // shared-memory kernel: rows per CTA (multiple of 8)
   float norm_over_max;                // descale = amax * norm_over_max
 };
 
@@ -94,17 +107,34 @@ __device__ __forceinline__ void load_sign_masks(const int8_t *signs, int p, uint
     }
 }
 
-// Load this thread's 32 elements of row `row` (zeros for a row past the slice end) and,
-// with ROTATE, apply the signs and the Walsh-Hadamard transform.  zp[k] holds the fp32
-// pair at positions (2k, 2k+1).
-template <bool ROTATE, bool LAST>
-__device__ __forceinline__ void load_transform(const uint16_t *x, long long row, bool valid,
-                                               int p, const uint32_t (&m)[16],
-                                               uint64_t (&zp)[16]) {
-  uint4 raw[4];
+// This thread's 32 elements of a row: 16-byte chunks 4 i + p of the row at `src` (global
+// memory), zeros for a row past the slice end.
+template <bool LAST>
+__device__ __forceinline__ void load_raw_global(const uint16_t *src, bool valid, int p,
+                                                uint4 (&raw)[4]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
-    raw[i] = valid ? ld_stream_v4<LAST>(x + row * D + (4 * i + p) * 8) : make_uint4(0, 0, 0, 0);
+    raw[i] = valid ? ld_stream_v4<LAST>(src + (4 * i + p) * 8) : make_uint4(0, 0, 0, 0);
+}
+
+// The same from a row held in shared memory at byte address `row_addr`.
+__device__ __forceinline__ void load_raw_shared(uint32_t row_addr, bool valid, int p,
+                                                uint4 (&raw)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    raw[i] = make_uint4(0, 0, 0, 0);
+    if (valid)
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(raw[i].x), "=r"(raw[i].y), "=r"(raw[i].z), "=r"(raw[i].w)
+                   : "r"(row_addr + (4 * i + p) * 16));
+  }
+}
+
+// bf16 -> fp32 and, with ROTATE, the signs and the Walsh-Hadamard transform.  zp[k] holds
+// the fp32 pair at positions (2k, 2k+1).
+template <bool ROTATE>
+__device__ __forceinline__ void transform_raw(const uint4 (&raw)[4], int p,
+                                              const uint32_t (&m)[16], uint64_t (&zp)[16]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
@@ -116,37 +146,170 @@ __device__ __forceinline__ void load_transform(const uint16_t *x, long long row,
       zp[4 * i + h] = ROTATE ? ptx::f2_pack(lo + hi, lo - hi) : ptx::f2_pack(lo, hi);
     }
   }
-  if (!ROTATE) return;
-  // in-thread strides 2, 4 (e) and 32, 64 (i): pair-index strides 1, 2, 4, 8
+  if constexpr (ROTATE) {
+    // in-thread strides 2, 4 (e) and 32, 64 (i): pair-index strides 1, 2, 4, 8
 #pragma unroll
-  for (int h = 1; h < 16; h <<= 1)
+    for (int h = 1; h < 16; h <<= 1)
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
-      if ((k & h) == 0) {
-        const uint64_t a = zp[k], b = zp[k + h];
-        zp[k] = ptx::f2_add(a, b);
-        zp[k + h] = ptx::f2_sub(a, b);
+      for (int k = 0; k < 16; ++k)
+        if ((k & h) == 0) {
+          const uint64_t a = zp[k], b = zp[k + h];
+          zp[k] = ptx::f2_add(a, b);
+          zp[k + h] = ptx::f2_sub(a, b);
+        }
+    // strides 8 and 16: the lower index of each pair adds, the upper subtracts itself
+    // from its partner: z <- other + sgn * z with sgn = +-1 (exact product, one rounding)
+#pragma unroll
+    for (int bit = 1; bit <= 2; bit <<= 1) {
+      const float sg = (p & bit) ? -1.f : 1.f;
+      const uint64_t sgn = ptx::f2_pack(sg, sg);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        float lo, hi;
+        ptx::f2_unpack(zp[k], lo, hi);
+        const float olo = __shfl_xor_sync(0xffffffffu, lo, bit);
+        const float ohi = __shfl_xor_sync(0xffffffffu, hi, bit);
+        zp[k] = ptx::f2_fma(zp[k], sgn, ptx::f2_pack(olo, ohi));
       }
-  // strides 8 and 16: the lower index of each pair adds, the upper subtracts itself
-  // from its partner: z <- other + sgn * z with sgn = +-1 (exact product, one rounding)
-#pragma unroll
-  for (int bit = 1; bit <= 2; bit <<= 1) {
-    const float sg = (p & bit) ? -1.f : 1.f;
-    const uint64_t sgn = ptx::f2_pack(sg, sg);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      float lo, hi;
-      ptx::f2_unpack(zp[k], lo, hi);
-      const float olo = __shfl_xor_sync(0xffffffffu, lo, bit);
-      const float ohi = __shfl_xor_sync(0xffffffffu, hi, bit);
-      zp[k] = ptx::f2_fma(zp[k], sgn, ptx::f2_pack(olo, ohi));
     }
   }
 }
 
-// One slice per cluster: grid = S * CLUSTER CTAs.  CTA c of the cluster takes the units
-// (8-row blocks) [c U / CLUSTER, (c+1) U / CLUSTER) of its slice, U = ceil(N / 8), and its
-// warps take every WARPS-th unit of that range, so a CTA step covers 64 consecutive rows.
+__device__ __forceinline__ float abs_max(float m, const uint64_t (&zp)[16]) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float lo, hi;
+    ptx::f2_unpack(zp[k], lo, hi);
+    m = ptx::max3(m, fabsf(lo), fabsf(hi));
+  }
+  return m;
+}
+
+// codes of this thread's 32 elements: element t = 32 i + 8 p + e goes to byte t of the row
+__device__ __forceinline__ void store_codes(uint8_t *row_codes, int p, float inv,
+                                            const uint64_t (&zp)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float z[8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) ptx::f2_unpack(zp[4 * i + h], z[2 * h], z[2 * h + 1]);
+    const uint32_t a = ptx::pack_e4m3x4(z[0] * inv, z[1] * inv, z[2] * inv, z[3] * inv);
+    const uint32_t b = ptx::pack_e4m3x4(z[4] * inv, z[5] * inv, z[6] * inv, z[7] * inv);
+    st_v2(row_codes + 32 * i + 8 * p, a, b);
+  }
+}
+
+// Block-wide maximum of m (non-negative) into every CTA of the cluster, then the maximum
+// over the cluster.  Every thread of every CTA must call it (it holds cluster barriers).
+__device__ __forceinline__ float cluster_amax(float m, float *warp_max, float *cta_max) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) warp_max[warp] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float c = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) c = fmaxf(c, warp_max[w]);
+    *cta_max = c;
+  }
+  // every CTA's value is written before anyone reads it, and read by everyone before any
+  // CTA of the cluster may exit
+  cluster.sync();
+  float amax = 0.f;
+  const int n = static_cast<int>(cluster.num_blocks());
+  for (int c = 0; c < n; ++c) amax = fmaxf(amax, *cluster.map_shared_rank(cta_max, c));
+  cluster.sync();
+  return amax;
+}
+
+// Bounded wait for a bulk copy (parity 0: each barrier completes once per launch).
+__device__ __forceinline__ bool quant_wait(uint32_t bar) {
+  if (ptx::mbar_try_wait(bar, 0)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1; it < WAIT_MAX_ITERS; ++it) {
+    if (ptx::mbar_try_wait(bar, 0)) return true;
+    if ((it & 255u) == 0 && ptx::globaltimer_ns() - t0 > WAIT_LIMIT_NS) break;
+  }
+  atomicOr(&g_fa_error, ERR_WAIT_QUANT);
+  return false;
+}
+
+// Slices of up to MAX_CLUSTER * MAX_SMEM_ROWS rows: grid = S * cluster CTAs (cluster size
+// 1 .. 8, set at launch); CTA c of the cluster holds rows [c * cta_rows, (c+1) * cta_rows) of its
+// slice in dynamic shared memory (cta_rows * 256 bytes).  Warp w processes the 8-row units
+// w, w + 8, ... of that share, so unit j of a warp lies in chunk j.
+template <bool ROTATE>
+__global__ void __launch_bounds__(THREADS, 3) fa_quant_smem_kernel(const QuantParams qp) {
+  namespace cg = cooperative_groups;
+  extern __shared__ __align__(128) uint8_t rows_smem[];
+  __shared__ __align__(8) uint64_t bars[MAX_CHUNKS];
+  __shared__ float warp_max[WARPS];
+  __shared__ float cta_max;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, p = lane & 3, r = lane >> 2;
+  const int cs = static_cast<int>(cluster.num_blocks());
+  const long long slice = blockIdx.x / cs;
+  const int row_begin = static_cast<int>(cluster.block_rank()) * qp.cta_rows;
+  const int nrows = max(0, min(qp.rows - row_begin, qp.cta_rows));
+  const int nchunks = (nrows + CHUNK_ROWS - 1) / CHUNK_ROWS;
+  const uint16_t *src = qp.x + (slice * qp.rows + row_begin) * D;
+  const uint32_t smem_rows = ptx::smem_addr(rows_smem);
+  const uint32_t bar0 = ptx::smem_addr(bars);
+
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < nchunks; ++c) ptx::mbar_init(bar0 + 8u * c, 1);
+    ptx::fence_mbar_init();
+    for (int c = 0; c < nchunks; ++c) {
+      const int n = min(CHUNK_ROWS, nrows - c * CHUNK_ROWS);
+      ptx::mbar_arrive_expect_tx(bar0 + 8u * c, n * ROW_BYTES);
+      ptx::bulk_load(smem_rows + c * CHUNK_ROWS * ROW_BYTES, src + c * CHUNK_ROWS * D,
+                     n * ROW_BYTES, bar0 + 8u * c);
+    }
+  }
+  uint32_t m16[16] = {};
+  if (ROTATE) load_sign_masks(qp.signs, p, m16);
+  __syncthreads();
+
+  // pass 1: amax of this CTA's rows, chunk by chunk as the copies land
+  float m = 0.f;
+  bool ok = true;
+  for (int u = warp; u * UNIT_ROWS < nrows; u += WARPS) {
+    ok = ok && quant_wait(bar0 + 8u * (u * UNIT_ROWS / CHUNK_ROWS));
+    const int row = u * UNIT_ROWS + r;
+    uint4 raw[4];
+    load_raw_shared(smem_rows + row * ROW_BYTES, ok && row < nrows, p, raw);
+    uint64_t zp[16];
+    transform_raw<ROTATE>(raw, p, m16, zp);
+    m = abs_max(m, zp);
+  }
+  const float amax = cluster_amax(m, warp_max, &cta_max);
+  if (cluster.block_rank() == 0 && threadIdx.x == 0)
+    qp.descale[slice] = amax > 0.f ? amax * qp.norm_over_max : 1.f;
+  const float inv = amax > 0.f ? __fdiv_rn(E4M3_MAX, amax) : 0.f;
+
+  // pass 2: the same rows from shared memory, scaled and rounded to e4m3
+  uint8_t *dst = qp.codes + (slice * qp.rows + row_begin) * D;
+  for (int u = warp; u * UNIT_ROWS < nrows; u += WARPS) {
+    const int row = u * UNIT_ROWS + r;
+    uint4 raw[4];
+    load_raw_shared(smem_rows + row * ROW_BYTES, ok && row < nrows, p, raw);
+    uint64_t zp[16];
+    transform_raw<ROTATE>(raw, p, m16, zp);
+    if (ok && row < nrows) store_codes(dst + static_cast<long long>(row) * D, p, inv, zp);
+  }
+  // a copy that timed out may still be in flight: let it land before the CTA exits
+  if (!ok && lane == 0)
+    for (int c = 0; c < nchunks; ++c) quant_wait(bar0 + 8u * c);
+}
+
+// Longer slices: grid = S * CLUSTER CTAs, one slice per cluster.  CTA c of the cluster
+// takes the units (8-row blocks) [c U / CLUSTER, (c+1) U / CLUSTER) of its slice,
+// U = ceil(N / 8), and its warps take every WARPS-th unit of that range, so a CTA step
+// covers 64 consecutive rows.  Pass 2 re-reads the rows from global memory.
 template <bool ROTATE>
 __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS, 3)
     fa_quant_kernel(const QuantParams qp) {
@@ -163,60 +326,28 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS, 3)
   uint32_t m16[16] = {};
   if (ROTATE) load_sign_masks(qp.signs, p, m16);
 
-  // pass 1: amax of this CTA's rows
   float m = 0.f;
   for (long long u = u0 + warp; u < u1; u += WARPS) {
-    const int row0 = static_cast<int>(u * UNIT_ROWS);
-    const bool valid = row0 + r < qp.rows;
+    const long long row = u * UNIT_ROWS + r;
+    uint4 raw[4];
+    load_raw_global<false>(qp.x + (slice * qp.rows + row) * D, row < qp.rows, p, raw);
     uint64_t zp[16];
-    load_transform<ROTATE, false>(qp.x, slice * qp.rows + row0 + r, valid, p, m16, zp);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      float lo, hi;
-      ptx::f2_unpack(zp[k], lo, hi);
-      m = ptx::max3(m, fabsf(lo), fabsf(hi));
-    }
+    transform_raw<ROTATE>(raw, p, m16, zp);
+    m = abs_max(m, zp);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) warp_max[warp] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float c = 0.f;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) c = fmaxf(c, warp_max[w]);
-    cta_max = c;
-  }
-  // every CTA's cta_max is written before anyone reads it, and read by everyone before
-  // any CTA of the cluster may exit
-  cluster.sync();
-  float amax = 0.f;
-#pragma unroll
-  for (int c = 0; c < CLUSTER; ++c) amax = fmaxf(amax, *cluster.map_shared_rank(&cta_max, c));
-  cluster.sync();
-
+  const float amax = cluster_amax(m, warp_max, &cta_max);
   if (crank == 0 && threadIdx.x == 0)
     qp.descale[slice] = amax > 0.f ? amax * qp.norm_over_max : 1.f;
   const float inv = amax > 0.f ? __fdiv_rn(E4M3_MAX, amax) : 0.f;
 
-  // pass 2: the same rows again (now from L2), scaled and rounded to e4m3
   for (long long u = u0 + warp; u < u1; u += WARPS) {
-    const int row0 = static_cast<int>(u * UNIT_ROWS);
-    const bool valid = row0 + r < qp.rows;
-    const long long row = slice * qp.rows + row0 + r;
+    const long long row = u * UNIT_ROWS + r;
+    const long long g = slice * qp.rows + row;
+    uint4 raw[4];
+    load_raw_global<true>(qp.x + g * D, row < qp.rows, p, raw);
     uint64_t zp[16];
-    load_transform<ROTATE, true>(qp.x, row, valid, p, m16, zp);
-    if (valid) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float z[8];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) ptx::f2_unpack(zp[4 * i + h], z[2 * h], z[2 * h + 1]);
-        const uint32_t a = ptx::pack_e4m3x4(z[0] * inv, z[1] * inv, z[2] * inv, z[3] * inv);
-        const uint32_t b = ptx::pack_e4m3x4(z[4] * inv, z[5] * inv, z[6] * inv, z[7] * inv);
-        st_v2(qp.codes + row * D + 32 * i + 8 * p, a, b);
-      }
-    }
+    transform_raw<ROTATE>(raw, p, m16, zp);
+    if (row < qp.rows) store_codes(qp.codes + g * D, p, inv, zp);
   }
 }
 

@@ -72,6 +72,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, 
       : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` bytes (a multiple of 16; both addresses
+// 16-byte aligned), completion signalled on `bar` as transaction bytes.  The destination
+// is this CTA's own shared memory.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // ------------------------------------------------------------------------ TMEM
 
 // Allocate `ncols` (power of two >= 32) tensor-memory columns; the base address is

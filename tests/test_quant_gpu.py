@@ -95,7 +95,10 @@ def check_against_oracle(x, signs, gcodes, gdescale, slices=None):
 
 
 @pytest.mark.parametrize("rotate", [False, True])
-@pytest.mark.parametrize("shape", [(1, 1, 1), (1, 2, 7), (2, 3, 33), (1, 4, 1000), (2, 1, 4096)])
+# N <= 2048 runs the shared-memory kernel (cluster sizes 1 .. 8), longer slices the kernel
+# that re-reads its rows from global memory.
+@pytest.mark.parametrize("shape", [(1, 1, 1), (1, 2, 7), (2, 3, 33), (1, 2, 257), (1, 4, 1000),
+                                   (1, 1, 2048), (1, 1, 2049), (2, 1, 4096), (1, 2, 13000)])
 def test_codes_and_descales_match_oracle(cuda_ok, rotate, shape):
     B, H, N = shape
     x = _bf16((B, H, N, 128), seed=N, outlier_rate=1e-3, outlier_scale=50.0)
