@@ -9,7 +9,8 @@ keys, takes its maximum ``m``, forms ``p_j = exp(s_j - m)``, ``l = sum_j p_j`` a
 returns ``O = sum_j p_j v_j / l`` and ``LSE = m + ln l``.  That is the attention formula
 ``softmax(Q K^T / sqrt(d_k)) V`` of the page "FlashAttention (DE)", section
 "Problematik der Standard-Attention", which the pages say FlashAttention reproduces
-exactly.  ``quant_oracle.c`` holds the per-head e4m3 quantisation with the random-sign
+exactly.  ``bwd_oracle.c`` holds the gradients of that formula (dQ, dK, dV for an upstream dO), and
+``quant_oracle.c`` the per-head e4m3 quantisation with the random-sign
 Hadamard rotation of the page "FlashAttention-3 (DE)", section "Niedrige Praezision
 (FP8) mit reduziertem Quantisierungsfehler".  This module only marshals arrays into that
 library.
@@ -46,6 +47,12 @@ def _bind(lib):
     lib.oracle_hadamard.argtypes = [ctypes.c_int64, ctypes.c_void_p]
     lib.oracle_encode_e4m3.restype = ctypes.c_uint8
     lib.oracle_encode_e4m3.argtypes = [ctypes.c_double]
+    lib.oracle_attention_bwd.restype = ctypes.c_int
+    lib.oracle_attention_bwd.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p, ctypes.c_int]
     lib.oracle_quantize_e4m3.restype = ctypes.c_int
     lib.oracle_quantize_e4m3.argtypes = [
         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
@@ -145,6 +152,31 @@ def decode_bf16(bits: int, _library=None) -> float:
 
 def decode_e4m3(code: int, _library=None) -> float:
     return float((_library or _load()).oracle_decode_e4m3(int(code)))
+
+
+def attention_bwd(q, k, v, dout, scale, causal=False, nthreads=0, _library=None):
+    """Gradients (dq, dk, dv) in float64 of O = softmax(scale Q K^T [+ causal mask]) V for
+    the upstream gradient dout.  q, dout: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; float64
+    or bf16 bits (all four of one kind)."""
+    arrs = [np.ascontiguousarray(_as_numpy(t)) for t in (q, k, v, dout)]
+    et = _elem_type(arrs[0])
+    if et == E4M3 or any(_elem_type(a) != et for a in arrs):
+        raise TypeError("q, k, v, dout must all be float64 or all bf16")
+    qa, ka, va, da = arrs
+    B, Hq, Nq, d = qa.shape
+    Bk, Hkv, Nk, dk_ = ka.shape
+    if va.shape != ka.shape or da.shape != qa.shape or Bk != B or dk_ != d:
+        raise ValueError("shape mismatch")
+    dq = np.empty(qa.shape, dtype=np.float64)
+    dk = np.empty(ka.shape, dtype=np.float64)
+    dv = np.empty(ka.shape, dtype=np.float64)
+    rc = (_library or _load()).oracle_attention_bwd(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data, et, B, Hq, Hkv, Nq,
+        Nk, d, float(scale), int(bool(causal)), dq.ctypes.data, dk.ctypes.data,
+        dv.ctypes.data, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_attention_bwd failed with code %d" % rc)
+    return dq, dk, dv
 
 
 def hadamard(d: int, _library=None) -> np.ndarray:

@@ -1,7 +1,8 @@
 """Build the fp64 CPU oracle (test infrastructure) as a shared library.
 
-Compiles ``attn_oracle.c`` (attention) and ``quant_oracle.c`` (fp8 quantisation with
-incoherent processing) with gcc and OpenMP into ``oracle/liboracle.so``.  Only the
+Compiles ``attn_oracle.c`` (attention), ``quant_oracle.c`` (fp8 quantisation with
+incoherent processing) and ``bwd_oracle.c`` (gradients) with gcc and OpenMP into
+``oracle/liboracle.so``.  Only the
 tests, the smoke check and the CPU-baseline leg of ``bench.py`` load that library.
 """
 import os
@@ -10,7 +11,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "attn_oracle.c")
 QUANT_SRC = os.path.join(HERE, "quant_oracle.c")
-SOURCES = (SRC, QUANT_SRC)
+BWD_SRC = os.path.join(HERE, "bwd_oracle.c")
+SOURCES = (SRC, QUANT_SRC, BWD_SRC)
 LIB = os.path.join(HERE, "liboracle.so")
 
 

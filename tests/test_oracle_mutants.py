@@ -1,6 +1,7 @@
 """The pins are not vacuous: each plausible mistake, planted in a copy of the oracle's C
 sources (a dropped term, a wrong sign or index, a transposed operand, a wrong log base, a
-mis-decoded format, a wrong rounding tie rule or scale), makes at least one pin fail,
+mis-decoded format, a wrong rounding tie rule or scale, a dropped gradient term), makes at
+least one pin fail,
 while the real oracle passes them all.  The mistakes are planted on the CPU only, in
 temporary builds."""
 import math
@@ -131,9 +132,23 @@ def pin_quantise_rounding_bound(lib):
     assert dz[0] == 1.0 and not z.any()
 
 
+def pin_bwd_autograd(lib):
+    for causal in (False, True):
+        q, do = rnd((1, 4, 7, 4), 30), rnd((1, 4, 7, 4), 31)
+        k, v = rnd((1, 2, 7, 4), 32), rnd((1, 2, 7, 4), 33)
+        got = oracle.attention_bwd(q, k, v, do, 0.45, causal, _library=lib)
+        tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk.repeat_interleave(2, 1), tv.repeat_interleave(2, 1), is_causal=causal,
+            scale=0.45)
+        o.backward(torch.tensor(do))
+        for g, r in zip(got, (tq.grad, tk.grad, tv.grad)):
+            assert np.abs(g - r.numpy()).max() < 1e-12
+
+
 PINS = [pin_sdpa, pin_bruteforce_lse, pin_gqa, pin_decoders, pin_e4m3_descales,
         pin_hadamard_scipy, pin_encoder_torch, pin_rotation_basis_and_norm,
-        pin_quantise_rounding_bound]
+        pin_quantise_rounding_bound, pin_bwd_autograd]
 
 MUTANTS = {
     "scale_dropped": ("srow[j] = scale * dot;", "srow[j] = dot;"),
@@ -170,6 +185,20 @@ MUTANTS = {
                            "descale[s] = amax > 0.0 ? amax / E4M3_MAX_FINITE : 0.0;"),
     "code_scale_wrong": ("oracle_encode_e4m3(y[e] * E4M3_MAX_FINITE / amax)",
                          "oracle_encode_e4m3(y[e] * 240.0 / amax)"),
+    # gradient oracle
+    "bwd_dq_row_term_dropped": ("acc += s[j] * (dp[j] - term) * ld(k, elem_type, kvoff + j * d + t);",
+                                "acc += s[j] * dp[j] * ld(k, elem_type, kvoff + j * d + t);"),
+    "bwd_dk_row_term_dropped": ("const double ds = p * (dpij - rowterm[gi]);",
+                                "const double ds = p * dpij;"),
+    "bwd_dq_scale_dropped": ("dq[qoff + t] = scale * acc;", "dq[qoff + t] = acc;"),
+    "bwd_dv_reads_q": ("dvr[t] += p * ld(dout, elem_type, qoff + t);",
+                       "dvr[t] += p * ld(q, elem_type, qoff + t);"),
+    "bwd_causal_off_by_one": ("if (causal && j > i) continue;", "if (causal && j >= i) continue;"),
+    "bwd_lse_without_sum": ("lse[gi] = m + log(l);", "lse[gi] = m;"),
+    "bwd_dp_reads_k": ("dp[j] = dot_rows(dout, qoff, v, kvoff + j * d, elem_type, d);",
+                       "dp[j] = dot_rows(dout, qoff, k, kvoff + j * d, elem_type, d);"),
+    "bwd_dk_reads_dout": ("dkr[t] += scale * ds * ld(q, elem_type, qoff + t);",
+                          "dkr[t] += scale * ds * ld(dout, elem_type, qoff + t);"),
 }
 
 
