@@ -1,10 +1,10 @@
 """B200-native fused exact attention forward: Python binding of ``libfa_b200.so``.
 
 The C ABI (``include/fa_b200.h``) is the product; this module only marshals arguments
-into it.  The functions ``fa_fwd``, ``fa_fwd_fp8``, ``fa_quantize_e4m3``,
+into it.  The functions ``fa_fwd``, ``fa_fwd_fp8``, ``fa_bwd``, ``fa_quantize_e4m3``,
 ``fa_check_device_error`` and ``fa_status_string`` have the names and argument order of
 the C entry points and take raw device pointers.  ``forward`` / ``forward_fp8`` /
-``quantize_e4m3`` are conveniences that take CUDA tensors (PyTorch provides device
+``backward`` / ``quantize_e4m3`` are conveniences that take CUDA tensors (PyTorch provides device
 memory and streams only), allocate the outputs and raise on a non-zero status.  Every step of the attention runs in the CUDA kernels; there
 is no CPU or library fallback -- if the shared library is missing, importing a function
 that needs it raises.
@@ -20,7 +20,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
-C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_quantize_e4m3", "fa_check_device_error",
+C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_quantize_e4m3", "fa_check_device_error",
              "fa_selftest_bounded_wait", "fa_status_string", "fa_version")
 
 _lib = None
@@ -45,6 +45,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
         L.fa_fwd_fp8.restype = i
         L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+        L.fa_bwd.restype = i
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
         L.fa_quantize_e4m3.restype = i
         L.fa_quantize_e4m3.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.fa_check_device_error.restype = i
@@ -71,6 +73,13 @@ def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
     """Raw ``fa_fwd_fp8``."""
     return lib().fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
                             descale_q, descale_k, descale_v, stream)
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+           stream) -> int:
+    """Raw ``fa_bwd``."""
+    return lib().fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
+                        causal, stream)
 
 
 def fa_quantize_e4m3(x, signs, x8, descale, B, H, N, d, stream) -> int:
@@ -170,6 +179,33 @@ def forward_fp8(q, k, v, descale_q, descale_k, descale_v, causal=False, scale=No
     if st != FA_OK:
         raise FaError(st, "fa_fwd_fp8")
     return out, lse
+
+
+def backward(q, k, v, o, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None,
+             stream=None):
+    """Gradients (dq, dk, dv) of the bf16 forward for the upstream gradient ``dout``;
+    ``o`` and ``lse`` are that forward's outputs.  All bf16 CUDA tensors in [B, H, N, d]
+    layout (lse fp32 [B, Hq, Nq])."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _check_inputs(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous bf16 CUDA tensor" % name)
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must have q's shape")
+    if (lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous()
+            or tuple(lse.shape) != (B, Hq, Nq)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, Hq, Nq]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq,
+                Nk, d, scale, int(bool(causal)), _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd")
+    return dq, dk, dv
 
 
 def quantize_e4m3(x, signs=None, out=None, descale=None, stream=None):

@@ -16,6 +16,7 @@
 #include <cuda_runtime.h>
 
 #include "fa_b200.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "fa_quant.cuh"
 
@@ -370,6 +371,134 @@ fa_status quantize_common(const void *x, const int8_t *signs, void *x8, float *d
   return quant_launch<false>(qp, s, dev, stream);
 }
 
+template <bool CAUSAL>
+fa_status bwd_launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     const CUtensorMap &tdo, const fa::bwd::BwdParams &p, int grid, int dev,
+                     cudaStream_t stream) {
+  auto kern = fa::bwd::fa_bwd_kernel<CAUSAL>;
+  static std::once_flag attr_once[kMaxDevices];
+  static fa_status attr_st[kMaxDevices];
+  std::call_once(attr_once[dev], [&] {
+    attr_st[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        fa::bwd::SMEM_BYTES) == cudaSuccess
+                       ? FA_OK
+                       : FA_ERR_CUDA;
+  });
+  if (attr_st[dev] != FA_OK) return attr_st[dev];
+  kern<<<grid, fa::bwd::NUM_THREADS, fa::bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Pure host-side checks of fa_bwd; no CUDA call.
+fa_status check_bwd_args(const void *q, const void *k, const void *v, const void *o,
+                         const void *dout, const float *lse, const void *dq, const void *dk,
+                         const void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         float scale, int causal) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  const int64_t bh = static_cast<int64_t>(B) * Hq;
+  const int64_t units = static_cast<int64_t>(B) * Hkv * ((static_cast<int64_t>(Nk) + fa::bwd::BN - 1) / fa::bwd::BN);
+  if (bh > INT32_MAX || units > INT32_MAX || Nq > INT32_MAX - 2 * fa::bwd::BM ||
+      Nk > INT32_MAX - 2 * fa::bwd::BN)
+    return FA_ERR_INVALID_ARG;
+  if (d != fa::bwd::D) return FA_ERR_UNSUPPORTED;
+  if (causal && Nq != Nk) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
+                     const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     cudaStream_t stream) {
+  fa_status st = check_bwd_args(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
+                                causal);
+  if (st != FA_OK) return st;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  DeviceInfo info;
+  st = device_info(dev, &info);
+  if (st != FA_OK) return st;
+  if (info.major != 10 || info.minor != 0) return FA_ERR_UNSUPPORTED;
+  if (!driver_fns().ok) return FA_ERR_CUDA;
+
+  const uint64_t q_bytes = static_cast<uint64_t>(B) * Hq * Nq * d * 2;
+  const uint64_t kv_bytes = static_cast<uint64_t>(B) * Hkv * Nk * d * 2;
+  const uint64_t lse_bytes = static_cast<uint64_t>(B) * Hq * Nq * 4;
+  if (!buffer_ok(q, q_bytes, dev) || !buffer_ok(k, kv_bytes, dev) || !buffer_ok(v, kv_bytes, dev) ||
+      !buffer_ok(o, q_bytes, dev) || !buffer_ok(dout, q_bytes, dev) ||
+      !buffer_ok(lse, lse_bytes, dev) || !buffer_ok(dq, q_bytes, dev) ||
+      !buffer_ok(dk, kv_bytes, dev) || !buffer_ok(dv, kv_bytes, dev))
+    return FA_ERR_INVALID_ARG;
+
+  fa::bwd::BwdParams p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.num_qb = (Nq + fa::bwd::BM - 1) / fa::bwd::BM;
+  p.Npad = p.num_qb * fa::bwd::BM;
+  p.num_kb = (Nk + fa::bwd::BN - 1) / fa::bwd::BN;
+  p.num_units = B * Hkv * p.num_kb;
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  p.dk = static_cast<uint16_t *>(dk);
+  p.dv = static_cast<uint16_t *>(dv);
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_tmap(&tq, q, false, d, Nq, static_cast<uint64_t>(B) * Hq, fa::bwd::BM) ||
+      !encode_tmap(&tdo, dout, false, d, Nq, static_cast<uint64_t>(B) * Hq, fa::bwd::BM) ||
+      !encode_tmap(&tk, k, false, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::bwd::BN) ||
+      !encode_tmap(&tv, v, false, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::bwd::BN))
+    return FA_ERR_INVALID_ARG;
+
+  // Scratch, stream-ordered: the fp32 dQ accumulator and the padded per-row LSE * log2(e)
+  // and D arrays.
+  const uint64_t rows_padded = static_cast<uint64_t>(B) * Hq * p.Npad;
+  const uint64_t acc_bytes = (q_bytes * 2 + 255) / 256 * 256;
+  const uint64_t vec_bytes = (rows_padded * 4 + 255) / 256 * 256;
+  void *ws = nullptr;
+  if (cudaMallocAsync(&ws, acc_bytes + 2 * vec_bytes, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  p.dq_acc = static_cast<float *>(ws);
+  p.l2 = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + acc_bytes);
+  p.dd = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + acc_bytes + vec_bytes);
+
+  st = FA_OK;
+  if (cudaMemsetAsync(p.dq_acc, 0, q_bytes * 2, stream) != cudaSuccess) st = FA_ERR_CUDA;
+  if (st == FA_OK) {
+    const unsigned blocks = static_cast<unsigned>((rows_padded + 7) / 8);
+    fa::bwd::fa_bwd_prep_kernel<<<blocks, 256, 0, stream>>>(
+        static_cast<const uint16_t *>(o), static_cast<const uint16_t *>(dout), lse,
+        const_cast<float *>(p.l2), const_cast<float *>(p.dd), static_cast<long long>(rows_padded),
+        Nq, p.Npad);
+    if (cudaGetLastError() != cudaSuccess) st = FA_ERR_CUDA;
+  }
+  if (st == FA_OK) {
+    const int grid = p.num_units < info.sms ? p.num_units : info.sms;
+    st = causal ? bwd_launch<true>(tq, tk, tv, tdo, p, grid, dev, stream)
+                : bwd_launch<false>(tq, tk, tv, tdo, p, grid, dev, stream);
+  }
+  if (st == FA_OK) {
+    const long long n4 = static_cast<long long>(q_bytes / 2 / 4);
+    fa::bwd::fa_bwd_dq_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
+        p.dq_acc, static_cast<uint16_t *>(dq), n4, scale);
+    if (cudaGetLastError() != cudaSuccess) st = FA_ERR_CUDA;
+  }
+  if (cudaFreeAsync(ws, stream) != cudaSuccess && st == FA_OK) st = FA_ERR_CUDA;
+  return st;
+}
+
 }  // namespace
 
 extern "C" {
@@ -395,6 +524,13 @@ fa_status fa_quantize_e4m3(const void *x, const int8_t *signs, void *x8, float *
                            int H, int N, int d, fa_stream_t stream) {
   return quantize_common(x, signs, x8, descale, B, H, N, d,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq,
+                 int Nk, int d, float scale, int causal, fa_stream_t stream) {
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_check_device_error(fa_stream_t stream) {

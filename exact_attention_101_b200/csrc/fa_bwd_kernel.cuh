@@ -1,0 +1,566 @@
+// fa_bwd_kernel.cuh -- backward pass of exact attention on sm_100a.
+//
+// The pages state that FlashAttention keeps no N x N matrix for the backward pass: it
+// computes the attention again from Q, K, V and the saved row log-sum-exp ("Flash
+// Attention" page, section "Zentrale technische Innovationen", the recomputation bullet).
+// For O = P V, P = softmax(S) row by row, S = scale * Q K^T (+ causal mask) and an
+// upstream gradient dO, the gradients are
+//
+//   P_ij  = exp(scale * q_i . k_j - LSE_i)        (recomputed from the forward's LSE)
+//   dV    = P^T dO
+//   dP    = dO V^T
+//   dS_ij = P_ij (dP_ij - D_i),  D_i = sum_t dO_it O_it  (= sum_j P_ij dP_ij)
+//   dK    = scale * dS^T Q
+//   dQ    = scale * dS K
+//
+// Work decomposition: a unit is one block of BN = 128 keys of one (batch, K/V head); its
+// CTA keeps K_j and V_j in shared memory and dK_j, dV_j in tensor memory for the whole
+// unit, and walks every query head of the group and every block of BM = 64 queries (from
+// the diagonal on under the causal mask).  Per step five tcgen05 MMAs:
+//
+//   S^T  = K_j Q_i^T      M=128 keys, N=64 queries, K=128 (SS, both K-major)
+//   dP^T = V_j dO_i^T     same shape
+//   dQ^T = K_j^T dS^T     M=128 head dims, N=64 queries, K=128 keys (SS, both MN-major)
+//   dV  += P^T dO_i       M=128 keys, N=128, K=64 queries (A = P^T from tensor memory)
+//   dK  += dS^T Q_i       same shape (A = dS^T from tensor memory)
+//
+// dQ^T goes through tensor memory to fp32 reduction-adds into a zeroed global accumulator
+// (each query block receives one contribution per key block); a last kernel scales it
+// and rounds to bf16.  dK, dV leave once per unit, with no atomics: the group's query heads
+// are summed inside the unit.
+//
+// Tensor memory (512 columns): S^T of step buffer b at b*128 (64 columns; after the
+// softmax, P^T and dS^T as packed bf16), dP^T of buffer b at b*128 + 64 (then dQ^T of the
+// same step), dV at 256, dK at 384.  Two step buffers let the softmax of step i+1 run
+// while the tensor core works on step i.
+//
+// Warps: 0-3 and 4-7 are the "softmax" warpgroups (thread = key row; warpgroup h takes
+// queries 32h .. 32h+31 of the step, and at the end of a unit writes dV (h=0) or dK
+// (h=1)); 8-11 drain dQ^T (thread = head dimension); 12 allocates tensor memory and issues
+// the MMAs; 13 issues the TMA copies.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa_fwd_kernel.cuh"  // device error word and bounded waits
+#include "sm100.cuh"
+
+namespace fa {
+namespace bwd {
+
+constexpr int D = 128;
+constexpr int BN = 128;                  // keys per unit (tensor-memory lanes)
+constexpr int BM = 64;                   // queries per step
+constexpr int NUM_THREADS = 448;         // 14 warps
+constexpr int DRAIN_WARP0 = 8;
+constexpr int MMA_WARP = 12;
+constexpr int TMA_WARP = 13;
+constexpr int ROW_BYTES = D * 2;
+constexpr int KV_BOX = BN * 128;         // one 128-byte-wide TMA box of a K or V tile
+constexpr int KV_TILE = 2 * KV_BOX;      // 32 KB
+constexpr int Q_BOX = BM * 128;
+constexpr int Q_TILE = 2 * Q_BOX;        // 16 KB
+constexpr int DS_TILE = BN * BM * 2;     // dS^T [keys][queries] bf16, 128-byte rows: 16 KB
+constexpr int VEC_BYTES = 2 * BM * 4;    // per step: LSE*log2(e) and D for BM queries
+
+// Shared memory map (offsets from a 1024-aligned base).
+constexpr int K_OFF = 0;
+constexpr int V_OFF = K_OFF + KV_TILE;
+constexpr int Q_OFF = V_OFF + KV_TILE;   // 2 step buffers
+constexpr int DO_OFF = Q_OFF + 2 * Q_TILE;
+constexpr int DS_OFF = DO_OFF + 2 * Q_TILE;
+constexpr int VEC_OFF = DS_OFF + 2 * DS_TILE;
+constexpr int BAR_OFF = VEC_OFF + 2 * VEC_BYTES;
+constexpr int NUM_BARS = 17;
+constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
+constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// Tensor-memory columns.
+__host__ __device__ constexpr uint32_t s_col(int b) { return b * 128; }
+__host__ __device__ constexpr uint32_t dp_col(int b) { return b * 128 + 64; }
+constexpr uint32_t DV_COL = 256, DK_COL = 384;
+
+constexpr uint32_t IDESC_S = ptx::make_idesc(1, BN, BM, 0);          // S^T, dP^T
+constexpr uint32_t IDESC_ACC = ptx::make_idesc(1, BN, D, 1);         // dV, dK
+constexpr uint32_t IDESC_DQ = ptx::make_idesc_ab(1, D, BM, 1, 1);    // dQ^T
+
+constexpr uint32_t ERR_WAIT_BWD = 1u << 6;
+
+struct BwdParams {
+  const float *l2;     // [B*Hq, Npad]: LSE * log2(e), +inf past Nq
+  const float *dd;     // [B*Hq, Npad]: D = rowsum(dO o O), 0 past Nq
+  float *dq_acc;       // [B*Hq, Nq, D] fp32, zeroed before the launch
+  uint16_t *dk, *dv;   // bf16 [B*Hkv, Nk, D]
+  int B, Hq, Hkv, Nq, Nk, Npad, group;
+  int num_kb;          // ceil(Nk / BN)
+  int num_qb;          // ceil(Nq / BM)
+  int num_units;       // B * Hkv * num_kb
+  float scale_log2;    // scale * log2(e)
+  float scale;
+};
+
+struct BUnit {
+  int bhk;    // b * Hkv + hk
+  int b, hk;
+  int j;      // key block
+  int i0;     // first query block visited
+  int nq;     // query blocks visited per query head
+  int steps;  // group * nq
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ BUnit decode_unit(const BwdParams &p, int u) {
+  BUnit w;
+  w.bhk = u / p.num_kb;
+  w.j = u % p.num_kb;
+  w.b = w.bhk / p.Hkv;
+  w.hk = w.bhk % p.Hkv;
+  // Under the causal mask query i sees key j only if j <= i: blocks of queries that end
+  // before the key block starts are skipped.
+  w.i0 = CAUSAL ? (w.j * BN) / BM : 0;
+  w.nq = p.num_qb - w.i0;
+  w.steps = p.group * w.nq;
+  return w;
+}
+
+// (query head row index b*Hq + hq, query block) of step s of unit w.
+__device__ __forceinline__ void step_coords(const BwdParams &p, const BUnit &w, int s, int &bh,
+                                            int &i) {
+  bh = w.b * p.Hq + w.hk * p.group + s / w.nq;
+  i = w.i0 + s % w.nq;
+}
+
+struct BBars {
+  uint32_t base;
+  __device__ uint32_t kv_full() const { return base; }
+  __device__ uint32_t kv_empty() const { return base + 8u; }
+  __device__ uint32_t q_full(int b) const { return base + 8u * (2 + b); }
+  __device__ uint32_t q_empty(int b) const { return base + 8u * (4 + b); }
+  __device__ uint32_t sdp_full(int b) const { return base + 8u * (6 + b); }
+  __device__ uint32_t ds_full(int b) const { return base + 8u * (8 + b); }
+  __device__ uint32_t dq_full(int b) const { return base + 8u * (10 + b); }
+  __device__ uint32_t dq_empty(int b) const { return base + 8u * (12 + b); }
+  __device__ uint32_t acc_full() const { return base + 8u * 14; }
+  __device__ uint32_t acc_empty() const { return base + 8u * 15; }
+  __device__ uint32_t drain() const { return base + 8u * 16; }
+};
+
+// ---------------------------------------------------------------------------- producer
+
+template <bool CAUSAL>
+__device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                          const CUtensorMap *tmDO, const BwdParams &p, uint32_t smem,
+                          const BBars &bar, volatile uint32_t *abort_flag) {
+  ptx::prefetch_tmap(tmQ);
+  ptx::prefetch_tmap(tmK);
+  ptx::prefetch_tmap(tmV);
+  ptx::prefetch_tmap(tmDO);
+  uint32_t units_issued = 0, steps_issued = 0;
+  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    const BUnit w = decode_unit<CAUSAL>(p, u);
+    if (!wait_phase(bar.kv_empty(), (units_issued & 1u) ^ 1u, abort_flag, ERR_WAIT_BWD))
+      goto drain;
+    ptx::mbar_arrive_expect_tx(bar.kv_full(), 2 * KV_TILE);
+#pragma unroll
+    for (int bx = 0; bx < 2; ++bx) {
+      ptx::tma_load_3d(smem + K_OFF + bx * KV_BOX, tmK, bar.kv_full(), bx * 64, w.j * BN, w.bhk);
+      ptx::tma_load_3d(smem + V_OFF + bx * KV_BOX, tmV, bar.kv_full(), bx * 64, w.j * BN, w.bhk);
+    }
+    ++units_issued;
+    for (int s = 0; s < w.steps; ++s) {
+      const int b = steps_issued & 1u;
+      const uint32_t use = steps_issued >> 1;
+      if (!wait_phase(bar.q_empty(b), (use & 1u) ^ 1u, abort_flag, ERR_WAIT_BWD)) goto drain;
+      int bh, i;
+      step_coords(p, w, s, bh, i);
+      ptx::mbar_arrive_expect_tx(bar.q_full(b), 2 * Q_TILE + VEC_BYTES);
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx) {
+        ptx::tma_load_3d(smem + Q_OFF + b * Q_TILE + bx * Q_BOX, tmQ, bar.q_full(b), bx * 64,
+                         i * BM, bh);
+        ptx::tma_load_3d(smem + DO_OFF + b * Q_TILE + bx * Q_BOX, tmDO, bar.q_full(b), bx * 64,
+                         i * BM, bh);
+      }
+      const long long voff = static_cast<long long>(bh) * p.Npad + i * BM;
+      ptx::bulk_load(smem + VEC_OFF + b * VEC_BYTES, p.l2 + voff, BM * 4, bar.q_full(b));
+      ptx::bulk_load(smem + VEC_OFF + b * VEC_BYTES + BM * 4, p.dd + voff, BM * 4,
+                     bar.q_full(b));
+      ++steps_issued;
+    }
+  }
+drain:
+  // Let every copy this thread started land before the CTA exits (immediate on the normal
+  // path, where the consumers have already waited for them).
+  if (units_issued > 0) drain_wait(bar.kv_full(), (units_issued - 1) & 1u);
+  for (uint32_t b = 0; b < 2; ++b)
+    if (steps_issued > b) {
+      const uint32_t last = b + 2 * ((steps_issued - 1 - b) / 2);
+      drain_wait(bar.q_full(b), (last >> 1) & 1u);
+    }
+}
+
+// ---------------------------------------------------------------------------- MMA issuer
+
+// S^T or dP^T: A = K_j or V_j (128 rows, two 128-byte column boxes, K-major), B = Q_i or
+// dO_i (64 rows, two boxes, K-major); K = 128 head dims in steps of 16.
+__device__ __forceinline__ void issue_sdp(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    constexpr uint32_t step = 32;  // bytes along the head dim per MMA
+    const uint32_t kb = kk * step;
+    const uint32_t aoff = ((kb / 128) * KV_BOX + (kb % 128)) >> 4;
+    const uint32_t boff = ((kb / 128) * Q_BOX + (kb % 128)) >> 4;
+    ptx::mma_bf16_ss_elect(tmem_d, a_desc + aoff, b_desc + boff, IDESC_S, kk > 0 ? 1u : 0u);
+  }
+}
+
+// dV += P^T dO_i or dK += dS^T Q_i: A from tensor memory (keys x 64 queries as packed
+// bf16; queries 0-31 at columns 0-15 (+16 for dS), queries 32-63 at 32-47), B = dO_i or
+// Q_i read MN-major (64 query rows of 128-byte head-dim boxes); K = 64 queries in steps
+// of 16 (8 packed columns, 16 rows of 128 bytes).
+__device__ __forceinline__ void issue_acc(uint32_t tmem_d, uint32_t tmem_a, uint64_t b_desc,
+                                          uint32_t accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < BM / 16; ++kk) {
+    const uint32_t a = tmem_a + (kk / 2) * 32 + (kk % 2) * 8;
+    const uint32_t boff = (kk * 16 * 128) >> 4;
+    ptx::mma_bf16_ts_elect(tmem_d, a, b_desc + boff, IDESC_ACC, kk > 0 ? 1u : accumulate);
+  }
+}
+
+// dQ^T = K_j^T dS^T: A = K_j read MN-major (M = head dims, two boxes 16 KB apart), B = dS^T
+// read MN-major (N = 64 queries in one 128-byte row); K = 128 keys in steps of 16 rows.
+__device__ __forceinline__ void issue_dq(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc) {
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk) {
+    const uint32_t off = (kk * 16 * 128) >> 4;
+    ptx::mma_bf16_ss_elect(tmem_d, a_desc + off, b_desc + off, IDESC_DQ, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <bool CAUSAL>
+__device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const BBars &bar,
+                         volatile uint32_t *abort_flag) {
+  const uint64_t k_a = ptx::smem_desc_sw128(smem + K_OFF, 16, 1024);
+  const uint64_t v_a = ptx::smem_desc_sw128(smem + V_OFF, 16, 1024);
+  const uint64_t k_t = ptx::smem_desc_sw128(smem + K_OFF, KV_BOX, 1024);
+  auto wait = [&](uint32_t b, uint32_t parity) {
+    const bool ok = wait_phase(b, parity, abort_flag, ERR_WAIT_BWD);
+    return __all_sync(0xffffffffu, ok);
+  };
+  // S^T and dP^T of global step g (buffer g & 1).
+  auto start_step = [&](uint32_t g) {
+    const int b = g & 1u;
+    const uint32_t use = g >> 1;
+    if (!wait(bar.q_full(b), use & 1u)) return false;
+    ptx::tc_fence_after();
+    issue_sdp(tmem + s_col(b), k_a, ptx::smem_desc_sw128(smem + Q_OFF + b * Q_TILE, 16, 1024));
+    // dP^T lands where dQ^T of this buffer's previous step was: wait for its drain.
+    if (!wait(bar.dq_empty(b), (use & 1u) ^ 1u)) return false;
+    ptx::tc_fence_after();
+    issue_sdp(tmem + dp_col(b), v_a, ptx::smem_desc_sw128(smem + DO_OFF + b * Q_TILE, 16, 1024));
+    ptx::mma_commit_elect(bar.sdp_full(b));
+    return true;
+  };
+  uint32_t gm = 0, unit_it = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++unit_it) {
+    const BUnit w = decode_unit<CAUSAL>(p, u);
+    if (!wait(bar.kv_full(), unit_it & 1u)) break;
+    ptx::tc_fence_after();
+    for (int s = 0; s < 2 && s < w.steps && ok; ++s) ok = start_step(gm + s);
+    for (int s = 0; s < w.steps && ok; ++s) {
+      const uint32_t g = gm + s;
+      const int b = g & 1u;
+      const uint32_t use = g >> 1;
+      if (!(ok = wait(bar.ds_full(b), use & 1u))) break;
+      ptx::tc_fence_after();
+      issue_dq(tmem + dp_col(b), k_t,
+               ptx::smem_desc_sw128(smem + DS_OFF + b * DS_TILE, DS_TILE, 1024));
+      ptx::mma_commit_elect(bar.dq_full(b));
+      if (s == 0) {
+        if (!(ok = wait(bar.acc_empty(), (unit_it & 1u) ^ 1u))) break;
+        ptx::tc_fence_after();
+      }
+      issue_acc(tmem + DV_COL, tmem + s_col(b),
+                ptx::smem_desc_sw128(smem + DO_OFF + b * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
+      issue_acc(tmem + DK_COL, tmem + s_col(b) + 16,
+                ptx::smem_desc_sw128(smem + Q_OFF + b * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
+      ptx::mma_commit_elect(bar.q_empty(b));
+      if (s == w.steps - 1) {
+        ptx::mma_commit_elect(bar.acc_full());
+        ptx::mma_commit_elect(bar.kv_empty());
+      }
+      if (s + 2 < w.steps) ok = start_step(g + 2);
+    }
+    gm += w.steps;
+  }
+  // Wait until every MMA issued by this warp has finished before tensor memory is freed.
+  ptx::mma_commit_elect(bar.drain());
+  drain_wait(bar.drain(), 0);
+}
+
+// ---------------------------------------------------------------------------- softmax
+
+// Recompute P^T and form dS^T for one step: this thread owns key row `key` and queries
+// q0 .. q0+31 (q0 = i*BM + 32h).  Writes P^T and dS^T as packed bf16 into its own 32
+// columns of the S^T buffer and dS^T into the shared-memory tile (128-byte swizzle: the
+// 16-byte chunk c of row r sits at chunk c ^ (r % 8)).
+template <bool CAUSAL>
+__device__ __forceinline__ void softmax_step(const BwdParams &p, uint32_t tmem_row, uint32_t smem,
+                                             int b, int h, int row, int key, int q0,
+                                             bool need_mask) {
+  uint32_t sr[2][16], dr[2][16];
+  ptx::tmem_ld16(tmem_row + s_col(b) + h * 32, sr[0]);
+  ptx::tmem_ld16(tmem_row + s_col(b) + h * 32 + 16, sr[1]);
+  ptx::tmem_ld16(tmem_row + dp_col(b) + h * 32, dr[0]);
+  ptx::tmem_ld16(tmem_row + dp_col(b) + h * 32 + 16, dr[1]);
+  ptx::tmem_wait_ld();
+  ptx::reg_fence16(sr[0]);
+  ptx::reg_fence16(sr[1]);
+  ptx::reg_fence16(dr[0]);
+  ptx::reg_fence16(dr[1]);
+  const float *vec = reinterpret_cast<const float *>(
+      __cvta_shared_to_generic(smem + VEC_OFF + b * VEC_BYTES));
+  const float4 *l2v = reinterpret_cast<const float4 *>(vec + h * 32);
+  const float4 *ddv = reinterpret_cast<const float4 *>(vec + BM + h * 32);
+  uint32_t pp[16], pd[16];
+#pragma unroll
+  for (int c4 = 0; c4 < 8; ++c4) {
+    const float4 l4 = l2v[c4], d4 = ddv[c4];
+    const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+    float pv[4], sv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = c4 * 4 + e;
+      const float s = __uint_as_float(sr[c / 16][c % 16]);
+      const float dpv = __uint_as_float(dr[c / 16][c % 16]);
+      float pe = ptx::ex2(fmaf(s, p.scale_log2, -lv[e]));
+      if (need_mask && (key >= p.Nk || (CAUSAL && key > q0 + c))) pe = 0.f;
+      pv[e] = pe;
+      sv[e] = pe * (dpv - dv[e]);
+    }
+    pp[c4 * 2] = ptx::pack_bf16x2(pv[0], pv[1]);
+    pp[c4 * 2 + 1] = ptx::pack_bf16x2(pv[2], pv[3]);
+    pd[c4 * 2] = ptx::pack_bf16x2(sv[0], sv[1]);
+    pd[c4 * 2 + 1] = ptx::pack_bf16x2(sv[2], sv[3]);
+  }
+  ptx::tmem_st16(tmem_row + s_col(b) + h * 32, pp);
+  ptx::tmem_st16(tmem_row + s_col(b) + h * 32 + 16, pd);
+  const uint32_t ds_row = smem + DS_OFF + b * DS_TILE + row * 128;
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const uint32_t chunk = static_cast<uint32_t>(h * 4 + cc) ^ static_cast<uint32_t>(row & 7);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ds_row + chunk * 16),
+                 "r"(pd[cc * 4]), "r"(pd[cc * 4 + 1]), "r"(pd[cc * 4 + 2]), "r"(pd[cc * 4 + 3])
+                 : "memory");
+  }
+  ptx::tmem_wait_st();
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+}
+
+template <bool CAUSAL>
+__device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const BBars &bar,
+                             volatile uint32_t *abort_flag) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = warp / 4;                     // query half of the step
+  const int row = (warp % 4) * 32 + lane;     // key row within the block
+  const uint32_t tmem_row = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+  uint32_t gs = 0, unit_it = 0;
+  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++unit_it) {
+    const BUnit w = decode_unit<CAUSAL>(p, u);
+    const int key = w.j * BN + row;
+    for (int s = 0; s < w.steps; ++s) {
+      const uint32_t g = gs + s;
+      const int b = g & 1u;
+      if (!wait_phase(bar.sdp_full(b), (g >> 1) & 1u, abort_flag, ERR_WAIT_BWD)) return;
+      ptx::tc_fence_after();
+      int bh, i;
+      step_coords(p, w, s, bh, i);
+      const int q0 = i * BM + h * 32;
+      // masking is needed on the key tail block and, causally, where the block of
+      // queries starts before the last key of the block
+      const bool need_mask = (w.j * BN + BN > p.Nk) || (CAUSAL && q0 < w.j * BN + BN - 1);
+      softmax_step<CAUSAL>(p, tmem_row, smem, b, h, row, key, q0, need_mask);
+      ptx::mbar_arrive(bar.ds_full(b));
+    }
+    gs += w.steps;
+    // Unit epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK, as bf16 rows.
+    if (!wait_phase(bar.acc_full(), unit_it & 1u, abort_flag, ERR_WAIT_BWD)) return;
+    ptx::tc_fence_after();
+    const float mult = h == 0 ? 1.f : p.scale;
+    uint16_t *out = (h == 0 ? p.dv : p.dk) + (static_cast<long long>(w.bhk) * p.Nk + key) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t r[16];
+      ptx::tmem_ld16(tmem_row + (h == 0 ? DV_COL : DK_COL) + c * 16, r);
+      ptx::tmem_wait_ld();
+      ptx::reg_fence16(r);
+      uint32_t o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        o[e] = ptx::pack_bf16x2(__uint_as_float(r[2 * e]) * mult,
+                                __uint_as_float(r[2 * e + 1]) * mult);
+      if (key < p.Nk) {
+        uint4 *dst = reinterpret_cast<uint4 *>(out + c * 16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    }
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(bar.acc_empty());
+  }
+}
+
+// ---------------------------------------------------------------------------- dQ drain
+
+// Thread = head dimension t: after each step's dQ^T lands, read its 64 query columns and
+// add them to dq_acc[bh, q, t] (32 consecutive t per warp: one 128-byte reduction per
+// query).
+template <bool CAUSAL>
+__device__ void dq_role(const BwdParams &p, uint32_t tmem, const BBars &bar,
+                        volatile uint32_t *abort_flag) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = (warp % 4) * 32 + lane;
+  const uint32_t tmem_row = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+  uint32_t gd = 0;
+  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    const BUnit w = decode_unit<CAUSAL>(p, u);
+    for (int s = 0; s < w.steps; ++s) {
+      const uint32_t g = gd + s;
+      const int b = g & 1u;
+      if (!wait_phase(bar.dq_full(b), (g >> 1) & 1u, abort_flag, ERR_WAIT_BWD)) return;
+      ptx::tc_fence_after();
+      uint32_t r[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::tmem_ld16(tmem_row + dp_col(b) + c * 16, r[c]);
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::reg_fence16(r[c]);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar.dq_empty(b));
+      int bh, i;
+      step_coords(p, w, s, bh, i);
+      const int q0 = i * BM;
+      float *dst = p.dq_acc + (static_cast<long long>(bh) * p.Nq + q0) * D + t;
+      const int nvalid = min(BM, p.Nq - q0);
+#pragma unroll
+      for (int c = 0; c < BM; ++c)
+        if (c < nvalid) ptx::red_add_f32(dst + static_cast<long long>(c) * D,
+                                         __uint_as_float(r[c / 16][c % 16]));
+    }
+    gd += w.steps;
+  }
+}
+
+// ---------------------------------------------------------------------------- kernels
+
+template <bool CAUSAL>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_addr(smem_raw);
+  const uint32_t smem = (raw + 1023u) & ~1023u;  // 1024-aligned for 128-byte swizzle
+  uint8_t *smem_gen = smem_raw + (smem - raw);
+  const BBars bar{smem + BAR_OFF};
+  uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + CTL_OFF);
+  volatile uint32_t *tmem_slot = ctl;
+  volatile uint32_t *abort_flag = ctl + 1;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar.kv_full(), 1);
+    ptx::mbar_init(bar.kv_empty(), 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar.q_full(b), 1);
+      ptx::mbar_init(bar.q_empty(b), 1);
+      ptx::mbar_init(bar.sdp_full(b), 1);
+      ptx::mbar_init(bar.ds_full(b), 256);
+      ptx::mbar_init(bar.dq_full(b), 1);
+      ptx::mbar_init(bar.dq_empty(b), 128);
+    }
+    ptx::mbar_init(bar.acc_full(), 1);
+    ptx::mbar_init(bar.acc_empty(), 256);
+    ptx::mbar_init(bar.drain(), 1);
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+  }
+  if (warp == MMA_WARP) {
+    ptx::tmem_alloc(ptx::smem_addr(ctl), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < DRAIN_WARP0) {
+    softmax_role<CAUSAL>(p, smem, tmem, bar, abort_flag);
+  } else if (warp < MMA_WARP) {
+    dq_role<CAUSAL>(p, tmem, bar, abort_flag);
+  } else if (warp == MMA_WARP) {
+    mma_role<CAUSAL>(p, smem, tmem, bar, abort_flag);
+    __syncwarp();
+  } else if (warp == TMA_WARP) {
+    if (lane == 0) load_role<CAUSAL>(&tmQ, &tmK, &tmV, &tmDO, p, smem, bar, abort_flag);
+    __syncwarp();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Per query row: D = sum_t dO_t O_t (fp32 from bf16) and LSE * log2(e), into arrays
+// padded to Npad rows per (batch, head) (D = 0, LSE = +inf on the padding, so padded
+// queries contribute nothing).  One warp per row, 4 elements per lane (D = 128).
+__global__ void fa_bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_t *__restrict__ dout,
+                                   const float *__restrict__ lse, float *__restrict__ l2,
+                                   float *__restrict__ dd, long long rows_padded, int Nq, int Npad) {
+  const long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (r >= rows_padded) return;
+  const long long bh = r / Npad;
+  const int q = static_cast<int>(r - bh * Npad);
+  if (q >= Nq) {
+    if (lane == 0) {
+      l2[r] = __int_as_float(0x7f800000);
+      dd[r] = 0.f;
+    }
+    return;
+  }
+  const long long row = bh * Nq + q;
+  const uint2 a = reinterpret_cast<const uint2 *>(o + row * D)[lane];
+  const uint2 g = reinterpret_cast<const uint2 *>(dout + row * D)[lane];
+  auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
+  auto hi = [](uint32_t x) { return __uint_as_float(x & 0xffff0000u); };
+  float s = lo(a.x) * lo(g.x) + hi(a.x) * hi(g.x) + lo(a.y) * lo(g.y) + hi(a.y) * hi(g.y);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) {
+    dd[r] = s;
+    l2[r] = lse[row] * 1.4426950408889634f;
+  }
+}
+
+// dQ = scale * dq_acc, rounded to bf16; 4 elements per thread.
+__global__ void fa_bwd_dq_kernel(const float *__restrict__ acc, uint16_t *__restrict__ dq,
+                                 long long n4, float scale) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = reinterpret_cast<const float4 *>(acc)[i];
+  reinterpret_cast<uint2 *>(dq)[i] =
+      make_uint2(ptx::pack_bf16x2(v.x * scale, v.y * scale), ptx::pack_bf16x2(v.z * scale, v.w * scale));
+}
+
+}  // namespace bwd
+}  // namespace fa

@@ -177,6 +177,23 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, uint32_t M
          | ((M >> 4) << 24);       // M / 16
 }
 
+// The same with the major-ness of A chosen too (a_mn_major = 1: A stored MN-major).
+__host__ __device__ constexpr uint32_t make_idesc_ab(uint32_t ab_format, uint32_t M, uint32_t N,
+                                                     uint32_t a_mn_major, uint32_t b_mn_major) {
+  return make_idesc(ab_format, M, N, b_mn_major) | (a_mn_major << 15);
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (the
+// tensor core reading them as an MMA operand).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// fp32 reduction-add to global memory (no return value).
+__device__ __forceinline__ void red_add_f32(float *p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {

@@ -99,6 +99,38 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
                      const float *descale_v, fa_stream_t stream);
 
 /*
+ * Backward pass of the bf16 forward above: the gradients of O with respect to Q, K and V
+ * for an upstream gradient dO.  The page "Flash Attention" (section "Zentrale technische
+ * Innovationen", the recomputation bullet) states that FlashAttention does not keep the
+ * attention matrix for the backward pass but computes it again; this call recomputes
+ * P = exp(scale * Q K^T - LSE) tile by tile from Q, K and the forward's LSE and forms
+ *
+ *     dV = P^T dO,   dS = P o (dO V^T - D),   D_i = sum_t dO_it O_it,
+ *     dQ = scale * dS K,   dK = scale * dS^T Q
+ *
+ * (o is the Hadamard product; D_i equals sum_j P_ij (dO V^T)_ij).  Under grouped heads
+ * the dK and dV of a K/V head sum the contributions of the query heads that read it.
+ *
+ *   q, k, v     the forward's inputs, bf16, layout as for fa_fwd
+ *   o, lse      the forward's outputs for these inputs (o bf16 [B,Hq,Nq,d], lse fp32)
+ *   dout        bf16 [B,Hq,Nq,d], the gradient of the loss with respect to o
+ *   dq          bf16 [B,Hq,Nq,d] out;  dk, dv  bf16 [B,Hkv,Nk,d] out
+ *   B, Hq, Hkv, Nq, Nk, scale, causal   as for fa_fwd;  d must be 128
+ *
+ * All pointers 16-byte aligned (lse 4-byte).  The outputs must not overlap the inputs.
+ * Scratch: the call allocates B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes on `stream` with
+ * cudaMallocAsync (an fp32 dQ accumulator and two per-row vectors) and frees it on the
+ * same stream with cudaFreeAsync.  dQ is summed with fp32 atomic additions, so its last
+ * bits may differ between runs.  Enqueues a memset and three kernels.  Returns FA_OK once
+ * enqueued; FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (d != 128, causal with Nq != Nk,
+ * GPU not sm_100) with nothing enqueued; FA_ERR_CUDA if the scratch allocation or a launch
+ * failed.
+ */
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv,
+                 int Nq, int Nk, int d, float scale, int causal, fa_stream_t stream);
+
+/*
  * Per-(batch, head) fp8-e4m3 quantisation of a bf16 tensor, optionally with incoherent
  * processing: the page "FlashAttention-3 (DE)", section "Niedrige Praezision (FP8) mit
  * reduziertem Quantisierungsfehler", multiplies the query and key vectors by a random

@@ -115,3 +115,29 @@ def test_quantize_invalid_arguments(kw):
 @pytest.mark.parametrize("d", [64, 256])
 def test_quantize_supports_head_dim_128_only(d):
     assert fa.fa_quantize_e4m3(A, None, A, A, 1, 2, 64, d, None) == fa.FA_ERR_UNSUPPORTED
+
+
+BWD_OK = dict(q=A, k=A, v=A, o=A, dout=A, lse=A, dq=A, dk=A, dv=A, B=1, Hq=4, Hkv=2, Nq=256,
+              Nk=256, d=128, scale=0.088, causal=0)
+
+
+def bwd_call(**kw):
+    a = dict(BWD_OK)
+    a.update(kw)
+    return fa.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["dout"], a["lse"], a["dq"], a["dk"],
+                     a["dv"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["d"], a["scale"],
+                     a["causal"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=0), dict(o=0), dict(dout=0), dict(lse=0), dict(dq=0), dict(dk=0), dict(dv=0),
+    dict(dout=A + 8), dict(dq=A + 4), dict(lse=A + 2), dict(B=0), dict(Nq=0), dict(Nk=0),
+    dict(Hq=3, Hkv=2), dict(causal=2), dict(scale=0.0), dict(scale=float("nan")),
+])
+def test_bwd_invalid_arguments(kw):
+    assert bwd_call(**kw) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(d=64), dict(d=256), dict(causal=1, Nq=128, Nk=256)])
+def test_bwd_unsupported_configurations(kw):
+    assert bwd_call(**kw) == fa.FA_ERR_UNSUPPORTED
