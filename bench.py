@@ -213,6 +213,28 @@ def oracle_timed_sample(w, inp, n_rows, seed=0):
     return _row_flops(w, rows) / dt / 1e12, desc, oracle.max_threads(), dt
 
 
+def oracle_bwd_sample(w, inp, target_s):
+    """Time the fp64 gradient oracle on the first n queries and keys of the first K/V head
+    and its query heads (n doubled until the run takes at least a quarter of target_s).
+    Returns (TFLOP/s, description, threads, seconds)."""
+    import oracle
+    g = w.Hq // w.Hkv
+    n, dt = 256, 0.0
+    while True:
+        sl = lambda t, h: t[:1, :h, :n].contiguous()
+        t0 = time.perf_counter()
+        oracle.attention_bwd(sl(inp.q, g), sl(inp.k, 1), sl(inp.v, 1), sl(inp.dout, g), w.scale,
+                             w.causal)
+        dt = time.perf_counter() - t0
+        if dt >= 0.25 * target_s or 2 * n > w.N:
+            break
+        n *= 2
+    flops = 2.5 * 4.0 * g * n * n * w.d / (2 if w.causal else 1)
+    desc = ("gradients of the first %d queries and keys of batch 0, K/V head 0 and its %d "
+            "query head(s) of workload %s, fp64" % (n, g, w.name))
+    return flops / dt / 1e12, desc, oracle.max_threads(), dt
+
+
 def oracle_sample_rate(w, inp, target_s, seed=0):
     """Calibrate, then time one sample of about target_s seconds."""
     n = oracle_calibrate(w, inp, target_s, seed)
@@ -253,8 +275,14 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     # Incoherent-processing workloads quantise their bf16 Q, K (rotated) and V on the GPU
     # every step, then run the fp8 kernel: 3 quantisation kernels + 1 attention kernel.
-    launches_per_step = 4 if w.rotate else 1
+    launches_per_step = 4 if w.rotate else (3 if w.kind == "bwd" else 1)
     split = None
+    if w.kind == "bwd":
+        # The forward's O and LSE, computed once before timing; each step is one backward.
+        host += [inp.dout]
+        dout = inp.dout.to(dev)
+        fa.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if w.rotate:
         host.append(inp.signs)
         signs = inp.signs.to(dev)
@@ -280,6 +308,9 @@ def run_ours(args):
                            lse=lse)
             if ev:
                 ev[2].record(stream)
+        elif w.kind == "bwd":
+            fa.backward(q, k, v, o, lse, dout, causal=w.causal, scale=w.scale, dq=dq, dk=dk,
+                        dv=dv)
         elif fp8:
             fa.forward_fp8(q, k, v, dq, dk, dv, causal=w.causal, scale=w.scale, out=o, lse=lse)
         else:
@@ -335,6 +366,13 @@ def run_ours(args):
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     hds = []
+    if w.kind == "bwd":
+        hdo_ = inp.dout.pin_memory()
+        ho_in = o.cpu().pin_memory()
+        hl_in = lse.cpu().pin_memory()
+        hdq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        hdk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+        hdv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
     if w.rotate:
         hs_ = inp.signs.pin_memory()
     elif fp8:
@@ -344,6 +382,13 @@ def run_ours(args):
         q.copy_(hq_, non_blocking=True)
         k.copy_(hk_, non_blocking=True)
         v.copy_(hv_, non_blocking=True)
+        if w.kind == "bwd":
+            for dst, src in ((dout, hdo_), (o, ho_in), (lse, hl_in)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in ((hdq, dq), (hdk, dk), (hdv, dv)):
+                dst.copy_(src, non_blocking=True)
+            return
         if w.rotate:
             signs.copy_(hs_, non_blocking=True)
         elif fp8:
@@ -369,6 +414,9 @@ def run_ours(args):
         h2d = sum(t.numel() * t.element_size() for t in host)
         h2d += sum(t.numel() * t.element_size() for t in hds)
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+        if w.kind == "bwd":
+            h2d += o.numel() * o.element_size() + lse.numel() * lse.element_size()
+            d2h = sum(t.numel() * t.element_size() for t in (dq, dk, dv))
         e2e = {"value": w.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
@@ -392,8 +440,15 @@ def run_ours(args):
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        rate, desc, cores, _, _ = oracle_sample_rate(w, inp, args.cpu_seconds)
+        if w.kind == "bwd":
+            rate, desc, cores, _ = oracle_bwd_sample(w, inp, args.cpu_seconds)
+        else:
+            rate, desc, cores, _, _ = oracle_sample_rate(w, inp, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+    kernel_name = "fa_fwd_kernel"
+    if w.kind == "bwd":
+        kernel_name = ("fa_bwd: prep kernel + fa_bwd_kernel + dQ kernel (and the dQ "
+                       "accumulator memset), timed together as one call")
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -406,7 +461,7 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": profiled_traffic(w.name),
                      "peak_source": "%s (%s)" % (peak_src, peak_note),
-                     "kernel": "fa_fwd_kernel"},
+                     "kernel": kernel_name},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * (args.steps + e2e_steps),
@@ -440,6 +495,8 @@ def run_reference(args):
     w = select_workload(args)
     inp = workloads.make_inputs(w)
     per_step = max(0.05, args.reference_budget_s / max(1, args.steps + args.warmup))
+    if w.kind == "bwd":
+        return run_reference_bwd(args, w, inp, per_step, world)
     n_rows = oracle_calibrate(w, inp, per_step)
     for i in range(args.warmup):
         oracle_timed_sample(w, inp, n_rows, seed=100 + i)
@@ -460,6 +517,30 @@ def run_reference(args):
                        parallelism="independent replicas of the workload per GPU"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": "per step: " + descs[-1]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line))
+
+
+def run_reference_bwd(args, w, inp, per_step, world):
+    for _ in range(args.warmup):
+        oracle_bwd_sample(w, inp, per_step)
+    rates, total_s, desc, cores = [], 0.0, "", 1
+    for _ in range(args.steps):
+        rate, desc, cores, dt = oracle_bwd_sample(w, inp, per_step)
+        rates.append(rate)
+        total_s += dt
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(w.describe(), l2="n/a (CPU)",
+                       parallelism="independent replicas of the workload per GPU"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }

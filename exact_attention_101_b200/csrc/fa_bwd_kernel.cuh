@@ -32,7 +32,10 @@
 // Tensor memory (512 columns): S^T of step buffer b at b*128 (64 columns; after the
 // softmax, P^T and dS^T as packed bf16), dP^T of buffer b at b*128 + 64 (then dQ^T of the
 // same step), dV at 256, dK at 384.  Two step buffers let the softmax of step i+1 run
-// while the tensor core works on step i.
+// while the tensor core works on step i.  Q_i, dO_i and the two per-query vectors sit in a
+// ring of QSTAGES shared-memory stages, so their copies run two steps ahead of the MMAs
+// that read them; dS^T has one shared-memory buffer (the softmax of step g writes it once
+// the dQ^T product of step g-1 has read it).
 //
 // Warps: 0-3 and 4-7 are the "softmax" warpgroups (thread = key row; warpgroup h takes
 // queries 32h .. 32h+31 of the step, and at the end of a unit writes dV (h=0) or dK
@@ -68,12 +71,13 @@ constexpr int VEC_BYTES = 2 * BM * 4;    // per step: LSE*log2(e) and D for BM q
 // Shared memory map (offsets from a 1024-aligned base).
 constexpr int K_OFF = 0;
 constexpr int V_OFF = K_OFF + KV_TILE;
-constexpr int Q_OFF = V_OFF + KV_TILE;   // 2 step buffers
-constexpr int DO_OFF = Q_OFF + 2 * Q_TILE;
-constexpr int DS_OFF = DO_OFF + 2 * Q_TILE;
-constexpr int VEC_OFF = DS_OFF + 2 * DS_TILE;
-constexpr int BAR_OFF = VEC_OFF + 2 * VEC_BYTES;
-constexpr int NUM_BARS = 17;
+constexpr int QSTAGES = 4;               // ring of Q, dO and vector stages
+constexpr int Q_OFF = V_OFF + KV_TILE;
+constexpr int DO_OFF = Q_OFF + QSTAGES * Q_TILE;
+constexpr int DS_OFF = DO_OFF + QSTAGES * Q_TILE;
+constexpr int VEC_OFF = DS_OFF + DS_TILE;
+constexpr int BAR_OFF = VEC_OFF + QSTAGES * VEC_BYTES;
+constexpr int NUM_BARS = 2 + 2 * QSTAGES + 2 * 4 + 3;
 constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
 constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -137,15 +141,16 @@ struct BBars {
   uint32_t base;
   __device__ uint32_t kv_full() const { return base; }
   __device__ uint32_t kv_empty() const { return base + 8u; }
-  __device__ uint32_t q_full(int b) const { return base + 8u * (2 + b); }
-  __device__ uint32_t q_empty(int b) const { return base + 8u * (4 + b); }
-  __device__ uint32_t sdp_full(int b) const { return base + 8u * (6 + b); }
-  __device__ uint32_t ds_full(int b) const { return base + 8u * (8 + b); }
-  __device__ uint32_t dq_full(int b) const { return base + 8u * (10 + b); }
-  __device__ uint32_t dq_empty(int b) const { return base + 8u * (12 + b); }
-  __device__ uint32_t acc_full() const { return base + 8u * 14; }
-  __device__ uint32_t acc_empty() const { return base + 8u * 15; }
-  __device__ uint32_t drain() const { return base + 8u * 16; }
+  __device__ uint32_t q_full(int st) const { return base + 8u * (2 + st); }
+  __device__ uint32_t q_empty(int st) const { return base + 8u * (2 + QSTAGES + st); }
+  static constexpr int B0 = 2 + 2 * QSTAGES;
+  __device__ uint32_t sdp_full(int b) const { return base + 8u * (B0 + b); }
+  __device__ uint32_t ds_full(int b) const { return base + 8u * (B0 + 2 + b); }
+  __device__ uint32_t dq_full(int b) const { return base + 8u * (B0 + 4 + b); }
+  __device__ uint32_t dq_empty(int b) const { return base + 8u * (B0 + 6 + b); }
+  __device__ uint32_t acc_full() const { return base + 8u * (B0 + 8); }
+  __device__ uint32_t acc_empty() const { return base + 8u * (B0 + 9); }
+  __device__ uint32_t drain() const { return base + 8u * (B0 + 10); }
 };
 
 // ---------------------------------------------------------------------------- producer
@@ -171,23 +176,23 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
     }
     ++units_issued;
     for (int s = 0; s < w.steps; ++s) {
-      const int b = steps_issued & 1u;
-      const uint32_t use = steps_issued >> 1;
-      if (!wait_phase(bar.q_empty(b), (use & 1u) ^ 1u, abort_flag, ERR_WAIT_BWD)) goto drain;
+      const int st = steps_issued % QSTAGES;
+      const uint32_t use = steps_issued / QSTAGES;
+      if (!wait_phase(bar.q_empty(st), (use & 1u) ^ 1u, abort_flag, ERR_WAIT_BWD)) goto drain;
       int bh, i;
       step_coords(p, w, s, bh, i);
-      ptx::mbar_arrive_expect_tx(bar.q_full(b), 2 * Q_TILE + VEC_BYTES);
+      ptx::mbar_arrive_expect_tx(bar.q_full(st), 2 * Q_TILE + VEC_BYTES);
 #pragma unroll
       for (int bx = 0; bx < 2; ++bx) {
-        ptx::tma_load_3d(smem + Q_OFF + b * Q_TILE + bx * Q_BOX, tmQ, bar.q_full(b), bx * 64,
+        ptx::tma_load_3d(smem + Q_OFF + st * Q_TILE + bx * Q_BOX, tmQ, bar.q_full(st), bx * 64,
                          i * BM, bh);
-        ptx::tma_load_3d(smem + DO_OFF + b * Q_TILE + bx * Q_BOX, tmDO, bar.q_full(b), bx * 64,
-                         i * BM, bh);
+        ptx::tma_load_3d(smem + DO_OFF + st * Q_TILE + bx * Q_BOX, tmDO, bar.q_full(st),
+                         bx * 64, i * BM, bh);
       }
       const long long voff = static_cast<long long>(bh) * p.Npad + i * BM;
-      ptx::bulk_load(smem + VEC_OFF + b * VEC_BYTES, p.l2 + voff, BM * 4, bar.q_full(b));
-      ptx::bulk_load(smem + VEC_OFF + b * VEC_BYTES + BM * 4, p.dd + voff, BM * 4,
-                     bar.q_full(b));
+      ptx::bulk_load(smem + VEC_OFF + st * VEC_BYTES, p.l2 + voff, BM * 4, bar.q_full(st));
+      ptx::bulk_load(smem + VEC_OFF + st * VEC_BYTES + BM * 4, p.dd + voff, BM * 4,
+                     bar.q_full(st));
       ++steps_issued;
     }
   }
@@ -195,10 +200,10 @@ drain:
   // Let every copy this thread started land before the CTA exits (immediate on the normal
   // path, where the consumers have already waited for them).
   if (units_issued > 0) drain_wait(bar.kv_full(), (units_issued - 1) & 1u);
-  for (uint32_t b = 0; b < 2; ++b)
-    if (steps_issued > b) {
-      const uint32_t last = b + 2 * ((steps_issued - 1 - b) / 2);
-      drain_wait(bar.q_full(b), (last >> 1) & 1u);
+  for (uint32_t st = 0; st < QSTAGES; ++st)
+    if (steps_issued > st) {
+      const uint32_t last = st + QSTAGES * ((steps_issued - 1 - st) / QSTAGES);
+      drain_wait(bar.q_full(st), (last / QSTAGES) & 1u);
     }
 }
 
@@ -253,15 +258,16 @@ __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const
   };
   // S^T and dP^T of global step g (buffer g & 1).
   auto start_step = [&](uint32_t g) {
-    const int b = g & 1u;
+    const int b = g & 1u, st = g % QSTAGES;
     const uint32_t use = g >> 1;
-    if (!wait(bar.q_full(b), use & 1u)) return false;
+    if (!wait(bar.q_full(st), (g / QSTAGES) & 1u)) return false;
     ptx::tc_fence_after();
-    issue_sdp(tmem + s_col(b), k_a, ptx::smem_desc_sw128(smem + Q_OFF + b * Q_TILE, 16, 1024));
+    issue_sdp(tmem + s_col(b), k_a, ptx::smem_desc_sw128(smem + Q_OFF + st * Q_TILE, 16, 1024));
     // dP^T lands where dQ^T of this buffer's previous step was: wait for its drain.
     if (!wait(bar.dq_empty(b), (use & 1u) ^ 1u)) return false;
     ptx::tc_fence_after();
-    issue_sdp(tmem + dp_col(b), v_a, ptx::smem_desc_sw128(smem + DO_OFF + b * Q_TILE, 16, 1024));
+    issue_sdp(tmem + dp_col(b), v_a,
+              ptx::smem_desc_sw128(smem + DO_OFF + st * Q_TILE, 16, 1024));
     ptx::mma_commit_elect(bar.sdp_full(b));
     return true;
   };
@@ -274,22 +280,21 @@ __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const
     for (int s = 0; s < 2 && s < w.steps && ok; ++s) ok = start_step(gm + s);
     for (int s = 0; s < w.steps && ok; ++s) {
       const uint32_t g = gm + s;
-      const int b = g & 1u;
+      const int b = g & 1u, st = g % QSTAGES;
       const uint32_t use = g >> 1;
       if (!(ok = wait(bar.ds_full(b), use & 1u))) break;
       ptx::tc_fence_after();
-      issue_dq(tmem + dp_col(b), k_t,
-               ptx::smem_desc_sw128(smem + DS_OFF + b * DS_TILE, DS_TILE, 1024));
+      issue_dq(tmem + dp_col(b), k_t, ptx::smem_desc_sw128(smem + DS_OFF, DS_TILE, 1024));
       ptx::mma_commit_elect(bar.dq_full(b));
       if (s == 0) {
         if (!(ok = wait(bar.acc_empty(), (unit_it & 1u) ^ 1u))) break;
         ptx::tc_fence_after();
       }
       issue_acc(tmem + DV_COL, tmem + s_col(b),
-                ptx::smem_desc_sw128(smem + DO_OFF + b * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
+                ptx::smem_desc_sw128(smem + DO_OFF + st * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
       issue_acc(tmem + DK_COL, tmem + s_col(b) + 16,
-                ptx::smem_desc_sw128(smem + Q_OFF + b * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
-      ptx::mma_commit_elect(bar.q_empty(b));
+                ptx::smem_desc_sw128(smem + Q_OFF + st * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
+      ptx::mma_commit_elect(bar.q_empty(st));
       if (s == w.steps - 1) {
         ptx::mma_commit_elect(bar.acc_full());
         ptx::mma_commit_elect(bar.kv_empty());
@@ -310,9 +315,11 @@ __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const
 // columns of the S^T buffer and dS^T into the shared-memory tile (128-byte swizzle: the
 // 16-byte chunk c of row r sits at chunk c ^ (r % 8)).
 template <bool CAUSAL>
-__device__ __forceinline__ void softmax_step(const BwdParams &p, uint32_t tmem_row, uint32_t smem,
-                                             int b, int h, int row, int key, int q0,
-                                             bool need_mask) {
+__device__ __forceinline__ bool softmax_step(const BwdParams &p, uint32_t tmem_row, uint32_t smem,
+                                             const BBars &bar, uint32_t g, int h, int row,
+                                             int key, int q0, bool need_mask,
+                                             volatile uint32_t *abort_flag) {
+  const int b = g & 1u, st = g % QSTAGES;
   uint32_t sr[2][16], dr[2][16];
   ptx::tmem_ld16(tmem_row + s_col(b) + h * 32, sr[0]);
   ptx::tmem_ld16(tmem_row + s_col(b) + h * 32 + 16, sr[1]);
@@ -324,7 +331,7 @@ __device__ __forceinline__ void softmax_step(const BwdParams &p, uint32_t tmem_r
   ptx::reg_fence16(dr[0]);
   ptx::reg_fence16(dr[1]);
   const float *vec = reinterpret_cast<const float *>(
-      __cvta_shared_to_generic(smem + VEC_OFF + b * VEC_BYTES));
+      __cvta_shared_to_generic(smem + VEC_OFF + st * VEC_BYTES));
   const float4 *l2v = reinterpret_cast<const float4 *>(vec + h * 32);
   const float4 *ddv = reinterpret_cast<const float4 *>(vec + BM + h * 32);
   uint32_t pp[16], pd[16];
@@ -350,7 +357,11 @@ __device__ __forceinline__ void softmax_step(const BwdParams &p, uint32_t tmem_r
   }
   ptx::tmem_st16(tmem_row + s_col(b) + h * 32, pp);
   ptx::tmem_st16(tmem_row + s_col(b) + h * 32 + 16, pd);
-  const uint32_t ds_row = smem + DS_OFF + b * DS_TILE + row * 128;
+  // the single dS^T buffer is free once the dQ^T product of the previous step has run
+  if (g > 0 && !wait_phase(bar.dq_full((g - 1) & 1u), ((g - 1) >> 1) & 1u, abort_flag,
+                           ERR_WAIT_BWD))
+    return false;
+  const uint32_t ds_row = smem + DS_OFF + row * 128;
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     const uint32_t chunk = static_cast<uint32_t>(h * 4 + cc) ^ static_cast<uint32_t>(row & 7);
@@ -361,6 +372,7 @@ __device__ __forceinline__ void softmax_step(const BwdParams &p, uint32_t tmem_r
   ptx::tmem_wait_st();
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
+  return true;
 }
 
 template <bool CAUSAL>
@@ -385,7 +397,9 @@ __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, c
       // masking is needed on the key tail block and, causally, where the block of
       // queries starts before the last key of the block
       const bool need_mask = (w.j * BN + BN > p.Nk) || (CAUSAL && q0 < w.j * BN + BN - 1);
-      softmax_step<CAUSAL>(p, tmem_row, smem, b, h, row, key, q0, need_mask);
+      if (!softmax_step<CAUSAL>(p, tmem_row, smem, bar, g, h, row, key, q0, need_mask,
+                                abort_flag))
+        return;
       ptx::mbar_arrive(bar.ds_full(b));
     }
     gs += w.steps;
@@ -477,9 +491,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar.kv_full(), 1);
     ptx::mbar_init(bar.kv_empty(), 1);
+    for (int st = 0; st < QSTAGES; ++st) {
+      ptx::mbar_init(bar.q_full(st), 1);
+      ptx::mbar_init(bar.q_empty(st), 1);
+    }
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(bar.q_full(b), 1);
-      ptx::mbar_init(bar.q_empty(b), 1);
       ptx::mbar_init(bar.sdp_full(b), 1);
       ptx::mbar_init(bar.ds_full(b), 256);
       ptx::mbar_init(bar.dq_full(b), 1);

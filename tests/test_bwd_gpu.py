@@ -103,9 +103,12 @@ def test_full_size_gradient_identities(cuda_ok, causal):
     """At the long-context size (too large for the full oracle) check what holds for any
     input: sum_j dV_j = sum_i dO_i, and sum_j dK_j = 0 (rows of dS sum to zero).
 
-    Error budget (u = 2^-8): the dV identity is limited by the bf16 rounding of the N
-    summed rows, independent errors: about u/sqrt(3) * sqrt(N) * rms(dV); the bound takes
-    3 u sum_j |dV_j| / sqrt(N).  In the dK identity the rounding of O inside D_i shifts
+    Error budget (u = 2^-8), per component (head, t): in the dV identity the bf16
+    rounding of the summed rows gives about u/sqrt(3) * sqrt(sum_j dV_jt^2), and rounding
+    P makes each row of P sum to 1 only within u, which adds at most about
+    u * sqrt(sum_i dO_it^2); the bound takes 4u times the sum of the two.  (Under the
+    causal mask a few early keys carry large dV, so the root of the sum of squares, not the
+    mean magnitude, sets the scale.)  In the dK identity the rounding of O inside D_i shifts
     the whole dS row i by the same amount, so the errors do not average over keys: the sum
     is off by about scale * u * sqrt(N) * rms(O) rms(dO) sqrt(d) rms(q) per component;
     the bound takes 6 times that (the maximum over all components, and margin).  rms(O) is
@@ -117,9 +120,10 @@ def test_full_size_gradient_identities(cuda_ok, causal):
     dq, dk, dv = run_fwd_bwd(q, k, v, do, causal, scale)
     u = 2.0 ** -8
     dsum = do.double().sum(dim=2)                        # [B, H, d]
-    err_v = (dv.double().sum(dim=2) - dsum).abs().max().item()
-    bound_v = 3 * u * dv.double().abs().sum(dim=2).max().item() / np.sqrt(N)
-    assert err_v <= bound_v, (err_v, bound_v)
+    err_v = (dv.double().sum(dim=2) - dsum).abs()
+    bound_v = 4 * u * (dv.double().square().sum(dim=2).sqrt() + do.double().square().sum(dim=2).sqrt())
+    assert bool((err_v <= bound_v).all()), (err_v.max().item(), bound_v.min().item())
+    err_v, bound_v = err_v.max().item(), (err_v / bound_v).max().item()
     rows = (np.arange(B * Hq)[:, None] * N
             + np.random.default_rng(0).integers(0, N, size=(B * Hq, 64))).reshape(-1)
     o_rows, _ = oracle.attention_rows(q, k, v, scale, causal, rows=rows)
@@ -128,5 +132,6 @@ def test_full_size_gradient_identities(cuda_ok, causal):
         * rms(q.double().numpy())
     err_k = dk.double().sum(dim=2).abs().max().item()
     assert err_k <= bound_k, (err_k, bound_k)
-    print("identities: dV %.3g (bound %.3g), dK %.3g (bound %.3g)" % (err_v, bound_v, err_k, bound_k))
+    print("identities: dV %.3g (largest error / bound %.2f), dK %.3g (bound %.3g)"
+          % (err_v, bound_v, err_k, bound_k))
     assert torch.isfinite(dq.float()).all()

@@ -19,6 +19,8 @@ Two more workloads feed the incoherent processing of that section (``rotate=True
 bf16 Q/K/V with the fp8 case's outliers, or with a few outlier channels shared by Q and
 K, that the library quantises itself after a random-sign Hadamard rotation of Q and K.
 Their sign vector is drawn here, after the values, and passed to the library as input.
+Backward workloads (``kind="bwd"``) use the forward shapes and draw the upstream gradient
+dO after V, i.i.d. N(0, 1) in bf16.
 """
 from __future__ import annotations
 
@@ -49,6 +51,7 @@ class Workload:
     #                               channels of Q and K (outlier_channels of them)
     outlier_channels: int = 0
     rotate: bool = False          # bf16 source quantised on the GPU with Hadamard rotation
+    kind: str = "fwd"             # "fwd": forward pass; "bwd": backward pass (dO drawn too)
 
     @property
     def scale(self) -> float:
@@ -57,8 +60,11 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """Algorithmic FLOPs: 4*B*Hq*Nq*Nk*d, halved under the causal mask."""
+        """Algorithmic FLOPs: forward 4*B*Hq*Nq*Nk*d (two products), backward 2.5 times
+        that (five products); halved under the causal mask."""
         f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
+        if self.kind == "bwd":
+            f *= 2.5
         return f / 2 if self.causal else f
 
     def describe(self) -> Dict[str, object]:
@@ -68,6 +74,8 @@ class Workload:
                "seed": self.seed}
         if self.rotate:
             out["quantise"] = "e4m3 per head on the GPU, Q and K after random-sign Hadamard"
+        if self.kind == "bwd":
+            out["pass"] = "backward (dQ, dK, dV from Q, K, V, O, LSE, dO)"
         return out
 
 
@@ -83,6 +91,9 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
              rotate=True),
     Workload("fp8_incoherent_channels", 8, 16, 16, 4096, 128, False, "bf16", "bf16", 1007,
              1.0, 10.0, outlier_kind="channel", outlier_channels=4, rotate=True),
+    Workload("long_bwd", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003, kind="bwd"),
+    Workload("long_causal_bwd", 1, 32, 32, 16384, 128, True, "bf16", "bf16", 1003, kind="bwd"),
+    Workload("gqa_causal_bwd", 4, 32, 8, 8192, 128, True, "bf16", "bf16", 1004, kind="bwd"),
 ]}
 
 
@@ -95,6 +106,7 @@ class Inputs:
     descale_k: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
     descale_v: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
     signs: Optional[torch.Tensor] = None       # int8 [d] of +-1 (rotate workloads only)
+    dout: Optional[torch.Tensor] = None        # bf16 [B, Hq, Nq, d] (backward workloads only)
 
 
 def _quantise_e4m3_per_head(x: torch.Tensor):
@@ -139,6 +151,8 @@ def make_inputs(w: Workload, seed: Optional[int] = None, *, B: Optional[int] = N
         inp = Inputs(q32.to(torch.bfloat16), k32.to(torch.bfloat16), v32.to(torch.bfloat16))
         if w.rotate:
             inp.signs = torch.where(torch.rand(d, generator=g) < 0.5, -1, 1).to(torch.int8)
+        if w.kind == "bwd":
+            inp.dout = torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
         return inp
     if w.in_dtype != "e4m3":
         raise ValueError(w.in_dtype)
