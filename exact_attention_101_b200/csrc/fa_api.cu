@@ -371,10 +371,24 @@ fa_status quantize_common(const void *x, const int8_t *signs, void *x8, float *d
   return quant_launch<false>(qp, s, dev, stream);
 }
 
+// 3-D tensor map over the fp32 dQ accumulator [heads, rows, d], box = [1, 64 rows, 32
+// floats], no swizzle: the target of the backward kernel's bulk reduce-adds.
+bool encode_tmap_dq(CUtensorMap *m, void *base, uint64_t d, uint64_t rows, uint64_t heads) {
+  cuuint64_t dims[3] = {d, rows, heads};
+  cuuint64_t strides[2] = {d * 4, rows * d * 4};
+  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(fa::bwd::BM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = driver_fns().encode(
+      m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <bool CAUSAL>
 fa_status bwd_launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                     const CUtensorMap &tdo, const fa::bwd::BwdParams &p, int grid, int dev,
-                     cudaStream_t stream) {
+                     const CUtensorMap &tdo, const CUtensorMap &tdq,
+                     const fa::bwd::BwdParams &p, int grid, int dev, cudaStream_t stream) {
   auto kern = fa::bwd::fa_bwd_kernel<CAUSAL>;
   static std::once_flag attr_once[kMaxDevices];
   static fa_status attr_st[kMaxDevices];
@@ -385,7 +399,7 @@ fa_status bwd_launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
                        : FA_ERR_CUDA;
   });
   if (attr_st[dev] != FA_OK) return attr_st[dev];
-  kern<<<grid, fa::bwd::NUM_THREADS, fa::bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, fa::bwd::NUM_THREADS, fa::bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -470,12 +484,14 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
     cudaGetLastError();
     return FA_ERR_CUDA;
   }
-  p.dq_acc = static_cast<float *>(ws);
+  float *dq_acc = static_cast<float *>(ws);
   p.l2 = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + acc_bytes);
   p.dd = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + acc_bytes + vec_bytes);
-
-  st = FA_OK;
-  if (cudaMemsetAsync(p.dq_acc, 0, q_bytes * 2, stream) != cudaSuccess) st = FA_ERR_CUDA;
+  CUtensorMap tdq;
+  st = encode_tmap_dq(&tdq, dq_acc, d, Nq, static_cast<uint64_t>(B) * Hq) ? FA_OK
+                                                                           : FA_ERR_INVALID_ARG;
+  if (st == FA_OK && cudaMemsetAsync(dq_acc, 0, q_bytes * 2, stream) != cudaSuccess)
+    st = FA_ERR_CUDA;
   if (st == FA_OK) {
     const unsigned blocks = static_cast<unsigned>((rows_padded + 7) / 8);
     fa::bwd::fa_bwd_prep_kernel<<<blocks, 256, 0, stream>>>(
@@ -486,13 +502,13 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
   }
   if (st == FA_OK) {
     const int grid = p.num_units < info.sms ? p.num_units : info.sms;
-    st = causal ? bwd_launch<true>(tq, tk, tv, tdo, p, grid, dev, stream)
-                : bwd_launch<false>(tq, tk, tv, tdo, p, grid, dev, stream);
+    st = causal ? bwd_launch<true>(tq, tk, tv, tdo, tdq, p, grid, dev, stream)
+                : bwd_launch<false>(tq, tk, tv, tdo, tdq, p, grid, dev, stream);
   }
   if (st == FA_OK) {
     const long long n4 = static_cast<long long>(q_bytes / 2 / 4);
     fa::bwd::fa_bwd_dq_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
-        p.dq_acc, static_cast<uint16_t *>(dq), n4, scale);
+        dq_acc, static_cast<uint16_t *>(dq), n4, scale);
     if (cudaGetLastError() != cudaSuccess) st = FA_ERR_CUDA;
   }
   if (cudaFreeAsync(ws, stream) != cudaSuccess && st == FA_OK) st = FA_ERR_CUDA;

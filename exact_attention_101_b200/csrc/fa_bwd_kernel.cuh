@@ -24,9 +24,9 @@
 //   dV  += P^T dO_i       M=128 keys, N=128, K=64 queries (A = P^T from tensor memory)
 //   dK  += dS^T Q_i       same shape (A = dS^T from tensor memory)
 //
-// dQ^T goes through tensor memory to fp32 reduction-adds into a zeroed global accumulator
-// (each query block receives one contribution per key block); a last kernel scales it
-// and rounds to bf16.  dK, dV leave once per unit, with no atomics: the group's query heads
+// dQ^T goes from tensor memory through a shared-memory staging tile to a bulk tensor
+// reduce-add (TMA) into a zeroed fp32 accumulator in global memory (each query block
+// receives one contribution per key block); a last kernel scales it and rounds to bf16.  dK, dV leave once per unit, with no atomics: the group's query heads
 // are summed inside the unit.
 //
 // Tensor memory (512 columns): S^T of step buffer b at b*128 (64 columns; after the
@@ -71,11 +71,13 @@ constexpr int VEC_BYTES = 2 * BM * 4;    // per step: LSE*log2(e) and D for BM q
 // Shared memory map (offsets from a 1024-aligned base).
 constexpr int K_OFF = 0;
 constexpr int V_OFF = K_OFF + KV_TILE;
-constexpr int QSTAGES = 4;               // ring of Q, dO and vector stages
+constexpr int QSTAGES = 3;               // ring of Q, dO and vector stages
+constexpr int DQ_STAGE = 32 * BM * 4;    // per drain warp: 64 queries x 32 head dims fp32
 constexpr int Q_OFF = V_OFF + KV_TILE;
 constexpr int DO_OFF = Q_OFF + QSTAGES * Q_TILE;
 constexpr int DS_OFF = DO_OFF + QSTAGES * Q_TILE;
-constexpr int VEC_OFF = DS_OFF + DS_TILE;
+constexpr int DQS_OFF = DS_OFF + DS_TILE;
+constexpr int VEC_OFF = DQS_OFF + 4 * DQ_STAGE;
 constexpr int BAR_OFF = VEC_OFF + QSTAGES * VEC_BYTES;
 constexpr int NUM_BARS = 2 + 2 * QSTAGES + 2 * 4 + 3;
 constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
@@ -96,7 +98,6 @@ constexpr uint32_t ERR_WAIT_BWD = 1u << 6;
 struct BwdParams {
   const float *l2;     // [B*Hq, Npad]: LSE * log2(e), +inf past Nq
   const float *dd;     // [B*Hq, Npad]: D = rowsum(dO o O), 0 past Nq
-  float *dq_acc;       // [B*Hq, Nq, D] fp32, zeroed before the launch
   uint16_t *dk, *dv;   // bf16 [B*Hkv, Nk, D]
   int B, Hq, Hkv, Nq, Nk, Npad, group;
   int num_kb;          // ceil(Nk / BN)
@@ -432,22 +433,28 @@ __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, c
 
 // ---------------------------------------------------------------------------- dQ drain
 
-// Thread = head dimension t: after each step's dQ^T lands, read its 64 query columns and
-// add them to dq_acc[bh, q, t] (32 consecutive t per warp: one 128-byte reduction per
-// query).
+// Thread = head dimension t (warp w of the group owns t = 32w .. 32w+31): after each
+// step's dQ^T lands, read its 64 query columns, write them as a [64 queries][32 dims]
+// fp32 tile into the warp's staging buffer (one 128-byte row per query, so every store
+// instruction of the warp fills one row) and add the tile into the accumulator with one
+// bulk tensor reduce-add.  Queries past Nq fall outside the tensor and are not written.
 template <bool CAUSAL>
-__device__ void dq_role(const BwdParams &p, uint32_t tmem, const BBars &bar,
-                        volatile uint32_t *abort_flag) {
+__device__ void dq_role(const CUtensorMap *tmDQ, const BwdParams &p, uint32_t smem, uint32_t tmem,
+                        const BBars &bar, volatile uint32_t *abort_flag) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t = (warp % 4) * 32 + lane;
-  const uint32_t tmem_row = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+  const int wq = warp % 4;
+  const uint32_t tmem_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const uint32_t stage = smem + DQS_OFF + wq * DQ_STAGE;
+  if (lane == 0) ptx::prefetch_tmap(tmDQ);
   uint32_t gd = 0;
+  bool pending = false;
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
     const BUnit w = decode_unit<CAUSAL>(p, u);
     for (int s = 0; s < w.steps; ++s) {
       const uint32_t g = gd + s;
       const int b = g & 1u;
-      if (!wait_phase(bar.dq_full(b), (g >> 1) & 1u, abort_flag, ERR_WAIT_BWD)) return;
+      const bool ok = wait_phase(bar.dq_full(b), (g >> 1) & 1u, abort_flag, ERR_WAIT_BWD);
+      if (!__all_sync(0xffffffffu, ok)) goto done;
       ptx::tc_fence_after();
       uint32_t r[4][16];
 #pragma unroll
@@ -457,18 +464,30 @@ __device__ void dq_role(const BwdParams &p, uint32_t tmem, const BBars &bar,
       for (int c = 0; c < 4; ++c) ptx::reg_fence16(r[c]);
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.dq_empty(b));
-      int bh, i;
-      step_coords(p, w, s, bh, i);
-      const int q0 = i * BM;
-      float *dst = p.dq_acc + (static_cast<long long>(bh) * p.Nq + q0) * D + t;
-      const int nvalid = min(BM, p.Nq - q0);
+      // the previous reduce must have read the staging tile before it is overwritten
+      if (pending && lane == 0) ptx::bulk_wait_read_all();
+      __syncwarp();
 #pragma unroll
       for (int c = 0; c < BM; ++c)
-        if (c < nvalid) ptx::red_add_f32(dst + static_cast<long long>(c) * D,
-                                         __uint_as_float(r[c / 16][c % 16]));
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage + c * 128 + lane * 4),
+                     "r"(r[c / 16][c % 16])
+                     : "memory");
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      int bh, i;
+      step_coords(p, w, s, bh, i);
+      if (lane == 0) {
+        ptx::tma_reduce_add_3d(tmDQ, stage, wq * 32, i * BM, bh);
+        ptx::bulk_commit_group();
+      }
+      pending = true;
     }
     gd += w.steps;
   }
+done:
+  // every reduce must be complete before the CTA exits
+  if (lane == 0) ptx::bulk_wait_all();
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------- kernels
@@ -477,7 +496,7 @@ template <bool CAUSAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t smem = (raw + 1023u) & ~1023u;  // 1024-aligned for 128-byte swizzle
@@ -519,7 +538,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp < DRAIN_WARP0) {
     softmax_role<CAUSAL>(p, smem, tmem, bar, abort_flag);
   } else if (warp < MMA_WARP) {
-    dq_role<CAUSAL>(p, tmem, bar, abort_flag);
+    dq_role<CAUSAL>(&tmDQ, p, smem, tmem, bar, abort_flag);
   } else if (warp == MMA_WARP) {
     mma_role<CAUSAL>(p, smem, tmem, bar, abort_flag);
     __syncwarp();
