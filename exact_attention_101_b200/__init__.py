@@ -20,8 +20,9 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
-C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_quantize_e4m3", "fa_check_device_error",
-             "fa_selftest_bounded_wait", "fa_status_string", "fa_version")
+C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
+             "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_string",
+             "fa_version")
 
 _lib = None
 
@@ -47,6 +48,9 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
         L.fa_bwd.restype = i
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
+        L.fa_bwd_noalloc.restype = i
+        L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
+                                     vp]
         L.fa_quantize_e4m3.restype = i
         L.fa_quantize_e4m3.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.fa_check_device_error.restype = i
@@ -80,6 +84,13 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, caus
     """Raw ``fa_bwd``."""
     return lib().fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
                         causal, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                   stream) -> int:
+    """Raw ``fa_bwd_noalloc`` (fa_bwd with the library's fixed per-device scratch)."""
+    return lib().fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d,
+                                scale, causal, stream)
 
 
 def fa_quantize_e4m3(x, signs, x8, descale, B, H, N, d, stream) -> int:

@@ -427,10 +427,21 @@ fa_status check_bwd_args(const void *q, const void *k, const void *v, const void
   return FA_OK;
 }
 
+// Bytes of backward scratch: the fp32 dQ accumulator and two padded per-row vectors,
+// each rounded up to 256 bytes.
+uint64_t bwd_scratch_bytes(int B, int Hq, int Nq, int d, uint64_t *acc_bytes, uint64_t *vec_bytes) {
+  const uint64_t npad = (static_cast<uint64_t>(Nq) + fa::bwd::BM - 1) / fa::bwd::BM * fa::bwd::BM;
+  *acc_bytes = (static_cast<uint64_t>(B) * Hq * Nq * d * 4 + 255) / 256 * 256;
+  *vec_bytes = (static_cast<uint64_t>(B) * Hq * npad * 4 + 255) / 256 * 256;
+  return *acc_bytes + 2 * *vec_bytes;
+}
+
+// fixed_ws == nullptr: scratch is allocated and freed on `stream` (cudaMallocAsync /
+// cudaFreeAsync); otherwise fixed_ws (large enough, checked by the caller) is used.
 fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
                      int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, void *fixed_ws = nullptr) {
   fa_status st = check_bwd_args(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
                                 causal);
   if (st != FA_OK) return st;
@@ -477,10 +488,10 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
   // Scratch, stream-ordered: the fp32 dQ accumulator and the padded per-row LSE * log2(e)
   // and D arrays.
   const uint64_t rows_padded = static_cast<uint64_t>(B) * Hq * p.Npad;
-  const uint64_t acc_bytes = (q_bytes * 2 + 255) / 256 * 256;
-  const uint64_t vec_bytes = (rows_padded * 4 + 255) / 256 * 256;
-  void *ws = nullptr;
-  if (cudaMallocAsync(&ws, acc_bytes + 2 * vec_bytes, stream) != cudaSuccess) {
+  uint64_t acc_bytes = 0, vec_bytes = 0;
+  const uint64_t ws_bytes = bwd_scratch_bytes(B, Hq, Nq, d, &acc_bytes, &vec_bytes);
+  void *ws = fixed_ws;
+  if (ws == nullptr && cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_CUDA;
   }
@@ -511,8 +522,55 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
         dq_acc, static_cast<uint16_t *>(dq), n4, scale);
     if (cudaGetLastError() != cudaSuccess) st = FA_ERR_CUDA;
   }
-  if (cudaFreeAsync(ws, stream) != cudaSuccess && st == FA_OK) st = FA_ERR_CUDA;
+  if (fixed_ws == nullptr && cudaFreeAsync(ws, stream) != cudaSuccess && st == FA_OK)
+    st = FA_ERR_CUDA;
   return st;
+}
+
+// Scratch of fa_bwd_noalloc.  Some callers cannot let the library allocate device memory
+// per call: a framework whose own caching allocator has reserved (nearly) all of the
+// device's memory, so that a stream-ordered allocation outside it can fail, or a service
+// that must keep a fixed, known memory footprint.  For them the backward pass runs in this
+// statically sized buffer, which exists once per device as part of the loaded library
+// (no allocation at call time).  One buffer per device means calls that overlap in time on
+// the same device (other streams, other host threads) would share it and race; such calls
+// must be serialised by the caller.
+constexpr uint64_t kNoAllocScratchBytes = 64ull << 20;
+static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the fixed scratch on device `dev` (looked up once per device).
+fa_status noalloc_scratch(int dev, void **out) {
+  static std::once_flag once[kMaxDevices];
+  static void *addr[kMaxDevices];
+  static fa_status st[kMaxDevices];
+  std::call_once(once[dev], [&] {
+    st[dev] = cudaGetSymbolAddress(&addr[dev], g_bwd_noalloc_scratch) == cudaSuccess
+                  ? FA_OK
+                  : FA_ERR_CUDA;
+    if (st[dev] != FA_OK) cudaGetLastError();
+  });
+  *out = addr[dev];
+  return st[dev];
+}
+
+fa_status bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                      int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                      cudaStream_t stream) {
+  fa_status st = check_bwd_args(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
+                                causal);
+  if (st != FA_OK) return st;
+  uint64_t acc_bytes = 0, vec_bytes = 0;
+  if (bwd_scratch_bytes(B, Hq, Nq, d, &acc_bytes, &vec_bytes) > kNoAllocScratchBytes)
+    return FA_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  void *ws = nullptr;
+  st = noalloc_scratch(dev, &ws);
+  if (st != FA_OK) return st;
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                    stream, ws);
 }
 
 }  // namespace
@@ -547,6 +605,14 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, con
                  int Nk, int d, float scale, int causal, fa_stream_t stream) {
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                         const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         fa_stream_t stream) {
+  return bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_check_device_error(fa_stream_t stream) {

@@ -22,11 +22,12 @@
  * reads K/V head hq / (Hq / Hkv) (consecutive query heads share a K/V head).
  * Causal masking admits key j for query i iff j <= i and requires Nq == Nk.
  *
- * Ownership: the caller allocates and owns every buffer.  The library allocates no
- * device memory in these calls and keeps no pointer after a call returns.
+ * Ownership: the caller allocates and owns every buffer.  The library keeps no pointer
+ * after a call returns and allocates no device memory, except fa_bwd, which allocates
+ * and frees its scratch in stream order on the caller's stream (see there).
  *
  * Execution: every call validates its arguments on the host first; on a validation error
- * it returns without touching the GPU.  Otherwise it enqueues one kernel on `stream`
+ * it returns without touching the GPU.  Otherwise it enqueues its kernels on `stream`
  * and returns immediately (asynchronous).  A device-side wait that gave up (see
  * fa_check_device_error) is reported by the next fa_check_device_error call.
  *
@@ -120,8 +121,8 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
  * All pointers 16-byte aligned (lse 4-byte).  The outputs must not overlap the inputs.
  * Scratch: the call allocates B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes on `stream` with
  * cudaMallocAsync (an fp32 dQ accumulator and two per-row vectors) and frees it on the
- * same stream with cudaFreeAsync.  dQ is summed with fp32 atomic additions, so its last
- * bits may differ between runs.  Enqueues a memset and three kernels.  Returns FA_OK once
+ * same stream with cudaFreeAsync.  dQ is summed with fp32 reduce-adds whose order varies,
+ * so its last bits may differ between runs (dK and dV do not).  Enqueues a memset and three kernels.  Returns FA_OK once
  * enqueued; FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (d != 128, causal with Nq != Nk,
  * GPU not sm_100) with nothing enqueued; FA_ERR_CUDA if the scratch allocation or a launch
  * failed.
@@ -129,6 +130,23 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
 fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
                  const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv,
                  int Nq, int Nk, int d, float scale, int causal, fa_stream_t stream);
+
+/*
+ * fa_bwd without any allocation at call time.  The pages describe nothing like it: it is
+ * an engineering variant for callers that cannot let the library allocate device memory
+ * per call (a framework whose own caching allocator holds nearly all of the device's
+ * memory, or a service that must keep a fixed footprint).  Arguments, results and errors
+ * are those of fa_bwd, except for the scratch: instead of allocating it on `stream`, the
+ * call uses one fixed 64 MiB buffer that the library holds per device.  A problem whose
+ * scratch, B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes (each part rounded up to 256 bytes),
+ * does not fit returns FA_ERR_UNSUPPORTED with nothing enqueued.  Calls on the same stream
+ * are ordered; calls that may overlap in time on the same device (other streams, other
+ * host threads) share the buffer and race, so the caller must serialise them.
+ */
+fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                         const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                         int causal, fa_stream_t stream);
 
 /*
  * Per-(batch, head) fp8-e4m3 quantisation of a bf16 tensor, optionally with incoherent
