@@ -23,9 +23,11 @@
  * the bullet on exact computation), so the plain definition is the oracle.
  *
  * Causal masking ("Flash Attention" page, section "Zentrale technische Innovationen",
- * the bullet on autoregressive models): key j is admissible for query i iff j <= i
- * (top-left alignment; the library only accepts causal with Nq == Nk, where top-left and
- * bottom-right alignment coincide).
+ * the bullet on autoregressive models): key j is admissible for query i iff
+ * j <= i + (Nk - Nq).  With Nq == Nk that is j <= i.  With Nq != Nk the pages say nothing;
+ * the queries are read as the last Nq positions of a sequence of Nk keys (bottom-right
+ * alignment: each query sees every key up to its own position).  A query with no
+ * admissible key (Nq > Nk) gets O = 0 and LSE = ln(empty sum) = -inf.
  *
  * Grouped/multi-query heads ("Flash Attention" page, same section, the MQA/GQA bullet; page
  * "FlashAttention 4: Praxisleitfaden ...", section "Kompatibilitaet und aktueller
@@ -144,9 +146,15 @@ int oracle_attention_rows(const void *q, const void *k, const void *v, int elem_
                 const int64_t kvoff = bhk * Nk * d;
                 for (int64_t t = 0; t < d; ++t) qrow[t] = load_elem(q, elem_type, qoff + t) * dq;
 
-                /* Admissible keys: all of them, or j <= i under the causal mask. */
+                /* Admissible keys: all of them, or j <= i + (Nk - Nq) under the causal
+                 * mask. */
                 int64_t nkeys = Nk;
-                if (causal && i + 1 < nkeys) nkeys = i + 1;
+                if (causal && i + 1 + (Nk - Nq) < nkeys) nkeys = i + 1 + (Nk - Nq);
+                if (nkeys <= 0) {
+                    for (int64_t t = 0; t < d; ++t) o_out[r * d + t] = 0.0;
+                    lse_out[r] = -INFINITY;
+                    continue;
+                }
 
                 /* Row i of S, materialised. */
                 double m = -INFINITY;

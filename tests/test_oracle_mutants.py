@@ -54,6 +54,16 @@ def pin_bruteforce_lse(lib):
         assert np.abs(o[0, 0] - bo).max() < 1e-12 and np.abs(lse[0, 0] - bl).max() < 1e-12
 
 
+def pin_bottom_right(lib):
+    q, k, v = rnd((1, 1, 4, 3), 10), rnd((1, 1, 7, 3), 11), rnd((1, 1, 7, 3), 12)
+    o, _ = oracle.attention(q, k, v, 0.5, True, _library=lib)
+    mask = torch.arange(7)[None, :] <= torch.arange(4)[:, None] + 3
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), attn_mask=mask,
+        scale=0.5).numpy()
+    assert np.abs(o - ref).max() < 1e-12
+
+
 def pin_gqa(lib):
     q, k, v = rnd((1, 8, 9, 4), 7), rnd((1, 2, 9, 4), 8), rnd((1, 2, 9, 4), 9)
     o1, l1 = oracle.attention(q, k, v, 0.3, False, _library=lib)
@@ -146,14 +156,17 @@ def pin_bwd_autograd(lib):
             assert np.abs(g - r.numpy()).max() < 1e-12
 
 
-PINS = [pin_sdpa, pin_bruteforce_lse, pin_gqa, pin_decoders, pin_e4m3_descales,
+PINS = [pin_sdpa, pin_bruteforce_lse, pin_bottom_right, pin_gqa, pin_decoders, pin_e4m3_descales,
         pin_hadamard_scipy, pin_encoder_torch, pin_rotation_basis_and_norm,
         pin_quantise_rounding_bound, pin_bwd_autograd]
 
 MUTANTS = {
     "scale_dropped": ("srow[j] = scale * dot;", "srow[j] = dot;"),
-    "causal_off_by_one": ("if (causal && i + 1 < nkeys) nkeys = i + 1;",
-                          "if (causal && i + 2 < nkeys) nkeys = i + 2;"),
+    "causal_off_by_one": ("if (causal && i + 1 + (Nk - Nq) < nkeys) nkeys = i + 1 + (Nk - Nq);",
+                          "if (causal && i + 2 + (Nk - Nq) < nkeys) nkeys = i + 2 + (Nk - Nq);"),
+    "causal_top_left_alignment": (
+        "if (causal && i + 1 + (Nk - Nq) < nkeys) nkeys = i + 1 + (Nk - Nq);",
+        "if (causal && i + 1 < nkeys) nkeys = i + 1;"),
     "gqa_head_mapping": ("const int64_t hk = hq / group;", "const int64_t hk = hq % Hkv;"),
     "lse_log_base": ("lse_out[r] = m + log(l);", "lse_out[r] = m + log2(l);"),
     "lse_max_dropped": ("lse_out[r] = m + log(l);", "lse_out[r] = log(l);"),

@@ -187,7 +187,38 @@ def test_nonsquare_noncausal_bruteforce():
     np.testing.assert_allclose(lse[0, 0], np.array(bl), atol=1e-12)
 
 
+@pytest.mark.parametrize("nq,nk", [(3, 5), (5, 3), (4, 4), (1, 6)])
+def test_bottom_right_causal_bruteforce(nq, nk):
+    """Causal with Nq != Nk: query i sees keys j <= i + (Nk - Nq); a query with no key
+    gets O = 0 and LSE = -inf."""
+    q, k, v = rnd((1, 1, nq, 3), 33), rnd((1, 1, nk, 3), 34), rnd((1, 1, nk, 3), 35)
+    o, lse = oracle.attention(q, k, v, 0.6, causal=True)
+    for i in range(nq):
+        keys = list(range(0, min(nk, i + 1 + nk - nq)))
+        if not keys:
+            assert np.all(o[0, 0, i] == 0.0) and lse[0, 0, i] == -np.inf
+            continue
+        e = [math.exp(0.6 * math.fsum(q[0, 0, i, t] * k[0, 0, j, t] for t in range(3)))
+             for j in keys]
+        z = math.fsum(e)
+        assert abs(lse[0, 0, i] - math.log(z)) < 1e-12
+        for t in range(3):
+            assert abs(o[0, 0, i, t] - math.fsum(e[n] * v[0, 0, j, t] for n, j in enumerate(keys)) / z) < 1e-12
+
+
 # ----------------------------------------------------------------------------- library routine
+
+@pytest.mark.parametrize("nq,nk", [(20, 45), (45, 20)])
+def test_bottom_right_causal_matches_torch_sdpa_with_explicit_mask(nq, nk):
+    q, k, v = rnd((1, 2, nq, 8), 36), rnd((1, 2, nk, 8), 37), rnd((1, 2, nk, 8), 38)
+    o, lse = oracle.attention(q, k, v, 0.3, causal=True)
+    mask = torch.arange(nk)[None, :] <= torch.arange(nq)[:, None] + (nk - nq)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), attn_mask=mask,
+        scale=0.3).numpy()
+    rows = mask.any(dim=1).numpy()      # rows with at least one key
+    np.testing.assert_allclose(o[:, :, rows], ref[:, :, rows], rtol=0, atol=1e-12)
+    assert np.all(o[:, :, ~rows] == 0.0) and np.all(lse[:, :, ~rows] == -np.inf)
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_matches_torch_sdpa_float64(causal):
