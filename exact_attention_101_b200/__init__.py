@@ -1,10 +1,10 @@
 """B200-native fused exact attention forward: Python binding of ``libfa_b200.so``.
 
 The C ABI (``include/fa_b200.h``) is the product; this module only marshals arguments
-into it.  The functions ``fa_fwd``, ``fa_fwd_fp8``, ``fa_bwd``, ``fa_quantize_e4m3``,
+into it.  The functions ``fa_fwd``, ``fa_fwd_varlen``, ``fa_fwd_fp8``, ``fa_bwd``, ``fa_quantize_e4m3``,
 ``fa_check_device_error`` and ``fa_status_string`` have the names and argument order of
-the C entry points and take raw device pointers.  ``forward`` / ``forward_fp8`` /
-``backward`` / ``quantize_e4m3`` are conveniences that take CUDA tensors (PyTorch provides device
+the C entry points and take raw device pointers.  ``forward`` / ``forward_varlen`` /
+``forward_fp8`` / ``backward`` / ``quantize_e4m3`` are conveniences that take CUDA tensors (PyTorch provides device
 memory and streams only), allocate the outputs and raise on a non-zero status.  Every step of the attention runs in the CUDA kernels; there
 is no CPU or library fallback -- if the shared library is missing, importing a function
 that needs it raises.
@@ -20,7 +20,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
-C_SYMBOLS = ("fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
+C_SYMBOLS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
              "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_string",
              "fa_version")
 
@@ -44,6 +44,8 @@ def lib() -> ctypes.CDLL:
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.fa_fwd.restype = i
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+        L.fa_fwd_varlen.restype = i
+        L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, vp]
         L.fa_fwd_fp8.restype = i
         L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
         L.fa_bwd.restype = i
@@ -70,6 +72,13 @@ def lib() -> ctypes.CDLL:
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
     """Raw ``fa_fwd``: pointers are ints (device addresses), stream an int handle."""
     return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, total_q, total_k,
+                  max_seqlen_q, d, scale, causal, dtype, stream) -> int:
+    """Raw ``fa_fwd_varlen``."""
+    return lib().fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv,
+                               total_q, total_k, max_seqlen_q, d, scale, causal, dtype, stream)
 
 
 def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
@@ -164,6 +173,42 @@ def forward(q, k, v, causal=False, scale=None, out_dtype=None, out=None, lse=Non
                 B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), dtype, _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=False,
+                   scale=None, out_dtype=None, out=None, lse=None, stream=None):
+    """Attention over packed sequences of different lengths: q [total_q, Hq, d], k, v
+    [total_k, Hkv, d] bf16, cu_seqlens_* int32 CUDA tensors of B+1 offsets.  Returns
+    ``(o [total_q, Hq, d], lse [Hq, total_q])``."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if (not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 3
+                or not t.is_contiguous()):
+            raise ValueError("%s must be a contiguous bf16 CUDA tensor [tokens, H, d]" % name)
+    total_q, Hq, d = q.shape
+    total_k, Hkv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or dk != d:
+        raise ValueError("shape mismatch between q, k and v")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if not t.is_cuda or t.dtype != torch.int32 or t.dim() != 1 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous int32 CUDA tensor" % name)
+    B = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((total_q, Hq, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    dtype = FA_BF16_OUT_F32 if out_dtype == torch.float32 else FA_BF16
+    st = fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                       cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, Hq, Hkv, total_q,
+                       total_k, int(max_seqlen_q), d, scale, int(bool(causal)), dtype,
+                       _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_varlen")
     return out, lse
 
 

@@ -119,11 +119,11 @@ bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool CAUSAL, bool OUT_F32, bool FP8>
+template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN = false>
 fa_status launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                  const fa::FwdParams &p, int grid, int dev, cudaStream_t stream) {
   using C = fa::TileCfg<D, FP8>;
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL, OUT_F32, FP8>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, OUT_F32, FP8, VARLEN>;
   static std::once_flag attr_once[kMaxDevices];
   static fa_status attr_st[kMaxDevices];
   std::call_once(attr_once[dev], [&] {
@@ -175,7 +175,6 @@ fa_status check_args(const void *q, const void *k, const void *v, const void *o,
     return FA_ERR_INVALID_ARG;
   if (Nk > INT32_MAX - 2 * fa::BN || Nq > INT32_MAX - 2 * fa::UNIT_ROWS) return FA_ERR_INVALID_ARG;
   if (fp8 ? d != 128 : (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
-  if (causal && Nq != Nk) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -219,6 +218,8 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
   p.descale_q = dq;
   p.descale_k = dk;
   p.descale_v = dv;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -246,6 +247,95 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
                    : launch<128, true, false, false>(tq, tk, tv, p, grid, dev, stream);
   return out_f32 ? launch<128, false, true, false>(tq, tk, tv, p, grid, dev, stream)
                  : launch<128, false, false, false>(tq, tk, tv, p, grid, dev, stream);
+}
+
+// 3-D tensor map over a packed [tokens, heads, d] bf16 tensor, box = [128 bytes of d,
+// 1 head, box_rows tokens], 128-byte swizzle: the same shared-memory tile as encode_tmap.
+bool encode_tmap_packed(CUtensorMap *m, const void *base, uint64_t d, uint64_t heads,
+                        uint64_t tokens, uint32_t box_rows) {
+  cuuint64_t dims[3] = {d, heads, tokens};
+  cuuint64_t strides[2] = {d * 2, heads * d * 2};
+  cuuint32_t box[3] = {64, 1, box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = driver_fns().encode(
+      m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+fa_status fwd_varlen_common(const void *q, const void *k, const void *v, void *o, float *lse,
+                            const int *cu_q, const int *cu_k, int B, int Hq, int Hkv,
+                            int total_q, int total_k, int max_q, int d, float scale,
+                            int causal, fa_dtype dtype, cudaStream_t stream) {
+  // Pure host checks first.
+  if (!q || !k || !v || !o || !lse || !cu_q || !cu_k) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      ((reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(cu_q) |
+        reinterpret_cast<uintptr_t>(cu_k)) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || total_q < 1 || total_k < 1 || max_q < 1 || d < 1)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_BF16_OUT_F32) return FA_ERR_INVALID_ARG;
+  const int64_t num_qb = (static_cast<int64_t>(max_q) + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  if (static_cast<int64_t>(B) * Hq * num_qb > INT32_MAX || max_q > INT32_MAX - 2 * fa::UNIT_ROWS ||
+      total_k > INT32_MAX - 2 * fa::BN || total_q > INT32_MAX - 2 * fa::UNIT_ROWS)
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  DeviceInfo info;
+  fa_status st = device_info(dev, &info);
+  if (st != FA_OK) return st;
+  if (info.major != 10 || info.minor != 0) return FA_ERR_UNSUPPORTED;
+  if (!driver_fns().ok) return FA_ERR_CUDA;
+  const bool out_f32 = dtype == FA_BF16_OUT_F32;
+  const uint64_t q_bytes = static_cast<uint64_t>(total_q) * Hq * d * 2;
+  const uint64_t kv_bytes = static_cast<uint64_t>(total_k) * Hkv * d * 2;
+  const uint64_t o_bytes = static_cast<uint64_t>(total_q) * Hq * d * (out_f32 ? 4 : 2);
+  if (!buffer_ok(q, q_bytes, dev) || !buffer_ok(k, kv_bytes, dev) || !buffer_ok(v, kv_bytes, dev) ||
+      !buffer_ok(o, o_bytes, dev) || !buffer_ok(lse, static_cast<uint64_t>(total_q) * Hq * 4, dev) ||
+      !buffer_ok(cu_q, static_cast<uint64_t>(B + 1) * 4, dev) ||
+      !buffer_ok(cu_k, static_cast<uint64_t>(B + 1) * 4, dev))
+    return FA_ERR_INVALID_ARG;
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_tmap_packed(&tq, q, d, Hq, total_q, fa::BM) ||
+      !encode_tmap_packed(&tk, k, d, Hkv, total_k, fa::BN) ||
+      !encode_tmap_packed(&tv, v, d, Hkv, total_k, fa::BN))
+    return FA_ERR_INVALID_ARG;
+
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.descale_q = p.descale_k = p.descale_v = nullptr;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = total_q;
+  p.Nk = total_k;
+  p.group = Hq / Hkv;
+  p.num_qb = static_cast<int>(num_qb);
+  p.num_units = static_cast<int>(B * Hq * num_qb);
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  const int grid = p.num_units < info.sms ? p.num_units : info.sms;
+  if (d == 64) {
+    if (causal)
+      return out_f32 ? launch<64, true, true, false, true>(tq, tk, tv, p, grid, dev, stream)
+                     : launch<64, true, false, false, true>(tq, tk, tv, p, grid, dev, stream);
+    return out_f32 ? launch<64, false, true, false, true>(tq, tk, tv, p, grid, dev, stream)
+                   : launch<64, false, false, false, true>(tq, tk, tv, p, grid, dev, stream);
+  }
+  if (causal)
+    return out_f32 ? launch<128, true, true, false, true>(tq, tk, tv, p, grid, dev, stream)
+                   : launch<128, true, false, false, true>(tq, tk, tv, p, grid, dev, stream);
+  return out_f32 ? launch<128, false, true, false, true>(tq, tk, tv, p, grid, dev, stream)
+                 : launch<128, false, false, false, true>(tq, tk, tv, p, grid, dev, stream);
 }
 
 // Shared-memory quantisation kernel: the smallest power-of-two cluster (<= 8 CTAs) that
@@ -598,6 +688,15 @@ fa_status fa_quantize_e4m3(const void *x, const int8_t *signs, void *x8, float *
                            int H, int N, int d, fa_stream_t stream) {
   return quantize_common(x, signs, x8, descale, B, H, N, d,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int Hq, int Hkv,
+                        int total_q, int total_k, int max_seqlen_q, int d, float scale,
+                        int causal, fa_dtype dtype, fa_stream_t stream) {
+  return fwd_varlen_common(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, total_q,
+                           total_k, max_seqlen_q, d, scale, causal, dtype,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,

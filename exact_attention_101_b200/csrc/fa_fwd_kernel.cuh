@@ -149,25 +149,45 @@ struct FwdParams {
   const float *descale_q;  // fp8 only: [B*Hq]
   const float *descale_k;  // fp8 only: [B*Hkv]
   const float *descale_v;  // fp8 only: [B*Hkv]
-  int B, Hq, Hkv, Nq, Nk;
+  const int *cu_q;         // varlen only: [B+1] first token of each query sequence
+  const int *cu_k;         // varlen only: [B+1] first token of each key sequence
+  int B, Hq, Hkv, Nq, Nk;  // varlen: Nq, Nk = total tokens of the packed Q and K tensors
   int group;        // Hq / Hkv
-  int num_qb;       // ceil(Nq / UNIT_ROWS)
+  int num_qb;       // ceil(Nq / UNIT_ROWS); varlen: ceil(longest query sequence / UNIT_ROWS)
   int num_units;    // B * Hq * num_qb
   float scale_log2; // softmax scale * log2(e)
 };
 
 struct Unit {
-  int bh;   // b * Hq + hq
-  int bhk;  // b * Hkv + hq / group
-  int r0;   // first query row of the unit
-  int n0;   // key tiles visited by Q tile 0
-  int n1;   // key tiles visited by Q tile 1 (>= n0)
+  int bh;     // b * Hq + hq
+  int bhk;    // b * Hkv + hq / group
+  int qh, kh; // head coordinate of the Q and K/V tensor maps (bh, bhk; varlen: hq, hk)
+  int q_tok;  // varlen: token of the sequence's first query in the packed tensor (else 0)
+  int k_tok;  // varlen: token of the sequence's first key (else 0)
+  int len_q;  // queries of the sequence (Nq for fixed length)
+  int len_k;  // keys of the sequence (Nk)
+  int off;    // causal diagonal: query i sees keys j <= i + off (off = len_k - len_q)
+  int r0;     // first query row of the unit, within its sequence
+  int n0;     // key tiles visited by Q tile 0 (at least 1)
+  int n1;     // key tiles visited by Q tile 1 (>= n0)
+  bool empty; // varlen: the unit starts past the end of its sequence
 };
+
+// Key tiles that query rows up to `last_row` visit: all of them, or under the causal mask
+// those up to the diagonal.  At least one, so that a row without admissible keys still
+// runs through the pipeline (its scores are all masked and it gets O = 0, LSE = -inf).
+template <bool CAUSAL>
+__device__ __forceinline__ int key_tiles(int last_row, int len_k, int off) {
+  const int last_key = CAUSAL ? min(len_k - 1, last_row + off) : len_k - 1;
+  return last_key < 0 ? 1 : last_key / BN + 1;
+}
 
 // Work list: head-major, so that the CTAs running at the same time share the K/V of a
 // few heads in L2 (and query heads that share a K/V head are neighbours); inside a head
-// the query blocks run last-first, i.e. longest-first under the causal mask.
-template <bool CAUSAL>
+// the query blocks run last-first, i.e. longest-first under the causal mask.  With
+// variable lengths every sequence gets num_qb blocks (those of the longest sequence); the
+// blocks past the end of a shorter sequence are empty and skipped by every role.
+template <bool CAUSAL, bool VARLEN>
 __device__ __forceinline__ Unit decode_unit(const FwdParams &p, int u) {
   const int qb = p.num_qb - 1 - u % p.num_qb;
   Unit w;
@@ -175,14 +195,25 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams &p, int u) {
   const int b = w.bh / p.Hq, hq = w.bh % p.Hq;
   w.bhk = b * p.Hkv + hq / p.group;
   w.r0 = qb * UNIT_ROWS;
-  const int nkt = (p.Nk + BN - 1) / BN;
-  if (CAUSAL) {
-    w.n0 = min(p.Nk - 1, w.r0 + BM - 1) / BN + 1;
-    w.n1 = min(p.Nk - 1, w.r0 + 2 * BM - 1) / BN + 1;
+  if (VARLEN) {
+    w.qh = hq;
+    w.kh = hq / p.group;
+    w.q_tok = p.cu_q[b];
+    w.k_tok = p.cu_k[b];
+    w.len_q = p.cu_q[b + 1] - w.q_tok;
+    w.len_k = p.cu_k[b + 1] - w.k_tok;
   } else {
-    w.n0 = nkt;
-    w.n1 = nkt;
+    w.qh = w.bh;
+    w.kh = w.bhk;
+    w.q_tok = 0;
+    w.k_tok = 0;
+    w.len_q = p.Nq;
+    w.len_k = p.Nk;
   }
+  w.empty = VARLEN && w.r0 >= w.len_q;
+  w.off = w.len_k - w.len_q;
+  w.n0 = key_tiles<CAUSAL>(w.r0 + BM - 1, w.len_k, w.off);
+  w.n1 = key_tiles<CAUSAL>(w.r0 + 2 * BM - 1, w.len_k, w.off);
   return w;
 }
 
@@ -241,7 +272,7 @@ struct Bars {
 
 // ---------------------------------------------------------------------------- producer
 
-template <int D, bool CAUSAL, bool FP8>
+template <int D, bool CAUSAL, bool FP8, bool VARLEN>
 __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                           const FwdParams &p, uint32_t smem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
                           volatile uint32_t *abort_flag) {
@@ -252,15 +283,18 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
   uint32_t issued = 0;    // K/V slot loads issued so far
   uint32_t q_issued = 0;  // Q loads issued so far
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const Unit w = decode_unit<CAUSAL>(p, u);
+    const Unit w = decode_unit<CAUSAL, VARLEN>(p, u);
+    if (VARLEN && w.empty) continue;
     if (!wait_phase(bar.q_empty(), (q_issued & 1u) ^ 1u, abort_flag, ERR_WAIT_LOAD)) goto drain;
     ptx::mbar_arrive_expect_tx(bar.q_full(), 2 * C::Q_TILE_BYTES);
 #pragma unroll
     for (int x = 0; x < 2; ++x)
 #pragma unroll
       for (int bx = 0; bx < C::NBOX; ++bx)
+        // fixed length: map {d, rows, heads}; packed varlen: map {d, heads, tokens}
         ptx::tma_load_3d(smem + C::Q_OFF + x * C::Q_TILE_BYTES + bx * C::Q_BOX_BYTES, tmQ,
-                         bar.q_full(), bx * C::BOX_ELEMS, w.r0 + x * BM, w.bh);
+                         bar.q_full(), bx * C::BOX_ELEMS,
+                         VARLEN ? w.qh : w.r0 + x * BM, VARLEN ? w.q_tok + w.r0 + x * BM : w.qh);
     ++q_issued;
     for (int j = 0; j < w.n1; ++j) {
 #pragma unroll
@@ -272,7 +306,8 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
           ptx::tma_load_3d(smem + C::RING_OFF + s * C::KV_TILE_BYTES + bx * C::KV_BOX_BYTES,
-                           t ? tmV : tmK, bar.slot_full(s), bx * C::BOX_ELEMS, j * BN, w.bhk);
+                           t ? tmV : tmK, bar.slot_full(s), bx * C::BOX_ELEMS,
+                           VARLEN ? w.kh : j * BN, VARLEN ? w.k_tok + j * BN : w.kh);
         ++issued;
       }
     }
@@ -338,7 +373,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint6
 // two arrivals, one per tile.  Key tiles that only tile 1 visits (causal) get tile 0's
 // arrival from tile 1's warp as a plain arrive; it happens only after the slot's load has
 // landed, so it can never complete the slot's previous phase early.
-template <int D, bool CAUSAL, bool FP8>
+template <int D, bool CAUSAL, bool FP8, bool VARLEN>
 __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
                          const Bars<TileCfg<D, FP8>::NSLOT> &bar, const int x,
                          volatile uint32_t *abort_flag) {
@@ -369,8 +404,9 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
     release(ki, x == 1 && j >= w.n0);
     if (j == nx - 1) ptx::mma_commit_elect(bar.q_empty());
   };
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++unit_it) {
-    const Unit w = decode_unit<CAUSAL>(p, u);
+  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    const Unit w = decode_unit<CAUSAL, VARLEN>(p, u);
+    if (VARLEN && w.empty) continue;
     const int nx = x ? w.n1 : w.n0;
     if (!wait(bar.q_full(), unit_it & 1u)) break;
     bool ok = true;
@@ -401,6 +437,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
     }
     if (!ok) break;
     kv_base += 2 * w.n1;
+    ++unit_it;
   }
   // Wait until every MMA issued by this warp has finished before TMEM is freed.
   ptx::mma_commit_elect(bar.drain(x));
@@ -499,7 +536,7 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], 
 // (TMEM lane).  Every 64-key score tile is loaded whole into registers, masked if it
 // crosses the diagonal or the end of the keys, turned into numerators in place, and the
 // row statistics are carried from tile to tile.
-template <int D, bool CAUSAL, bool OUT_F32, bool FP8>
+template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN>
 __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
                              volatile uint32_t *abort_flag) {
   using C = TileCfg<D, FP8>;
@@ -514,15 +551,17 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
   uint32_t pv_base = 0;  // P.V products of this tile in earlier units
   uint32_t unit_it = 0;
 
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++unit_it) {
-    const Unit w = decode_unit<CAUSAL>(p, u);
+  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    const Unit w = decode_unit<CAUSAL, VARLEN>(p, u);
+    if (VARLEN && w.empty) continue;
     const int nx = x ? w.n1 : w.n0;
     const int row = w.r0 + x * BM + row_in_tile;     // query row of this thread
     const int tile_row0 = w.r0 + x * BM;
     float sl2 = p.scale_log2;
     if (FP8) sl2 *= p.descale_q[w.bh] * p.descale_k[w.bhk];
-    // Last admissible key for this row (keys beyond Nk never count).
-    const int key_lim = CAUSAL ? min(row, p.Nk - 1) : p.Nk - 1;
+    // Last admissible key for this row (keys beyond the sequence never count; negative if
+    // the row has none).
+    const int key_lim = CAUSAL ? min(row + w.off, w.len_k - 1) : w.len_k - 1;
     float m_used = NEG_INF;  // running maximum in use, base-2 scaled domain
     float l = 0.f;           // running sum of the numerators as rounded for the P V product
     float l_exact = 0.f;     // running sum of the unrounded numerators (for the LSE)
@@ -543,7 +582,8 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       for (int c = 0; c < 4; ++c) ptx::reg_fence16(sr[c]);
 
       const int kv0 = j * BN;
-      const bool need_mask = (CAUSAL && kv0 + BN - 1 > tile_row0) || (kv0 + BN > p.Nk);
+      const bool need_mask =
+          (CAUSAL && kv0 + BN - 1 > tile_row0 + w.off) || (kv0 + BN > w.len_k);
       if (need_mask) {
         const int lim = key_lim - kv0;  // column c is admissible iff c <= lim
 #pragma unroll
@@ -621,10 +661,17 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       bool ok = wait_phase(bar.o_full(x), unit_it & 1u, abort_flag, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;
       ptx::tc_fence_after();
-      float inv = 1.f / l;
+      // a row without admissible keys (causal, more queries than keys) has l = 0: O = 0
+      float inv = l > 0.f ? 1.f / l : 0.f;
       if (FP8) inv *= p.descale_v[w.bhk];
-      const bool valid = row < p.Nq;
-      const size_t orow = static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
+      // packed varlen output: O [tokens, Hq, d], LSE [Hq, tokens]; the token check keeps
+      // the stores inside the tensors whatever the offsets say
+      const bool valid = row < w.len_q && (!VARLEN || w.q_tok + row < p.Nq);
+      const int hq = w.bh % p.Hq;
+      const size_t orow = VARLEN ? static_cast<size_t>(w.q_tok + (valid ? row : 0)) * p.Hq + hq
+                                 : static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
+      const size_t lrow = VARLEN ? static_cast<size_t>(hq) * p.Nq + w.q_tok + (valid ? row : 0)
+                                 : orow;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t a[16], bb[16];
@@ -658,16 +705,19 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
           }
         }
       }
-      if (valid) p.lse[orow] = (m_used + log2f(l_exact)) * 0.69314718055994530942f;
+      if (valid)
+        p.lse[lrow] = l_exact > 0.f ? (m_used + log2f(l_exact)) * 0.69314718055994530942f
+                                    : NEG_INF;
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.o_empty(x));
     }
+    ++unit_it;
   }
 }
 
 // ---------------------------------------------------------------------------- kernel
 
-template <int D, bool CAUSAL, bool OUT_F32, bool FP8>
+template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -720,12 +770,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::setmaxnreg_dec<OTHER_REGS>();
 
   if (warp < 8) {
-    softmax_role<D, CAUSAL, OUT_F32, FP8>(p, tmem, bar, abort_flag);
+    softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN>(p, tmem, bar, abort_flag);
   } else if (warp == MMA_WARP || warp == MMA_WARP + 2) {
-    mma_role<D, CAUSAL, FP8>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, abort_flag);
+    mma_role<D, CAUSAL, FP8, VARLEN>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, abort_flag);
     __syncwarp();
   } else if (warp == TMA_WARP) {
-    if (lane == 0) load_role<D, CAUSAL, FP8>(&tmQ, &tmK, &tmV, p, smem, bar, abort_flag);
+    if (lane == 0) load_role<D, CAUSAL, FP8, VARLEN>(&tmQ, &tmK, &tmV, p, smem, bar, abort_flag);
     __syncwarp();
   }
 

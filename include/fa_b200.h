@@ -20,7 +20,10 @@
  *   o : [B, Hq,  Nq, d]      lse  : [B, Hq,  Nq]  (fp32)
  * Grouped-query / multi-query attention: Hq must be a multiple of Hkv and query head hq
  * reads K/V head hq / (Hq / Hkv) (consecutive query heads share a K/V head).
- * Causal masking admits key j for query i iff j <= i and requires Nq == Nk.
+ * Causal masking admits key j for query i iff j <= i + (Nk - Nq): with Nq == Nk that is
+ * j <= i, and otherwise the queries are taken as the last Nq positions of the Nk keys
+ * (bottom-right alignment).  A query row with no admissible key (Nq > Nk) gets O = 0 and
+ * LSE = -inf.
  *
  * Ownership: the caller allocates and owns every buffer.  The library keeps no pointer
  * after a call returns and allocates no device memory, except fa_bwd, which allocates
@@ -50,7 +53,8 @@ typedef enum fa_status {
     FA_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, bad size, bad scale, buffer
                                 too small for the given shape or not device memory */
     FA_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement: head
-                                dim not 64/128, causal with Nq != Nk, GPU not sm_100 */
+                                dim not 64/128, GPU not sm_100, and the limits stated
+                                at each entry point */
     FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, attribute) */
     FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (see below) */
 } fa_status;
@@ -80,6 +84,32 @@ typedef enum fa_dtype {
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                  int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                  fa_dtype dtype, fa_stream_t stream);
+
+/*
+ * Fused attention forward over a batch of sequences of different lengths, packed without
+ * padding: the page "FlashAttention 4: Praxisleitfaden ..." (section "Kompatibilitaet und
+ * aktueller Stand") describes variable sequence lengths as batching sequences of
+ * different length without padding, addressed through cu_seqlens offsets.
+ *
+ *   q           bf16 [total_q, Hq, d]   (token-major: the Hq heads of a token adjacent)
+ *   k, v        bf16 [total_k, Hkv, d]
+ *   o           bf16 or fp32 (dtype) [total_q, Hq, d]
+ *   lse         fp32 [Hq, total_q]
+ *   cu_seqlens_q, cu_seqlens_k   device int32 arrays of B+1 entries: sequence b has
+ *               query tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and key tokens
+ *               cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1.  Entries must be non-decreasing,
+ *               start at 0 and end at total_q / total_k.
+ *   max_seqlen_q   at least the longest query sequence (work is planned for it)
+ *   d           64 or 128;  dtype FA_BF16 or FA_BF16_OUT_F32
+ *
+ * Each sequence is attended on its own; causal masking is per sequence, bottom-right
+ * aligned as above.  The offsets are read on the device: wrong offsets give wrong results
+ * but every load and store stays inside the tensors.  Errors as for fa_fwd.
+ */
+fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int Hq,
+                        int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
+                        float scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
  * Fused attention forward, fp8 (OCP e4m3) inputs with per-(batch, head) scales, fp32
@@ -116,7 +146,8 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
  *   o, lse      the forward's outputs for these inputs (o bf16 [B,Hq,Nq,d], lse fp32)
  *   dout        bf16 [B,Hq,Nq,d], the gradient of the loss with respect to o
  *   dq          bf16 [B,Hq,Nq,d] out;  dk, dv  bf16 [B,Hkv,Nk,d] out
- *   B, Hq, Hkv, Nq, Nk, scale, causal   as for fa_fwd;  d must be 128
+ *   B, Hq, Hkv, Nq, Nk, scale, causal   as for fa_fwd;  d must be 128; causal requires
+ *   Nq == Nk
  *
  * All pointers 16-byte aligned (lse 4-byte).  The outputs must not overlap the inputs.
  * Scratch: the call allocates B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes on `stream` with

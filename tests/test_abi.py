@@ -74,7 +74,7 @@ def test_invalid_arguments(kw):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(d=96), dict(d=256), dict(d=32), dict(causal=1, Nq=256, Nk=512),
+    dict(d=96), dict(d=256), dict(d=32),
 ])
 def test_unsupported_configurations(kw):
     assert call(**kw) == fa.FA_ERR_UNSUPPORTED
@@ -152,3 +152,29 @@ def test_bwd_noalloc_validates_like_fa_bwd_and_rejects_oversize_scratch():
     assert fa.fa_bwd_noalloc(*args(d=64)) == fa.FA_ERR_UNSUPPORTED
     # B*Hq*Nq*d*4 = 128 MiB of dQ accumulator: more than the fixed 64 MiB scratch
     assert fa.fa_bwd_noalloc(*args(Hq=16, Hkv=16, Nq=16384, Nk=16384)) == fa.FA_ERR_UNSUPPORTED
+
+
+VL_OK = dict(q=A, k=A, v=A, o=A, lse=A, cq=A, ck=A, B=2, Hq=4, Hkv=2, tq=300, tk=300, maxq=200,
+             d=128, scale=0.088, causal=0, dtype=fa.FA_BF16)
+
+
+def varlen_call(**kw):
+    a = dict(VL_OK)
+    a.update(kw)
+    return fa.fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cq"], a["ck"], a["B"],
+                            a["Hq"], a["Hkv"], a["tq"], a["tk"], a["maxq"], a["d"], a["scale"],
+                            a["causal"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=0), dict(cq=0), dict(ck=0), dict(cq=A + 2), dict(o=A + 8), dict(B=0), dict(tq=0),
+    dict(tk=0), dict(maxq=0), dict(Hq=3), dict(causal=3), dict(scale=-1.0),
+    dict(dtype=fa.FA_E4M3),
+])
+def test_varlen_invalid_arguments(kw):
+    assert varlen_call(**kw) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [32, 96, 256])
+def test_varlen_unsupported_head_dims(d):
+    assert varlen_call(d=d) == fa.FA_ERR_UNSUPPORTED

@@ -1,0 +1,117 @@
+"""GPU parity of variable-length (packed, cu_seqlens) attention and of causal attention with
+Nq != Nk (bottom-right alignment) against the fp64 oracle, sequence by sequence.
+
+Variable sequence lengths batch sequences of different length without padding (page
+"FlashAttention 4: Praxisleitfaden ...", section "Kompatibilitaet und aktueller Stand").
+Rows without any admissible key (causal with more queries than keys, or no keys at all)
+must come out as O = 0 and LSE = -inf.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_101_b200 as fa
+import oracle
+from parity_util import compare_bf16
+from workloads import random_bf16
+
+pytestmark = pytest.mark.gpu
+
+D_SCALE = {64: 0.125, 128: float(torch.tensor(1 / np.sqrt(128), dtype=torch.float32))}
+
+
+def packed(lengths, H, d, seed):
+    total = int(sum(lengths))
+    return random_bf16((max(total, 1), H, d), seed)[:total].contiguous()
+
+
+def cu(lengths):
+    return torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
+
+
+def check_rows(o_gpu, lse_gpu, o_ref, lse_ref):
+    """Rows with keys: bf16 tolerances.  Rows without: O = 0, LSE = -inf exactly."""
+    empty = np.isneginf(lse_ref)
+    lg = lse_gpu.double().numpy()
+    assert np.all(np.isneginf(lg[empty])), "rows without keys must have LSE = -inf"
+    assert np.all(o_gpu.double().numpy()[empty] == 0.0), "rows without keys must have O = 0"
+    if (~empty).any():
+        return compare_bf16(o_gpu[torch.from_numpy(~empty)], lse_gpu[torch.from_numpy(~empty)],
+                            o_ref[~empty], lse_ref[~empty])
+    return {}
+
+
+def run_varlen_case(lq, lk, Hq, Hkv, d, causal, seed, out_dtype=torch.bfloat16):
+    dev = torch.device("cuda", 0)
+    q, k, v = packed(lq, Hq, d, seed), packed(lk, Hkv, d, seed + 1), packed(lk, Hkv, d, seed + 2)
+    cq, ck = cu(lq), cu(lk)
+    scale = D_SCALE[d]
+    o, lse = fa.forward_varlen(q.to(dev), k.to(dev), v.to(dev), cq.to(dev), ck.to(dev),
+                               max(max(lq), 1), causal=causal, scale=scale, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+    o, lse = o.cpu(), lse.cpu()
+    stats = []
+    for b in range(len(lq)):
+        if lq[b] == 0:
+            continue
+        qs = q[cq[b]:cq[b + 1]].transpose(0, 1).unsqueeze(0).contiguous()
+        if lk[b] == 0:   # no keys at all: every row is empty
+            assert torch.all(o[cq[b]:cq[b + 1]] == 0) and torch.isneginf(lse[:, cq[b]:cq[b + 1]]).all()
+            continue
+        ks = k[ck[b]:ck[b + 1]].transpose(0, 1).unsqueeze(0).contiguous()
+        vs = v[ck[b]:ck[b + 1]].transpose(0, 1).unsqueeze(0).contiguous()
+        ro, rl = oracle.attention(qs, ks, vs, scale, causal)
+        go = o[cq[b]:cq[b + 1]].transpose(0, 1)           # [Hq, len, d]
+        gl = lse[:, cq[b]:cq[b + 1]]                     # [Hq, len]
+        stats.append(check_rows(go.reshape(-1, d), gl.reshape(-1), ro[0].reshape(-1, d),
+                                rl[0].reshape(-1)))
+    return stats
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_self_attention(cuda_ok, d, causal):
+    lengths = [1, 17, 128, 129, 256, 300, 511, 64, 1000]
+    print(run_varlen_case(lengths, lengths, 4, 2, d, causal, seed=100 + d))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_cross_lengths_and_empty_sequences(cuda_ok, causal):
+    lq = [5, 0, 300, 70, 257, 3]
+    lk = [9, 4, 100, 0, 600, 3]
+    print(run_varlen_case(lq, lk, 2, 1, 128, causal, seed=200))
+
+
+def test_varlen_fp32_output(cuda_ok):
+    print(run_varlen_case([33, 190, 700], [33, 190, 700], 2, 2, 128, True, seed=300,
+                          out_dtype=torch.float32))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equal_lengths_equal_fixed_length_bits(cuda_ok, causal):
+    """Packed sequences of one length run the same tiles as the [B, H, N, d] path."""
+    dev = torch.device("cuda", 0)
+    B, H, N, d = 3, 4, 385, 128
+    q, k, v = (random_bf16((B, H, N, d), 400 + s) for s in range(3))
+    o1, l1 = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal=causal, scale=D_SCALE[d])
+    pk = lambda t: t.permute(0, 2, 1, 3).reshape(B * N, H, d).contiguous().to(dev)
+    c = cu([N] * B).to(dev)
+    o2, l2 = fa.forward_varlen(pk(q), pk(k), pk(v), c, c, N, causal=causal, scale=D_SCALE[d])
+    torch.cuda.synchronize()
+    assert torch.equal(o1.permute(0, 2, 1, 3).reshape(B * N, H, d), o2)
+    assert torch.equal(l1.permute(1, 0, 2).reshape(H, B * N), l2)
+
+
+@pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (129, 513), (513, 129), (1, 700)])
+def test_fixed_length_causal_bottom_right(cuda_ok, nq, nk):
+    dev = torch.device("cuda", 0)
+    B, Hq, Hkv, d = 1, 4, 2, 128
+    q = random_bf16((B, Hq, nq, d), 500)
+    k, v = random_bf16((B, Hkv, nk, d), 501), random_bf16((B, Hkv, nk, d), 502)
+    o, lse = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal=True, scale=D_SCALE[d])
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+    ro, rl = oracle.attention(q, k, v, D_SCALE[d], True)
+    print(check_rows(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), ro.reshape(-1, d),
+                     rl.reshape(-1)))
