@@ -235,6 +235,35 @@ def oracle_bwd_sample(w, inp, target_s):
     return flops / dt / 1e12, desc, oracle.max_threads(), dt
 
 
+def oracle_varlen_sample(w, inp, target_s, seed=0):
+    """Time the fp64 oracle on random (sequence, head, query) rows of a varlen workload,
+    drawing rows until about target_s of oracle time.  Returns (TFLOP/s, description,
+    threads, seconds)."""
+    import numpy as np
+    import torch
+    import oracle
+    rng = np.random.default_rng(seed)
+    cu = inp.cu_seqlens.tolist()
+    flops, dt, rows = 0.0, 0.0, 0
+    while dt < target_s:
+        b = int(rng.integers(0, w.B))
+        n = cu[b + 1] - cu[b]
+        # bf16 bits as numpy, prepared outside the timed call
+        seq = lambda t: t[cu[b]:cu[b + 1]].transpose(0, 1).unsqueeze(0).contiguous().view(
+            torch.int16).numpy()
+        q, k, v = seq(inp.q), seq(inp.k), seq(inp.v)
+        r = rng.integers(0, w.Hq * n, size=256)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, w.scale, w.causal, rows=r)
+        dt += time.perf_counter() - t0
+        keys = (r % n + 1) if w.causal else np.full(r.shape, n)
+        flops += 4.0 * w.d * float(keys.sum())
+        rows += len(r)
+    desc = ("%d random (sequence, head, query) rows of workload %s, each over its admissible "
+            "keys, fp64" % (rows, w.name))
+    return flops / dt / 1e12, desc, oracle.max_threads(), dt
+
+
 def oracle_sample_rate(w, inp, target_s, seed=0):
     """Calibrate, then time one sample of about target_s seconds."""
     n = oracle_calibrate(w, inp, target_s, seed)
@@ -277,6 +306,13 @@ def run_ours(args):
     # every step, then run the fp8 kernel: 3 quantisation kernels + 1 attention kernel.
     launches_per_step = 4 if w.rotate else (3 if w.kind == "bwd" else 1)
     split = None
+    if w.kind == "varlen":
+        host.append(inp.cu_seqlens)
+        cu_d = inp.cu_seqlens.to(dev)
+        total = int(inp.cu_seqlens[-1])
+        max_len = max(workloads.varlen_lengths(w))
+        o = torch.empty((total, w.Hq, w.d), dtype=out_dtype, device=dev)
+        lse = torch.empty((w.Hq, total), dtype=torch.float32, device=dev)
     if w.kind == "bwd":
         # The forward's O and LSE, computed once before timing; each step is one backward.
         host += [inp.dout]
@@ -311,6 +347,9 @@ def run_ours(args):
         elif w.kind == "bwd":
             fa.backward(q, k, v, o, lse, dout, causal=w.causal, scale=w.scale, dq=dq, dk=dk,
                         dv=dv)
+        elif w.kind == "varlen":
+            fa.forward_varlen(q, k, v, cu_d, cu_d, max_len, causal=w.causal, scale=w.scale,
+                              out_dtype=out_dtype, out=o, lse=lse)
         elif fp8:
             fa.forward_fp8(q, k, v, dq, dk, dv, causal=w.causal, scale=w.scale, out=o, lse=lse)
         else:
@@ -373,6 +412,8 @@ def run_ours(args):
         hdq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
         hdk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
         hdv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+    if w.kind == "varlen":
+        hcu_ = inp.cu_seqlens.pin_memory()
     if w.rotate:
         hs_ = inp.signs.pin_memory()
     elif fp8:
@@ -389,6 +430,8 @@ def run_ours(args):
             for dst, src in ((hdq, dq), (hdk, dk), (hdv, dv)):
                 dst.copy_(src, non_blocking=True)
             return
+        if w.kind == "varlen":
+            cu_d.copy_(hcu_, non_blocking=True)
         if w.rotate:
             signs.copy_(hs_, non_blocking=True)
         elif fp8:
@@ -442,6 +485,8 @@ def run_ours(args):
     if not args.no_cpu_baseline and world == 1:
         if w.kind == "bwd":
             rate, desc, cores, _ = oracle_bwd_sample(w, inp, args.cpu_seconds)
+        elif w.kind == "varlen":
+            rate, desc, cores, _ = oracle_varlen_sample(w, inp, args.cpu_seconds)
         else:
             rate, desc, cores, _, _ = oracle_sample_rate(w, inp, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
@@ -497,6 +542,8 @@ def run_reference(args):
     per_step = max(0.05, args.reference_budget_s / max(1, args.steps + args.warmup))
     if w.kind == "bwd":
         return run_reference_bwd(args, w, inp, per_step, world)
+    if w.kind == "varlen":
+        return run_reference_sampled(args, w, inp, per_step, world, oracle_varlen_sample)
     n_rows = oracle_calibrate(w, inp, per_step)
     for i in range(args.warmup):
         oracle_timed_sample(w, inp, n_rows, seed=100 + i)
@@ -524,11 +571,15 @@ def run_reference(args):
 
 
 def run_reference_bwd(args, w, inp, per_step, world):
+    return run_reference_sampled(args, w, inp, per_step, world, oracle_bwd_sample)
+
+
+def run_reference_sampled(args, w, inp, per_step, world, sampler):
     for _ in range(args.warmup):
-        oracle_bwd_sample(w, inp, per_step)
+        sampler(w, inp, per_step)
     rates, total_s, desc, cores = [], 0.0, "", 1
     for _ in range(args.steps):
-        rate, desc, cores, dt = oracle_bwd_sample(w, inp, per_step)
+        rate, desc, cores, dt = sampler(w, inp, per_step)
         rates.append(rate)
         total_s += dt
     value = statistics.median(rates)

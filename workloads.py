@@ -20,7 +20,9 @@ bf16 Q/K/V with the fp8 case's outliers, or with a few outlier channels shared b
 K, that the library quantises itself after a random-sign Hadamard rotation of Q and K.
 Their sign vector is drawn here, after the values, and passed to the library as input.
 Backward workloads (``kind="bwd"``) use the forward shapes and draw the upstream gradient
-dO after V, i.i.d. N(0, 1) in bf16.
+dO after V, i.i.d. N(0, 1) in bf16.  The variable-length workload (``kind="varlen"``)
+packs B sequences whose lengths are drawn uniformly (the pages give no length mix) into
+token-major tensors with cu_seqlens offsets.
 """
 from __future__ import annotations
 
@@ -51,7 +53,10 @@ class Workload:
     #                               channels of Q and K (outlier_channels of them)
     outlier_channels: int = 0
     rotate: bool = False          # bf16 source quantised on the GPU with Hadamard rotation
-    kind: str = "fwd"             # "fwd": forward pass; "bwd": backward pass (dO drawn too)
+    kind: str = "fwd"             # "fwd": forward pass; "bwd": backward pass (dO drawn too);
+    #                               "varlen": B packed sequences of lengths drawn in
+    #                               [min_len, N] (token-major [tokens, H, d] tensors)
+    min_len: int = 0
 
     @property
     def scale(self) -> float:
@@ -61,7 +66,11 @@ class Workload:
     @property
     def flops(self) -> float:
         """Algorithmic FLOPs: forward 4*B*Hq*Nq*Nk*d (two products), backward 2.5 times
-        that (five products); halved under the causal mask."""
+        that (five products); halved under the causal mask.  Variable lengths: the sum of
+        4*Hq*len^2*d over the sequences."""
+        if self.kind == "varlen":
+            f = sum(4.0 * self.Hq * n * n * self.d for n in varlen_lengths(self))
+            return f / 2 if self.causal else f
         f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
         if self.kind == "bwd":
             f *= 2.5
@@ -76,6 +85,11 @@ class Workload:
             out["quantise"] = "e4m3 per head on the GPU, Q and K after random-sign Hadamard"
         if self.kind == "bwd":
             out["pass"] = "backward (dQ, dK, dV from Q, K, V, O, LSE, dO)"
+        if self.kind == "varlen":
+            lens = varlen_lengths(self)
+            out.update({"Nq": None, "Nk": None, "sequences": self.B, "total_tokens": sum(lens),
+                        "lengths": "uniform integers in [%d, %d], seeded" % (self.min_len, self.N),
+                        "layout": "packed [tokens, H, d] with cu_seqlens"})
         return out
 
 
@@ -91,6 +105,8 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
              rotate=True),
     Workload("fp8_incoherent_channels", 8, 16, 16, 4096, 128, False, "bf16", "bf16", 1007,
              1.0, 10.0, outlier_kind="channel", outlier_channels=4, rotate=True),
+    Workload("varlen_causal", 16, 32, 32, 8192, 128, True, "bf16", "bf16", 1008, kind="varlen",
+             min_len=256),
     Workload("long_bwd", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003, kind="bwd"),
     Workload("long_causal_bwd", 1, 32, 32, 16384, 128, True, "bf16", "bf16", 1003, kind="bwd"),
     Workload("gqa_causal_bwd", 4, 32, 8, 8192, 128, True, "bf16", "bf16", 1004, kind="bwd"),
@@ -106,6 +122,7 @@ class Inputs:
     descale_k: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
     descale_v: Optional[torch.Tensor] = None   # fp32 [B*Hkv]
     signs: Optional[torch.Tensor] = None       # int8 [d] of +-1 (rotate workloads only)
+    cu_seqlens: Optional[torch.Tensor] = None  # int32 [B+1] (varlen workloads only)
     dout: Optional[torch.Tensor] = None        # bf16 [B, Hq, Nq, d] (backward workloads only)
 
 
@@ -122,6 +139,14 @@ def _quantise_e4m3_per_head(x: torch.Tensor):
     return y.to(torch.float8_e4m3fn).contiguous(), s.reshape(B * H).contiguous()
 
 
+def varlen_lengths(w: Workload):
+    """Sequence lengths of a varlen workload: B uniform integers in [min_len, N], from their
+    own generator seeded with the workload seed."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    return [int(n) for n in torch.randint(w.min_len, w.N + 1, (w.B,), generator=g)]
+
+
 def make_inputs(w: Workload, seed: Optional[int] = None, *, B: Optional[int] = None,
                 Hq: Optional[int] = None, Hkv: Optional[int] = None,
                 Nq: Optional[int] = None, Nk: Optional[int] = None,
@@ -136,6 +161,14 @@ def make_inputs(w: Workload, seed: Optional[int] = None, *, B: Optional[int] = N
     d = w.d if d is None else d
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed if seed is None else seed)
+    if w.kind == "varlen":
+        lens = varlen_lengths(w)
+        total = sum(lens)
+        q = torch.randn((total, Hq, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+        k = torch.randn((total, Hkv, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+        v = torch.randn((total, Hkv, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+        cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0)), dtype=torch.int32)
+        return Inputs(q, k, v, cu_seqlens=cu)
     q32 = torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32)
     k32 = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
     v32 = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
