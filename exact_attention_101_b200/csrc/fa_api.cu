@@ -170,11 +170,12 @@ fa_status check_args(const void *q, const void *k, const void *v, const void *o,
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   // Index ranges: work-unit and row counts must fit the kernel's 32-bit arithmetic.
   const int64_t bh = static_cast<int64_t>(B) * Hq;
-  const int64_t units = bh * ((static_cast<int64_t>(Nq) + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS);
+  const int64_t unit_rows = d > 128 ? fa::BM : fa::UNIT_ROWS;
+  const int64_t units = bh * ((static_cast<int64_t>(Nq) + unit_rows - 1) / unit_rows);
   if (bh > INT32_MAX || static_cast<int64_t>(B) * Hkv > INT32_MAX || units > INT32_MAX)
     return FA_ERR_INVALID_ARG;
   if (Nk > INT32_MAX - 2 * fa::BN || Nq > INT32_MAX - 2 * fa::UNIT_ROWS) return FA_ERR_INVALID_ARG;
-  if (fp8 ? d != 128 : (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (fp8 ? d != 128 : (d != 64 && d != 128 && d != 256)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -226,7 +227,8 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
   p.Nq = Nq;
   p.Nk = Nk;
   p.group = Hq / Hkv;
-  p.num_qb = (Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  const int unit_rows = d > 128 ? fa::BM : fa::UNIT_ROWS;  // one Q tile per unit at d = 256
+  p.num_qb = (Nq + unit_rows - 1) / unit_rows;
   p.num_units = B * Hq * p.num_qb;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   const int grid = p.num_units < info.sms ? p.num_units : info.sms;
@@ -241,6 +243,13 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
                      : launch<64, true, false, false>(tq, tk, tv, p, grid, dev, stream);
     return out_f32 ? launch<64, false, true, false>(tq, tk, tv, p, grid, dev, stream)
                    : launch<64, false, false, false>(tq, tk, tv, p, grid, dev, stream);
+  }
+  if (d == 256) {
+    if (causal)
+      return out_f32 ? launch<256, true, true, false>(tq, tk, tv, p, grid, dev, stream)
+                     : launch<256, true, false, false>(tq, tk, tv, p, grid, dev, stream);
+    return out_f32 ? launch<256, false, true, false>(tq, tk, tv, p, grid, dev, stream)
+                   : launch<256, false, false, false>(tq, tk, tv, p, grid, dev, stream);
   }
   if (causal)
     return out_f32 ? launch<128, true, true, false>(tq, tk, tv, p, grid, dev, stream)
@@ -279,11 +288,12 @@ fa_status fwd_varlen_common(const void *q, const void *k, const void *v, void *o
   if (Hq % Hkv != 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_BF16_OUT_F32) return FA_ERR_INVALID_ARG;
-  const int64_t num_qb = (static_cast<int64_t>(max_q) + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  const int64_t unit_rows = d > 128 ? fa::BM : fa::UNIT_ROWS;  // one Q tile per unit at d = 256
+  const int64_t num_qb = (static_cast<int64_t>(max_q) + unit_rows - 1) / unit_rows;
   if (static_cast<int64_t>(B) * Hq * num_qb > INT32_MAX || max_q > INT32_MAX - 2 * fa::UNIT_ROWS ||
       total_k > INT32_MAX - 2 * fa::BN || total_q > INT32_MAX - 2 * fa::UNIT_ROWS)
     return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
 
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
@@ -330,6 +340,13 @@ fa_status fwd_varlen_common(const void *q, const void *k, const void *v, void *o
                      : launch<64, true, false, false, true>(tq, tk, tv, p, grid, dev, stream);
     return out_f32 ? launch<64, false, true, false, true>(tq, tk, tv, p, grid, dev, stream)
                    : launch<64, false, false, false, true>(tq, tk, tv, p, grid, dev, stream);
+  }
+  if (d == 256) {
+    if (causal)
+      return out_f32 ? launch<256, true, true, false, true>(tq, tk, tv, p, grid, dev, stream)
+                     : launch<256, true, false, false, true>(tq, tk, tv, p, grid, dev, stream);
+    return out_f32 ? launch<256, false, true, false, true>(tq, tk, tv, p, grid, dev, stream)
+                   : launch<256, false, false, false, true>(tq, tk, tv, p, grid, dev, stream);
   }
   if (causal)
     return out_f32 ? launch<128, true, true, false, true>(tq, tk, tv, p, grid, dev, stream)

@@ -17,6 +17,10 @@
 //   warp  9     TMA producer (one lane)
 //   warp  10    tcgen05.mma issuer for Q tile 1
 //   warp  11    idle (it completes the third warpgroup)
+// A unit is NT = 2 Q tiles (256 query rows) for head dims 64 and 128.  At head dim 256 a
+// second tile fits neither in tensor memory (two 256-column O accumulators) nor next to a
+// useful K/V ring in shared memory, so a unit is one Q tile (NT = 1) and warps 4-7 and 10
+// stay idle.
 //
 // Key tiles are BN = 64 keys, and every Q tile has TWO score buffers in tensor memory:
 // while the softmax warps of a tile turn S(j) into P(j), the tensor core already
@@ -109,6 +113,8 @@ constexpr uint32_t WAIT_MAX_ITERS = 1u << 28;
 
 template <int D, bool FP8>
 struct TileCfg {
+  static constexpr int NT = D > 128 ? 1 : 2;         // Q tiles per unit
+  static constexpr int UNIT = NT * BM;               // query rows per unit
   static constexpr int ELEM = FP8 ? 1 : 2;           // bytes per element
   static constexpr int ROW_BYTES = D * ELEM;         // bytes per tile row
   static_assert(ROW_BYTES % 128 == 0, "tile rows must be whole 128-byte swizzle rows");
@@ -118,7 +124,7 @@ struct TileCfg {
   static constexpr int KV_BOX_BYTES = BN * 128;      // 64 rows x 128 bytes
   static constexpr int Q_TILE_BYTES = NBOX * Q_BOX_BYTES;
   static constexpr int KV_TILE_BYTES = NBOX * KV_BOX_BYTES;
-  static constexpr int NSLOT = 131072 / KV_TILE_BYTES;  // 128 KB ring: 8 or 16 slots
+  static constexpr int NSLOT = 131072 / KV_TILE_BYTES;  // 128 KB ring: 4, 8 or 16 slots
   static_assert((NSLOT & (NSLOT - 1)) == 0, "ring size must be a power of two");
   static constexpr int MMA_K = FP8 ? 32 : 16;        // K extent of one MMA instruction
   static constexpr int S_KSTEPS = D / MMA_K;         // MMAs per S = Q K^T
@@ -129,10 +135,10 @@ struct TileCfg {
   // TMEM column map.
   static constexpr uint32_t P_OFF = 32;                  // P inside a 64-column S buffer
   static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
-  static_assert(256 + 2 * D <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(256 + NT * D <= (int)TMEM_COLS, "TMEM budget");
   // Shared memory map (offsets from a 1024-aligned base).
   static constexpr int Q_OFF = 0;
-  static constexpr int RING_OFF = 2 * Q_TILE_BYTES;
+  static constexpr int RING_OFF = NT * Q_TILE_BYTES;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * KV_TILE_BYTES;
   static constexpr int NUM_BARS = 2 * NSLOT + 18;
   static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
@@ -153,7 +159,7 @@ struct FwdParams {
   const int *cu_k;         // varlen only: [B+1] first token of each key sequence
   int B, Hq, Hkv, Nq, Nk;  // varlen: Nq, Nk = total tokens of the packed Q and K tensors
   int group;        // Hq / Hkv
-  int num_qb;       // ceil(Nq / UNIT_ROWS); varlen: ceil(longest query sequence / UNIT_ROWS)
+  int num_qb;       // ceil(Nq / unit rows); varlen: ceil(longest query sequence / unit rows)
   int num_units;    // B * Hq * num_qb
   float scale_log2; // softmax scale * log2(e)
 };
@@ -187,14 +193,14 @@ __device__ __forceinline__ int key_tiles(int last_row, int len_k, int off) {
 // the query blocks run last-first, i.e. longest-first under the causal mask.  With
 // variable lengths every sequence gets num_qb blocks (those of the longest sequence); the
 // blocks past the end of a shorter sequence are empty and skipped by every role.
-template <bool CAUSAL, bool VARLEN>
+template <bool CAUSAL, bool VARLEN, int UNIT = UNIT_ROWS>
 __device__ __forceinline__ Unit decode_unit(const FwdParams &p, int u) {
   const int qb = p.num_qb - 1 - u % p.num_qb;
   Unit w;
   w.bh = u / p.num_qb;
   const int b = w.bh / p.Hq, hq = w.bh % p.Hq;
   w.bhk = b * p.Hkv + hq / p.group;
-  w.r0 = qb * UNIT_ROWS;
+  w.r0 = qb * UNIT;
   if (VARLEN) {
     w.qh = hq;
     w.kh = hq / p.group;
@@ -213,7 +219,8 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams &p, int u) {
   w.empty = VARLEN && w.r0 >= w.len_q;
   w.off = w.len_k - w.len_q;
   w.n0 = key_tiles<CAUSAL>(w.r0 + BM - 1, w.len_k, w.off);
-  w.n1 = key_tiles<CAUSAL>(w.r0 + 2 * BM - 1, w.len_k, w.off);
+  // with one Q tile per unit there is no tile 1: the ring holds tile 0's key tiles only
+  w.n1 = UNIT > BM ? key_tiles<CAUSAL>(w.r0 + 2 * BM - 1, w.len_k, w.off) : w.n0;
   return w;
 }
 
@@ -283,12 +290,12 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
   uint32_t issued = 0;    // K/V slot loads issued so far
   uint32_t q_issued = 0;  // Q loads issued so far
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const Unit w = decode_unit<CAUSAL, VARLEN>(p, u);
+    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, u);
     if (VARLEN && w.empty) continue;
     if (!wait_phase(bar.q_empty(), (q_issued & 1u) ^ 1u, abort_flag, ERR_WAIT_LOAD)) goto drain;
-    ptx::mbar_arrive_expect_tx(bar.q_full(), 2 * C::Q_TILE_BYTES);
+    ptx::mbar_arrive_expect_tx(bar.q_full(), C::NT * C::Q_TILE_BYTES);
 #pragma unroll
-    for (int x = 0; x < 2; ++x)
+    for (int x = 0; x < C::NT; ++x)
 #pragma unroll
       for (int bx = 0; bx < C::NBOX; ++bx)
         // fixed length: map {d, rows, heads}; packed varlen: map {d, heads, tokens}
@@ -405,7 +412,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
     if (j == nx - 1) ptx::mma_commit_elect(bar.q_empty());
   };
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const Unit w = decode_unit<CAUSAL, VARLEN>(p, u);
+    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, u);
     if (VARLEN && w.empty) continue;
     const int nx = x ? w.n1 : w.n0;
     if (!wait(bar.q_full(), unit_it & 1u)) break;
@@ -552,7 +559,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
   uint32_t unit_it = 0;
 
   for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const Unit w = decode_unit<CAUSAL, VARLEN>(p, u);
+    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, u);
     if (VARLEN && w.empty) continue;
     const int nx = x ? w.n1 : w.n0;
     const int row = w.r0 + x * BM + row_in_tile;     // query row of this thread
@@ -737,10 +744,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
       ptx::mbar_init(bar.slot_full(s), 1);
-      ptx::mbar_init(bar.slot_empty(s), 2);   // one arrival per Q tile
+      ptx::mbar_init(bar.slot_empty(s), C::NT);   // one arrival per Q tile
     }
     ptx::mbar_init(bar.q_full(), 1);
-    ptx::mbar_init(bar.q_empty(), 2);
+    ptx::mbar_init(bar.q_empty(), C::NT);
     for (int x = 0; x < 2; ++x) {
       for (int b = 0; b < 2; ++b) {
         ptx::mbar_init(bar.s_full(x, b), 1);
@@ -769,9 +776,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   else
     ptx::setmaxnreg_dec<OTHER_REGS>();
 
-  if (warp < 8) {
+  if (warp < 4 * C::NT) {
     softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN>(p, tmem, bar, abort_flag);
-  } else if (warp == MMA_WARP || warp == MMA_WARP + 2) {
+  } else if (warp == MMA_WARP || (C::NT == 2 && warp == MMA_WARP + 2)) {
     mma_role<D, CAUSAL, FP8, VARLEN>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, abort_flag);
     __syncwarp();
   } else if (warp == TMA_WARP) {

@@ -74,7 +74,7 @@ def test_invalid_arguments(kw):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(d=96), dict(d=256), dict(d=32),
+    dict(d=96), dict(d=512), dict(d=32),
 ])
 def test_unsupported_configurations(kw):
     assert call(**kw) == fa.FA_ERR_UNSUPPORTED
@@ -88,6 +88,7 @@ def test_fp8_entry_validation():
     assert fa.fa_fwd_fp8(*args, 128, 0.1, 0, A + 2, A, A, None) == fa.FA_ERR_INVALID_ARG
     # fp8 supports d = 128 only
     assert fa.fa_fwd_fp8(*args, 64, 0.1, 0, A, A, A, None) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_fp8(*args, 256, 0.1, 0, A, A, A, None) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_status_strings():
@@ -175,6 +176,6 @@ def test_varlen_invalid_arguments(kw):
     assert varlen_call(**kw) == fa.FA_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("d", [32, 96, 256])
+@pytest.mark.parametrize("d", [32, 96, 512])
 def test_varlen_unsupported_head_dims(d):
     assert varlen_call(d=d) == fa.FA_ERR_UNSUPPORTED

@@ -32,12 +32,15 @@ def test_tiny_workload_full_tensor(cuda_ok):
 
 
 # Odd shapes: single rows/keys, tile and unit boundaries (128, 256), ragged tails,
-# d = 64/128, MHA/GQA/MQA, causal on and off, bf16 and fp32 outputs.
+# d = 64/128/256, MHA/GQA/MQA, causal on and off, bf16 and fp32 outputs.
 SHAPES = [
     # B, Hq, Hkv, N, d
     (1, 1, 1, 1, 64), (1, 1, 1, 17, 128), (1, 2, 1, 127, 64), (1, 2, 2, 128, 128),
     (2, 2, 2, 129, 64), (1, 4, 2, 255, 128), (1, 2, 2, 256, 64), (1, 2, 1, 257, 128),
     (1, 3, 3, 383, 64), (2, 4, 1, 513, 128), (1, 8, 8, 1000, 64), (1, 4, 4, 1000, 128),
+    # head dim 256: one 128-row Q tile per unit
+    (1, 1, 1, 1, 256), (1, 2, 1, 127, 256), (1, 2, 2, 128, 256), (2, 2, 2, 129, 256),
+    (1, 4, 2, 513, 256), (1, 2, 2, 1000, 256),
 ]
 
 
@@ -49,7 +52,8 @@ def test_odd_shapes_full_tensor(cuda_ok, shape, causal):
     full_compare(inp, causal, 1.0 / np.sqrt(d))
 
 
-@pytest.mark.parametrize("nq,nk,d", [(1, 300, 64), (200, 1, 128), (300, 1000, 128), (700, 129, 64)])
+@pytest.mark.parametrize("nq,nk,d", [(1, 300, 64), (200, 1, 128), (300, 1000, 128), (700, 129, 64),
+                                     (300, 700, 256)])
 def test_non_square_non_causal(cuda_ok, nq, nk, d):
     inp = small_case(1, 2, 2, nq, nk, d, seed=nq * 7 + nk)
     full_compare(inp, False, 1.0 / np.sqrt(d))

@@ -17,7 +17,8 @@ from workloads import random_bf16
 
 pytestmark = pytest.mark.gpu
 
-D_SCALE = {64: 0.125, 128: float(torch.tensor(1 / np.sqrt(128), dtype=torch.float32))}
+D_SCALE = {64: 0.125, 128: float(torch.tensor(1 / np.sqrt(128), dtype=torch.float32)),
+           256: 0.0625}
 
 
 def packed(lengths, H, d, seed):
@@ -70,7 +71,7 @@ def run_varlen_case(lq, lk, Hq, Hkv, d, causal, seed, out_dtype=torch.bfloat16):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_varlen_self_attention(cuda_ok, d, causal):
     lengths = [1, 17, 128, 129, 256, 300, 511, 64, 1000]
     print(run_varlen_case(lengths, lengths, 4, 2, d, causal, seed=100 + d))

@@ -15,7 +15,9 @@ that the page "FlashAttention-3 (DE)" names as the risk of FP8 quantisation, sec
 "Niedrige Praezision (FP8) mit reduziertem Quantisierungsfehler").  None of the pages
 benchmarks on a public dataset, so the values are i.i.d. standard normal.
 
-Two more workloads feed the incoherent processing of that section (``rotate=True``):
+Two workloads with head dimension 256 (FA2's largest, page "Flash Attention", section on
+the versions) keep the long workload's FLOPs with 16 heads.  Two more workloads feed the
+incoherent processing of that section (``rotate=True``):
 bf16 Q/K/V with the fp8 case's outliers, or with a few outlier channels shared by Q and
 K, that the library quantises itself after a random-sign Hadamard rotation of Q and K.
 Their sign vector is drawn here, after the values, and passed to the library as input.
@@ -107,6 +109,8 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
              1.0, 10.0, outlier_kind="channel", outlier_channels=4, rotate=True),
     Workload("varlen_causal", 16, 32, 32, 8192, 128, True, "bf16", "bf16", 1008, kind="varlen",
              min_len=256),
+    Workload("long_d256", 1, 16, 16, 16384, 256, False, "bf16", "bf16", 1009),
+    Workload("long_d256_causal", 1, 16, 16, 16384, 256, True, "bf16", "bf16", 1009),
     Workload("long_bwd", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003, kind="bwd"),
     Workload("long_causal_bwd", 1, 32, 32, 16384, 128, True, "bf16", "bf16", 1003, kind="bwd"),
     Workload("gqa_causal_bwd", 4, 32, 8, 8192, 128, True, "bf16", "bf16", 1004, kind="bwd"),
