@@ -9,7 +9,8 @@ keys, takes its maximum ``m``, forms ``p_j = exp(s_j - m)``, ``l = sum_j p_j`` a
 returns ``O = sum_j p_j v_j / l`` and ``LSE = m + ln l``.  That is the attention formula
 ``softmax(Q K^T / sqrt(d_k)) V`` of the page "FlashAttention (DE)", section
 "Problematik der Standard-Attention", which the pages say FlashAttention reproduces
-exactly.  ``bwd_oracle.c`` holds the gradients of that formula (dQ, dK, dV for an upstream dO), and
+exactly.  ``dropout_oracle.c`` holds attention with dropout on the weights (Philox4x64 bytes),
+``bwd_oracle.c`` the gradients of that formula (dQ, dK, dV for an upstream dO), and
 ``quant_oracle.c`` the per-head e4m3 quantisation with the random-sign
 Hadamard rotation of the page "FlashAttention-3 (DE)", section "Niedrige Praezision
 (FP8) mit reduziertem Quantisierungsfehler".  This module only marshals arrays into that
@@ -53,6 +54,17 @@ def _bind(lib):
         ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
         ctypes.c_int64, ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_void_p, ctypes.c_int]
+    lib.oracle_philox4x64.restype = None
+    lib.oracle_philox4x64.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    lib.oracle_dropout_byte.restype = ctypes.c_uint8
+    lib.oracle_dropout_byte.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_int64]
+    lib.oracle_attention_dropout_rows.restype = ctypes.c_int
+    lib.oracle_attention_dropout_rows.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+        ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64,
+        ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.oracle_quantize_e4m3.restype = ctypes.c_int
     lib.oracle_quantize_e4m3.argtypes = [
         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
@@ -177,6 +189,47 @@ def attention_bwd(q, k, v, dout, scale, causal=False, nthreads=0, _library=None)
     if rc != 0:
         raise ValueError("oracle_attention_bwd failed with code %d" % rc)
     return dq, dk, dv
+
+
+def philox4x64(counter, key, _library=None):
+    """Philox4x64-10 block for a 4-word counter and a 2-word key (uint64 each)."""
+    c = np.ascontiguousarray(np.asarray(counter, dtype=np.uint64).reshape(4))
+    k = np.ascontiguousarray(np.asarray(key, dtype=np.uint64).reshape(2))
+    out = np.empty(4, dtype=np.uint64)
+    (_library or _load()).oracle_philox4x64(c.ctypes.data, k.ctypes.data, out.ctypes.data)
+    return out
+
+
+def dropout_byte(seed, offset, bh, i, j, _library=None) -> int:
+    return int((_library or _load()).oracle_dropout_byte(int(seed), int(offset), int(bh),
+                                                        int(i), int(j)))
+
+
+def attention_dropout_rows(q, k, v, scale, causal, threshold, seed, offset, rows=None,
+                           nthreads=0, _library=None):
+    """Attention with dropout on the weights (keep key j iff its Philox byte >= threshold,
+    kept weights scaled by 1 / (1 - threshold/256)) for selected query rows.  q: [B, Hq,
+    Nq, d]; k, v: [B, Hkv, Nk, d]; float64 or bf16 bits.  Returns (o [nrows, d], lse)."""
+    qa, ka, va = (np.ascontiguousarray(_as_numpy(t)) for t in (q, k, v))
+    et = _elem_type(qa)
+    if et == E4M3 or _elem_type(ka) != et or _elem_type(va) != et:
+        raise TypeError("q, k and v must all be float64 or all bf16")
+    B, Hq, Nq, d = qa.shape
+    _, Hkv, Nk, _ = ka.shape
+    if rows is None:
+        nrows, rows_ptr = B * Hq * Nq, None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        nrows, rows_ptr = rows_arr.size, rows_arr.ctypes.data
+    o = np.empty((nrows, d), dtype=np.float64)
+    lse = np.empty((nrows,), dtype=np.float64)
+    rc = (_library or _load()).oracle_attention_dropout_rows(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, int(et == BF16), B, Hq, Hkv, Nq, Nk,
+        d, float(scale), int(bool(causal)), int(threshold), int(seed), int(offset), rows_ptr,
+        nrows, o.ctypes.data, lse.ctypes.data, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_attention_dropout_rows failed with code %d" % rc)
+    return o, lse
 
 
 def hadamard(d: int, _library=None) -> np.ndarray:

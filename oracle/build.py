@@ -1,8 +1,8 @@
 """Build the fp64 CPU oracle (test infrastructure) as a shared library.
 
 Compiles ``attn_oracle.c`` (attention), ``quant_oracle.c`` (fp8 quantisation with
-incoherent processing) and ``bwd_oracle.c`` (gradients) with gcc and OpenMP into
-``oracle/liboracle.so``.  Only the
+incoherent processing), ``bwd_oracle.c`` (gradients) and ``dropout_oracle.c`` (dropout and
+its Philox generator) with gcc and OpenMP into ``oracle/liboracle.so``.  Only the
 tests, the smoke check and the CPU-baseline leg of ``bench.py`` load that library.
 """
 import os
@@ -12,7 +12,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "attn_oracle.c")
 QUANT_SRC = os.path.join(HERE, "quant_oracle.c")
 BWD_SRC = os.path.join(HERE, "bwd_oracle.c")
-SOURCES = (SRC, QUANT_SRC, BWD_SRC)
+DROPOUT_SRC = os.path.join(HERE, "dropout_oracle.c")
+SOURCES = (SRC, QUANT_SRC, BWD_SRC, DROPOUT_SRC)
 LIB = os.path.join(HERE, "liboracle.so")
 
 

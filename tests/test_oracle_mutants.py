@@ -156,9 +156,34 @@ def pin_bwd_autograd(lib):
             assert np.abs(g - r.numpy()).max() < 1e-12
 
 
+def _np_block(counter, key):
+    value = (sum(int(w) << (64 * n) for n, w in enumerate(counter)) - 1) % 2**256
+    start = np.array([(value >> (64 * n)) & (2**64 - 1) for n in range(4)], dtype=np.uint64)
+    return np.random.Philox(counter=start, key=np.array(key, dtype=np.uint64)).random_raw(4)
+
+
+def pin_philox_numpy(lib):
+    for ctr, key in (([6, 7, 9, 11], [3, 5]), ([0, 1, 2, 0], [2**63, 1])):
+        assert np.array_equal(oracle.philox4x64(ctr, key, _library=lib), _np_block(ctr, key))
+
+
+def pin_dropout_bruteforce(lib):
+    q, k, v = rnd((1, 2, 5, 3), 40), rnd((1, 2, 40, 3), 41), rnd((1, 2, 40, 3), 42)
+    thr, seed, off = 90, 7, 1
+    o, _ = oracle.attention_dropout_rows(q, k, v, 0.5, False, thr, seed, off, _library=lib)
+    o = o.reshape(2, 5, 3)
+    for h in range(2):
+        for i in range(5):
+            e = np.exp(0.5 * (k[0, h] @ q[0, h, i]))
+            keep = np.array([((int(_np_block([j // 32, i, h, 0], [seed, off])[(j % 32) // 8])
+                               >> (8 * (j % 8))) & 0xFF) >= thr for j in range(40)])
+            ref = (e * keep) @ v[0, h] / e.sum() / (1 - thr / 256)
+            assert np.abs(o[h, i] - ref).max() < 1e-12
+
+
 PINS = [pin_sdpa, pin_bruteforce_lse, pin_bottom_right, pin_gqa, pin_decoders, pin_e4m3_descales,
         pin_hadamard_scipy, pin_encoder_torch, pin_rotation_basis_and_norm,
-        pin_quantise_rounding_bound, pin_bwd_autograd]
+        pin_quantise_rounding_bound, pin_bwd_autograd, pin_philox_numpy, pin_dropout_bruteforce]
 
 MUTANTS = {
     "scale_dropped": ("srow[j] = scale * dot;", "srow[j] = dot;"),
@@ -212,6 +237,18 @@ MUTANTS = {
                        "dp[j] = dot_rows(dout, qoff, k, kvoff + j * d, elem_type, d);"),
     "bwd_dk_reads_dout": ("dkr[t] += scale * ds * ld(q, elem_type, qoff + t);",
                           "dkr[t] += scale * ds * ld(dout, elem_type, qoff + t);"),
+    # dropout oracle
+    "philox_key_dropped": ("c0 = hi1 ^ c1 ^ k0;", "c0 = hi1 ^ c1;"),
+    "philox_weyl_wrong": ("k1 += W1;", "k1 += W0;"),
+    "dropout_byte_order": ("return (uint8_t)(o[t >> 3] >> (8 * (t & 7)));",
+                           "return (uint8_t)(o[t >> 3] >> (8 * (7 - (t & 7))));"),
+    "dropout_counter_swapped": (
+        "const uint64_t ctr[4] = {(uint64_t)(j >> 5), (uint64_t)i, (uint64_t)bh, 0};",
+        "const uint64_t ctr[4] = {(uint64_t)(j >> 5), (uint64_t)bh, (uint64_t)i, 0};"),
+    "dropout_keep_strict": ("if (oracle_dropout_byte(seed, offset, bh, i, j) >= thr)",
+                            "if (oracle_dropout_byte(seed, offset, bh, i, j) > thr)"),
+    "dropout_scale_dropped": ("o_out[r * d + t] = acc[t] * keep_scale / row_sum;",
+                              "o_out[r * d + t] = acc[t] / row_sum;"),
 }
 
 
