@@ -263,8 +263,12 @@ def oracle_timed_sample(w, inp, n_rows, seed=0):
     total_rows = w.B * w.Hq * w.N
     rows = rng.integers(0, total_rows, size=n_rows)
     t0 = time.perf_counter()
-    oracle.attention_rows(inp.q, inp.k, inp.v, w.scale, w.causal, rows=rows,
-                          **_oracle_kwargs(inp))
+    if w.dropout:
+        oracle.attention_dropout_rows(inp.q, inp.k, inp.v, w.scale, w.causal,
+                                      min(255, round(256 * w.dropout)), w.seed, 0, rows=rows)
+    else:
+        oracle.attention_rows(inp.q, inp.k, inp.v, w.scale, w.causal, rows=rows,
+                              **_oracle_kwargs(inp))
     dt = time.perf_counter() - t0
     desc = ("%d random query rows (of %d) of workload %s, each over its full admissible key "
             "range, fp64" % (n_rows, total_rows, w.name))
@@ -413,6 +417,11 @@ def run_ours(args):
                               out_dtype=out_dtype, out=o, lse=lse)
         elif fp8:
             fa.forward_fp8(q, k, v, dq, dk, dv, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        elif w.dropout:
+            # a new mask every step, as in training (the offset is the step number)
+            fa.forward_dropout(q, k, v, w.dropout, seed=w.seed, offset=0 if i is None else i,
+                               causal=w.causal, scale=w.scale, out_dtype=out_dtype, out=o,
+                               lse=lse)
         else:
             fa.forward(q, k, v, causal=w.causal, scale=w.scale, out_dtype=out_dtype, out=o,
                        lse=lse)

@@ -1,9 +1,9 @@
 """B200-native fused exact attention forward: Python binding of ``libfa_b200.so``.
 
 The C ABI (``include/fa_b200.h``) is the product; this module only marshals arguments
-into it.  The functions ``fa_fwd``, ``fa_fwd_varlen``, ``fa_fwd_fp8``, ``fa_bwd``, ``fa_quantize_e4m3``,
+into it.  The functions ``fa_fwd``, ``fa_fwd_dropout``, ``fa_fwd_varlen``, ``fa_fwd_fp8``, ``fa_bwd``, ``fa_quantize_e4m3``,
 ``fa_check_device_error`` and ``fa_status_string`` have the names and argument order of
-the C entry points and take raw device pointers.  ``forward`` / ``forward_varlen`` /
+the C entry points and take raw device pointers.  ``forward`` / ``forward_dropout`` / ``forward_varlen`` /
 ``forward_fp8`` / ``backward`` / ``quantize_e4m3`` are conveniences that take CUDA tensors (PyTorch provides device
 memory and streams only), allocate the outputs and raise on a non-zero status.  Every step of the attention runs in the CUDA kernels; there
 is no CPU or library fallback -- if the shared library is missing, importing a function
@@ -20,7 +20,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
-C_SYMBOLS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
+C_SYMBOLS = ("fa_fwd", "fa_fwd_dropout", "fa_fwd_varlen", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
              "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_string",
              "fa_version")
 
@@ -44,6 +44,9 @@ def lib() -> ctypes.CDLL:
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.fa_fwd.restype = i
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+        L.fa_fwd_dropout.restype = i
+        L.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, f,
+                                     ctypes.c_uint64, ctypes.c_uint64, i, vp]
         L.fa_fwd_varlen.restype = i
         L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, vp]
         L.fa_fwd_fp8.restype = i
@@ -72,6 +75,13 @@ def lib() -> ctypes.CDLL:
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
     """Raw ``fa_fwd``: pointers are ints (device addresses), stream an int handle."""
     return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream)
+
+
+def fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dropout_p, seed,
+                   offset, dtype, stream) -> int:
+    """Raw ``fa_fwd_dropout``."""
+    return lib().fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                float(dropout_p), int(seed), int(offset), dtype, stream)
 
 
 def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, total_q, total_k,
@@ -173,6 +183,29 @@ def forward(q, k, v, causal=False, scale=None, out_dtype=None, out=None, lse=Non
                 B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), dtype, _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def forward_dropout(q, k, v, dropout_p, seed, offset=0, causal=False, scale=None,
+                    out_dtype=None, out=None, lse=None, stream=None):
+    """``forward`` with dropout on the attention weights (probability rounded to a multiple
+    of 1/256; the mask is a function of (seed, offset, batch, head, query, key))."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _check_inputs(q, k, v)
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise ValueError("forward_dropout() takes bf16 q, k, v")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    dtype = FA_BF16_OUT_F32 if out_dtype == torch.float32 else FA_BF16
+    st = fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                        lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
+                        dropout_p, seed, offset, dtype, _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_dropout")
     return out, lse
 
 

@@ -119,11 +119,11 @@ bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN = false>
+template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN = false, bool DROPOUT = false>
 fa_status launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                  const fa::FwdParams &p, int grid, int dev, cudaStream_t stream) {
   using C = fa::TileCfg<D, FP8>;
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL, OUT_F32, FP8, VARLEN>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, OUT_F32, FP8, VARLEN, DROPOUT>;
   static std::once_flag attr_once[kMaxDevices];
   static fa_status attr_st[kMaxDevices];
   std::call_once(attr_once[dev], [&] {
@@ -179,10 +179,19 @@ fa_status check_args(const void *q, const void *k, const void *v, const void *o,
   return FA_OK;
 }
 
+// Dropout threshold for probability p (the nearest multiple of 1/256), -1 if p is not in
+// [0, 1).
+int dropout_threshold(float p) {
+  if (!(p >= 0.f) || !(p < 1.f)) return -1;
+  const int thr = static_cast<int>(std::lrint(static_cast<double>(p) * 256.0));
+  return thr > 255 ? 255 : thr;
+}
+
 fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                      int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                      bool out_f32, bool fp8, const float *dq, const float *dk, const float *dv,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, int drop_thr = 0, uint64_t seed = 0,
+                     uint64_t offset = 0) {
   fa_status st = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, fp8, dq, dk, dv);
   if (st != FA_OK) return st;
 
@@ -221,6 +230,10 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
   p.descale_v = dv;
   p.cu_q = nullptr;
   p.cu_k = nullptr;
+  p.seed = seed;
+  p.offset = offset;
+  p.drop_thr4 = static_cast<uint32_t>(drop_thr) * 0x01010101u;
+  p.keep_scale = static_cast<float>(256.0 / (256.0 - drop_thr));
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -236,6 +249,21 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
   if (fp8) {
     if (causal) return launch<128, true, false, true>(tq, tk, tv, p, grid, dev, stream);
     return launch<128, false, false, true>(tq, tk, tv, p, grid, dev, stream);
+  }
+  if (drop_thr > 0) {
+#define FA_DROP(DD)                                                                           \
+  if (d == DD) {                                                                              \
+    if (causal)                                                                               \
+      return out_f32 ? launch<DD, true, true, false, false, true>(tq, tk, tv, p, grid, dev, stream) \
+                     : launch<DD, true, false, false, false, true>(tq, tk, tv, p, grid, dev, stream); \
+    return out_f32 ? launch<DD, false, true, false, false, true>(tq, tk, tv, p, grid, dev, stream) \
+                   : launch<DD, false, false, false, false, true>(tq, tk, tv, p, grid, dev, stream); \
+  }
+    FA_DROP(64)
+    FA_DROP(128)
+    FA_DROP(256)
+#undef FA_DROP
+    return FA_ERR_UNSUPPORTED;
   }
   if (d == 64) {
     if (causal)
@@ -324,6 +352,9 @@ fa_status fwd_varlen_common(const void *q, const void *k, const void *v, void *o
   p.descale_q = p.descale_k = p.descale_v = nullptr;
   p.cu_q = cu_q;
   p.cu_k = cu_k;
+  p.seed = p.offset = 0;
+  p.drop_thr4 = 0;
+  p.keep_scale = 1.f;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -705,6 +736,18 @@ fa_status fa_quantize_e4m3(const void *x, const int8_t *signs, void *x8, float *
                            int H, int N, int d, fa_stream_t stream) {
   return quantize_common(x, signs, x8, descale, B, H, N, d,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         float dropout_p, uint64_t seed, uint64_t offset, fa_dtype dtype,
+                         fa_stream_t stream) {
+  if (dtype != FA_BF16 && dtype != FA_BF16_OUT_F32) return FA_ERR_INVALID_ARG;
+  const int thr = dropout_threshold(dropout_p);
+  if (thr < 0) return FA_ERR_INVALID_ARG;
+  return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                    dtype == FA_BF16_OUT_F32, false, nullptr, nullptr, nullptr,
+                    reinterpret_cast<cudaStream_t>(stream), thr, seed, offset);
 }
 
 fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,

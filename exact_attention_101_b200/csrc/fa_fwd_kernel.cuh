@@ -162,6 +162,13 @@ struct FwdParams {
   int num_qb;       // ceil(Nq / unit rows); varlen: ceil(longest query sequence / unit rows)
   int num_units;    // B * Hq * num_qb
   float scale_log2; // softmax scale * log2(e)
+  // dropout (kernels instantiated with DROPOUT only): key j of query row i of (batch,
+  // head) bh is kept iff byte j mod 32 of the Philox4x64-10 block for counter
+  // (j / 32, i, bh, 0) and key (seed, offset) is >= drop_thr; kept weights are scaled by
+  // keep_scale = 1 / (1 - drop_thr / 256)
+  uint64_t seed, offset;
+  uint32_t drop_thr4;  // drop_thr in every byte
+  float keep_scale;
 };
 
 struct Unit {
@@ -483,10 +490,21 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, fl
 // numerators as rounded for the tensor core (bf16 only) to lr and of the unrounded
 // numerators to le.  NPOLY of every 8 column pairs use the polynomial exponential.
 // Numerators are packed and stored to TMEM 32 columns at a time (64 for e4m3).
-template <bool FP8, int NPOLY>
+// Keep masks of a 32-key block: bytes >= thr become 0xff (two keys per 16-bit mask half
+// below), from the four 64-bit Philox words.
+__device__ __forceinline__ void keep_bytes(const uint64_t (&r)[4], uint32_t thr4,
+                                           uint32_t (&kb)[8]) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    kb[2 * w] = __vcmpgeu4(static_cast<uint32_t>(r[w]), thr4);
+    kb[2 * w + 1] = __vcmpgeu4(static_cast<uint32_t>(r[w] >> 32), thr4);
+  }
+}
+
+template <bool FP8, int NPOLY, bool DROPOUT = false>
 __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], float sl2,
                                                    float neg_m, uint32_t t_p, float &lr,
-                                                   float &le) {
+                                                   float &le, const uint32_t (*keep)[8] = nullptr) {
   const uint64_t scale2 = ptx::f2_pack(sl2, sl2);
   const uint64_t bias2 = ptx::f2_pack(neg_m, neg_m);
   uint64_t acc_r[2] = {0ull, 0ull};  // packed (0.f, 0.f)
@@ -522,6 +540,11 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], 
         acc_r[(e / 2) & 1] = ptx::f2_add(
             acc_r[(e / 2) & 1],
             ptx::f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u)));
+        if (DROPOUT) {
+          // dropped keys leave the product (not the sum): key byte masks to 16-bit halves
+          const uint32_t kb = keep[q][e / 4];
+          pk[e / 2] &= ptx::prmt(kb, 0u, (e & 2) ? 0x3322u : 0x1100u);
+        }
       }
     } else {
 #pragma unroll
@@ -543,7 +566,7 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], 
 // (TMEM lane).  Every 64-key score tile is loaded whole into registers, masked if it
 // crosses the diagonal or the end of the keys, turned into numerators in place, and the
 // row statistics are carried from tile to tile.
-template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN>
+template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN, bool DROPOUT>
 __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
                              volatile uint32_t *abort_flag) {
   using C = TileCfg<D, FP8>;
@@ -645,7 +668,18 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       // polynomial and the rest to the MUFU unit.
       float lr = 0.f, le = 0.f;
       const uint32_t t_p = t_s + C::P_OFF;
-      if (EXP2_POLY_PAIRS == 0)   // one copy of the unrolled loop: smaller code, faster
+      if (DROPOUT) {
+        // two Philox blocks: keys kv0 .. kv0+31 and kv0+32 .. kv0+63 of this row
+        uint32_t keep[2][8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint64_t r[4];
+          ptx::philox4x64(static_cast<uint64_t>(kv0 / 32 + h), static_cast<uint64_t>(row),
+                          static_cast<uint64_t>(w.bh), 0ull, p.seed, p.offset, r);
+          keep_bytes(r, p.drop_thr4, keep[h]);
+        }
+        softmax_numerators<FP8, 0, true>(sr, sl2, neg_m, t_p, lr, le, keep);
+      } else if (EXP2_POLY_PAIRS == 0)   // one copy of the unrolled loop: smaller code, faster
         softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, lr, le);
       else if (need_mask)
         softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, lr, le);
@@ -670,6 +704,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       ptx::tc_fence_after();
       // a row without admissible keys (causal, more queries than keys) has l = 0: O = 0
       float inv = l > 0.f ? 1.f / l : 0.f;
+      if (DROPOUT) inv *= p.keep_scale;
       if (FP8) inv *= p.descale_v[w.bhk];
       // packed varlen output: O [tokens, Hq, d], LSE [Hq, tokens]; the token check keeps
       // the stores inside the tensors whatever the offsets say
@@ -724,7 +759,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
 
 // ---------------------------------------------------------------------------- kernel
 
-template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN>
+template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN, bool DROPOUT = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -777,7 +812,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::setmaxnreg_dec<OTHER_REGS>();
 
   if (warp < 4 * C::NT) {
-    softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN>(p, tmem, bar, abort_flag);
+    softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN, DROPOUT>(p, tmem, bar, abort_flag);
   } else if (warp == MMA_WARP || (C::NT == 2 && warp == MMA_WARP + 2)) {
     mma_role<D, CAUSAL, FP8, VARLEN>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, abort_flag);
     __syncwarp();

@@ -53,7 +53,7 @@ typedef enum fa_status {
     FA_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, bad size, bad scale, buffer
                                 too small for the given shape or not device memory */
     FA_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement: head
-                                dim not 64/128, GPU not sm_100, and the limits stated
+                                dim not 64/128/256, GPU not sm_100, and the limits stated
                                 at each entry point */
     FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, attribute) */
     FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (see below) */
@@ -72,7 +72,7 @@ typedef enum fa_dtype {
  *   o        device pointer, bf16 (FA_BF16) or fp32 (FA_BF16_OUT_F32), [B,Hq,Nq,d]
  *   lse      device pointer, fp32 [B,Hq,Nq]: LSE = ln sum_j exp(scale * q_i . k_j)
  *   B, Hq, Hkv, Nq, Nk   >= 1; Hq % Hkv == 0
- *   d        head dimension, 64 or 128
+ *   d        head dimension, 64, 128 or 256
  *   scale    softmax scale (> 0, finite); callers normally pass 1/sqrt(d)
  *   causal   0 or 1
  *   dtype    FA_BF16 or FA_BF16_OUT_F32 (FA_E4M3 is rejected: use fa_fwd_fp8)
@@ -84,6 +84,27 @@ typedef enum fa_dtype {
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                  int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                  fa_dtype dtype, fa_stream_t stream);
+
+/*
+ * fa_fwd with dropout on the attention weights, fused into the kernel: the page "Flash
+ * Attention" (section "Zentrale technische Innovationen", the fusion bullet) lists dropout
+ * among the operations fused with the softmax.  With P the attention weights of a row,
+ *
+ *     O_i = sum_j P_ij keep_ij v_j / (1 - thr/256),    thr = round(256 * dropout_p)
+ *
+ * and LSE as without dropout.  keep_ij = 1 iff byte (j mod 32), little-endian in the four
+ * 64-bit words, of the Philox4x64-10 block (Salmon et al., SC'11) for counter
+ * (j / 32, i, b*Hq + hq, 0) and key (seed, offset) is >= thr.  The dropout probability is
+ * thus thr/256; the same (seed, offset) gives the same mask.
+ *
+ *   dropout_p   in [0, 1) (else FA_ERR_INVALID_ARG); rounded to a multiple of 1/256
+ *   dtype       FA_BF16 or FA_BF16_OUT_F32;  d 64, 128 or 256
+ *   other arguments as for fa_fwd
+ */
+fa_status fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                         int causal, float dropout_p, uint64_t seed, uint64_t offset,
+                         fa_dtype dtype, fa_stream_t stream);
 
 /*
  * Fused attention forward over a batch of sequences of different lengths, packed without
@@ -100,7 +121,7 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *ls
  *               cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1.  Entries must be non-decreasing,
  *               start at 0 and end at total_q / total_k.
  *   max_seqlen_q   at least the longest query sequence (work is planned for it)
- *   d           64 or 128;  dtype FA_BF16 or FA_BF16_OUT_F32
+ *   d           64, 128 or 256;  dtype FA_BF16 or FA_BF16_OUT_F32
  *
  * Each sequence is attended on its own; causal masking is per sequence, bottom-right
  * aligned as above.  The offsets are read on the device: wrong offsets give wrong results

@@ -179,3 +179,16 @@ def test_varlen_invalid_arguments(kw):
 @pytest.mark.parametrize("d", [32, 96, 512])
 def test_varlen_unsupported_head_dims(d):
     assert varlen_call(d=d) == fa.FA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("p", [-0.1, 1.0, 1.5, float("nan"), float("inf")])
+def test_dropout_probability_range(p):
+    assert fa.fa_fwd_dropout(A, A, A, A, A, 1, 2, 2, 128, 128, 128, 0.088, 0, p, 1, 0,
+                             fa.FA_BF16, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_dropout_dtypes():
+    assert fa.fa_fwd_dropout(A, A, A, A, A, 1, 2, 2, 128, 128, 128, 0.088, 0, 0.1, 1, 0,
+                             fa.FA_E4M3, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_dropout(A, A, A, A, A, 1, 2, 2, 128, 128, 96, 0.088, 0, 0.1, 1, 0,
+                             fa.FA_BF16, None) == fa.FA_ERR_UNSUPPORTED

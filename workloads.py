@@ -59,6 +59,7 @@ class Workload:
     #                               "varlen": B packed sequences of lengths drawn in
     #                               [min_len, N] (token-major [tokens, H, d] tensors)
     min_len: int = 0
+    dropout: float = 0.0          # dropout probability on the attention weights (fwd)
 
     @property
     def scale(self) -> float:
@@ -87,6 +88,8 @@ class Workload:
             out["quantise"] = "e4m3 per head on the GPU, Q and K after random-sign Hadamard"
         if self.kind == "bwd":
             out["pass"] = "backward (dQ, dK, dV from Q, K, V, O, LSE, dO)"
+        if self.dropout:
+            out["dropout"] = self.dropout
         if self.kind == "varlen":
             lens = varlen_lengths(self)
             out.update({"Nq": None, "Nk": None, "sequences": self.B, "total_tokens": sum(lens),
@@ -109,6 +112,7 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
              1.0, 10.0, outlier_kind="channel", outlier_channels=4, rotate=True),
     Workload("varlen_causal", 16, 32, 32, 8192, 128, True, "bf16", "bf16", 1008, kind="varlen",
              min_len=256),
+    Workload("long_dropout", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003, dropout=0.1),
     Workload("long_d256", 1, 16, 16, 16384, 256, False, "bf16", "bf16", 1009),
     Workload("long_d256_causal", 1, 16, 16, 16384, 256, True, "bf16", "bf16", 1009),
     Workload("long_bwd", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003, kind="bwd"),
