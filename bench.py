@@ -583,6 +583,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "ms_median": per_step[len(per_step) // 2], "ms_best": per_step[0],
+        "ms_worst": per_step[-1],
         "first_call_ms": first_call_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",

@@ -523,21 +523,22 @@ bool encode_tmap_dq(CUtensorMap *m, void *base, uint64_t d, uint64_t rows, uint6
   return r == CUDA_SUCCESS;
 }
 
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 fa_status bwd_launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      const CUtensorMap &tdo, const CUtensorMap &tdq,
                      const fa::bwd::BwdParams &p, int grid, int dev, cudaStream_t stream) {
-  auto kern = fa::bwd::fa_bwd_kernel<CAUSAL>;
+  auto kern = fa::bwd::fa_bwd_kernel<D, CAUSAL>;
+  constexpr int smem_bytes = fa::bwd::BCfg<D>::SMEM_BYTES;
   static std::once_flag attr_once[kMaxDevices];
   static fa_status attr_st[kMaxDevices];
   std::call_once(attr_once[dev], [&] {
     attr_st[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        fa::bwd::SMEM_BYTES) == cudaSuccess
+                                        smem_bytes) == cudaSuccess
                        ? FA_OK
                        : FA_ERR_CUDA;
   });
   if (attr_st[dev] != FA_OK) return attr_st[dev];
-  kern<<<grid, fa::bwd::NUM_THREADS, fa::bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+  kern<<<grid, fa::bwd::NUM_THREADS, smem_bytes, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -560,7 +561,7 @@ fa_status check_bwd_args(const void *q, const void *k, const void *v, const void
   if (bh > INT32_MAX || units > INT32_MAX || Nq > INT32_MAX - 2 * fa::bwd::BM ||
       Nk > INT32_MAX - 2 * fa::bwd::BN)
     return FA_ERR_INVALID_ARG;
-  if (d != fa::bwd::D) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (causal && Nq != Nk) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
@@ -574,8 +575,37 @@ uint64_t bwd_scratch_bytes(int B, int Hq, int Nq, int d, uint64_t *acc_bytes, ui
   return *acc_bytes + 2 * *vec_bytes;
 }
 
-// fixed_ws == nullptr: scratch is allocated and freed on `stream` (cudaMallocAsync /
-// cudaFreeAsync); otherwise fixed_ws (large enough, checked by the caller) is used.
+// Stream-ordered memory pool of the backward's scratch, one per device, created on first
+// use and kept for the life of the process.  Freed scratch stays in the pool up to
+// kScratchKeepBytes across synchronisations, so repeated calls of similar size take it
+// back without asking the driver for memory again (the device's default pool hands
+// everything back at each synchronisation, and the next call then waits on the driver).
+constexpr uint64_t kScratchKeepBytes = 4ull << 30;
+
+fa_status scratch_pool(int dev, cudaMemPool_t *out) {
+  static std::once_flag once[kMaxDevices];
+  static cudaMemPool_t pool[kMaxDevices];
+  static fa_status st[kMaxDevices];
+  std::call_once(once[dev], [&] {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    uint64_t keep = kScratchKeepBytes;
+    st[dev] = cudaMemPoolCreate(&pool[dev], &props) == cudaSuccess &&
+                      cudaMemPoolSetAttribute(pool[dev], cudaMemPoolAttrReleaseThreshold,
+                                              &keep) == cudaSuccess
+                  ? FA_OK
+                  : FA_ERR_CUDA;
+    if (st[dev] != FA_OK) cudaGetLastError();
+  });
+  *out = pool[dev];
+  return st[dev];
+}
+
+// fixed_ws == nullptr: scratch is taken from and returned to the library's pool on
+// `stream` (stream-ordered); otherwise fixed_ws (large enough, checked by the caller) is
+// used.
 fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
                      int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
@@ -629,9 +659,13 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
   uint64_t acc_bytes = 0, vec_bytes = 0;
   const uint64_t ws_bytes = bwd_scratch_bytes(B, Hq, Nq, d, &acc_bytes, &vec_bytes);
   void *ws = fixed_ws;
-  if (ws == nullptr && cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess) {
-    cudaGetLastError();
-    return FA_ERR_CUDA;
+  if (ws == nullptr) {
+    cudaMemPool_t pool;
+    if (scratch_pool(dev, &pool) != FA_OK) return FA_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(&ws, ws_bytes, pool, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
   }
   float *dq_acc = static_cast<float *>(ws);
   p.l2 = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + acc_bytes);
@@ -643,16 +677,21 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
     st = FA_ERR_CUDA;
   if (st == FA_OK) {
     const unsigned blocks = static_cast<unsigned>((rows_padded + 7) / 8);
-    fa::bwd::fa_bwd_prep_kernel<<<blocks, 256, 0, stream>>>(
-        static_cast<const uint16_t *>(o), static_cast<const uint16_t *>(dout), lse,
-        const_cast<float *>(p.l2), const_cast<float *>(p.dd), static_cast<long long>(rows_padded),
-        Nq, p.Npad);
+    auto prep = d == 64 ? fa::bwd::fa_bwd_prep_kernel<64> : fa::bwd::fa_bwd_prep_kernel<128>;
+    prep<<<blocks, 256, 0, stream>>>(static_cast<const uint16_t *>(o),
+                                     static_cast<const uint16_t *>(dout), lse,
+                                     const_cast<float *>(p.l2), const_cast<float *>(p.dd),
+                                     static_cast<long long>(rows_padded), Nq, p.Npad);
     if (cudaGetLastError() != cudaSuccess) st = FA_ERR_CUDA;
   }
   if (st == FA_OK) {
     const int grid = p.num_units < info.sms ? p.num_units : info.sms;
-    st = causal ? bwd_launch<true>(tq, tk, tv, tdo, tdq, p, grid, dev, stream)
-                : bwd_launch<false>(tq, tk, tv, tdo, tdq, p, grid, dev, stream);
+    if (d == 64)
+      st = causal ? bwd_launch<64, true>(tq, tk, tv, tdo, tdq, p, grid, dev, stream)
+                  : bwd_launch<64, false>(tq, tk, tv, tdo, tdq, p, grid, dev, stream);
+    else
+      st = causal ? bwd_launch<128, true>(tq, tk, tv, tdo, tdq, p, grid, dev, stream)
+                  : bwd_launch<128, false>(tq, tk, tv, tdo, tdq, p, grid, dev, stream);
   }
   if (st == FA_OK) {
     const long long n4 = static_cast<long long>(q_bytes / 2 / 4);

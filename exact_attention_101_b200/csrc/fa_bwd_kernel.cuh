@@ -18,11 +18,14 @@
 // unit, and walks every query head of the group and every block of BM = 64 queries (from
 // the diagonal on under the causal mask).  Per step five tcgen05 MMAs:
 //
-//   S^T  = K_j Q_i^T      M=128 keys, N=64 queries, K=128 (SS, both K-major)
+//   S^T  = K_j Q_i^T      M=128 keys, N=64 queries, K=D (SS, both K-major)
 //   dP^T = V_j dO_i^T     same shape
-//   dQ^T = K_j^T dS^T     M=128 head dims, N=64 queries, K=128 keys (SS, both MN-major)
-//   dV  += P^T dO_i       M=128 keys, N=128, K=64 queries (A = P^T from tensor memory)
+//   dQ^T = K_j^T dS^T     M=128 head dims, N=64 queries, K=128 keys (SS, both MN-major;
+//                         at D = 64 the upper 64 rows of K_j^T are a tile of zeros)
+//   dV  += P^T dO_i       M=128 keys, N=D, K=64 queries (A = P^T from tensor memory)
 //   dK  += dS^T Q_i       same shape (A = dS^T from tensor memory)
+//
+// D (the head dimension) is 64 or 128.
 //
 // dQ^T goes from tensor memory through a shared-memory staging tile to a bulk tensor
 // reduce-add (TMA) into a zeroed fp32 accumulator in global memory (each query block
@@ -31,7 +34,7 @@
 //
 // Tensor memory (512 columns): S^T of step buffer b at b*128 (64 columns; after the
 // softmax, P^T and dS^T as packed bf16), dP^T of buffer b at b*128 + 64 (then dQ^T of the
-// same step), dV at 256, dK at 384.  Two step buffers let the softmax of step i+1 run
+// same step), dV at 256, dK at 256 + D.  Two step buffers let the softmax of step i+1 run
 // while the tensor core works on step i.  Q_i, dO_i and the two per-query vectors sit in a
 // ring of QSTAGES shared-memory stages, so their copies run two steps ahead of the MMAs
 // that read them; dS^T has one shared-memory buffer (the softmax of step g writes it once
@@ -40,7 +43,7 @@
 // Warps: 0-3 and 4-7 are the "softmax" warpgroups (thread = key row; warpgroup h takes
 // queries 32h .. 32h+31 of the step, and at the end of a unit writes dV (h=0) or dK
 // (h=1)); 8-11 drain dQ^T (thread = head dimension); 12 allocates tensor memory and issues
-// the MMAs; 13 issues the TMA copies.
+// the MMAs; 13 issues the TMA copies.  At D = 64 only drain warps 8-9 own head dims.
 #pragma once
 
 #include <cstdint>
@@ -53,45 +56,57 @@
 namespace fa {
 namespace bwd {
 
-constexpr int D = 128;
 constexpr int BN = 128;                  // keys per unit (tensor-memory lanes)
 constexpr int BM = 64;                   // queries per step
 constexpr int NUM_THREADS = 448;         // 14 warps
 constexpr int DRAIN_WARP0 = 8;
 constexpr int MMA_WARP = 12;
 constexpr int TMA_WARP = 13;
-constexpr int ROW_BYTES = D * 2;
-constexpr int KV_BOX = BN * 128;         // one 128-byte-wide TMA box of a K or V tile
-constexpr int KV_TILE = 2 * KV_BOX;      // 32 KB
-constexpr int Q_BOX = BM * 128;
-constexpr int Q_TILE = 2 * Q_BOX;        // 16 KB
+constexpr int KV_BOX = BN * 128;         // one 128-byte-wide TMA box of a K or V tile (16 KB)
+constexpr int Q_BOX = BM * 128;          // one box of a Q or dO tile (8 KB)
 constexpr int DS_TILE = BN * BM * 2;     // dS^T [keys][queries] bf16, 128-byte rows: 16 KB
 constexpr int VEC_BYTES = 2 * BM * 4;    // per step: LSE*log2(e) and D for BM queries
-
-// Shared memory map (offsets from a 1024-aligned base).
-constexpr int K_OFF = 0;
-constexpr int V_OFF = K_OFF + KV_TILE;
 constexpr int QSTAGES = 3;               // ring of Q, dO and vector stages
 constexpr int DQ_STAGE = 32 * BM * 4;    // per drain warp: 64 queries x 32 head dims fp32
-constexpr int Q_OFF = V_OFF + KV_TILE;
-constexpr int DO_OFF = Q_OFF + QSTAGES * Q_TILE;
-constexpr int DS_OFF = DO_OFF + QSTAGES * Q_TILE;
-constexpr int DQS_OFF = DS_OFF + DS_TILE;
-constexpr int VEC_OFF = DQS_OFF + 4 * DQ_STAGE;
-constexpr int BAR_OFF = VEC_OFF + QSTAGES * VEC_BYTES;
 constexpr int NUM_BARS = 2 + 2 * QSTAGES + 2 * 4 + 3;
-constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
-constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// Tensor-memory columns.
+// Tensor-memory columns of the step buffers.
 __host__ __device__ constexpr uint32_t s_col(int b) { return b * 128; }
 __host__ __device__ constexpr uint32_t dp_col(int b) { return b * 128 + 64; }
-constexpr uint32_t DV_COL = 256, DK_COL = 384;
 
-constexpr uint32_t IDESC_S = ptx::make_idesc(1, BN, BM, 0);          // S^T, dP^T
-constexpr uint32_t IDESC_ACC = ptx::make_idesc(1, BN, D, 1);         // dV, dK
-constexpr uint32_t IDESC_DQ = ptx::make_idesc_ab(1, D, BM, 1, 1);    // dQ^T
+// Head-dimension-dependent layout (D = 64 or 128).  The dQ^T product always has M = 128
+// head-dimension rows: at D = 64 the second 64 rows of its A operand (K^T) come from a
+// 16 KB tile of zeros, so rows 64..127 of dQ^T are zero and are not reduced.  That costs
+// half a product per step and keeps the tensor-memory lane layout of M = 128.
+template <int D>
+struct BCfg {
+  static_assert(D == 64 || D == 128, "head dims of the backward kernel");
+  static constexpr int NBOX = D * 2 / 128;             // 128-byte boxes per row
+  static constexpr int KV_TILE = NBOX * KV_BOX;
+  static constexpr int Q_TILE = NBOX * Q_BOX;
+  static constexpr int DRAIN_WARPS = D / 32;           // drain warps that own head dims
+  // Shared memory map (offsets from a 1024-aligned base).
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + KV_TILE;
+  static constexpr int Z_OFF = V_OFF + KV_TILE;
+  static constexpr int Z_BYTES = D < 128 ? KV_BOX : 0;
+  static constexpr int Q_OFF = Z_OFF + Z_BYTES;
+  static constexpr int DO_OFF = Q_OFF + QSTAGES * Q_TILE;
+  static constexpr int DS_OFF = DO_OFF + QSTAGES * Q_TILE;
+  static constexpr int DQS_OFF = DS_OFF + DS_TILE;
+  static constexpr int VEC_OFF = DQS_OFF + DRAIN_WARPS * DQ_STAGE;
+  static constexpr int BAR_OFF = VEC_OFF + QSTAGES * VEC_BYTES;
+  static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // Tensor memory: step buffers at 0..255, dV at 256, dK after it.
+  static constexpr uint32_t DV_COL = 256, DK_COL = 256 + D;
+  static constexpr uint32_t IDESC_S = ptx::make_idesc(1, BN, BM, 0);        // S^T, dP^T
+  static constexpr uint32_t IDESC_ACC = ptx::make_idesc(1, BN, D, 1);       // dV, dK
+  static constexpr uint32_t IDESC_DQ = ptx::make_idesc_ab(1, 128, BM, 1, 1);  // dQ^T
+  // leading-byte offset of the K^T operand: from head dims 0..63 to 64..127
+  static constexpr uint32_t KT_LBO = D == 128 ? KV_BOX : Z_OFF - K_OFF;
+};
 
 constexpr uint32_t ERR_WAIT_BWD = 1u << 6;
 
@@ -156,10 +171,11 @@ struct BBars {
 
 // ---------------------------------------------------------------------------- producer
 
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                           const CUtensorMap *tmDO, const BwdParams &p, uint32_t smem,
                           const BBars &bar, volatile uint32_t *abort_flag) {
+  using C = BCfg<D>;
   ptx::prefetch_tmap(tmQ);
   ptx::prefetch_tmap(tmK);
   ptx::prefetch_tmap(tmV);
@@ -169,11 +185,11 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
     const BUnit w = decode_unit<CAUSAL>(p, u);
     if (!wait_phase(bar.kv_empty(), (units_issued & 1u) ^ 1u, abort_flag, ERR_WAIT_BWD))
       goto drain;
-    ptx::mbar_arrive_expect_tx(bar.kv_full(), 2 * KV_TILE);
+    ptx::mbar_arrive_expect_tx(bar.kv_full(), 2 * C::KV_TILE);
 #pragma unroll
-    for (int bx = 0; bx < 2; ++bx) {
-      ptx::tma_load_3d(smem + K_OFF + bx * KV_BOX, tmK, bar.kv_full(), bx * 64, w.j * BN, w.bhk);
-      ptx::tma_load_3d(smem + V_OFF + bx * KV_BOX, tmV, bar.kv_full(), bx * 64, w.j * BN, w.bhk);
+    for (int bx = 0; bx < C::NBOX; ++bx) {
+      ptx::tma_load_3d(smem + C::K_OFF + bx * KV_BOX, tmK, bar.kv_full(), bx * 64, w.j * BN, w.bhk);
+      ptx::tma_load_3d(smem + C::V_OFF + bx * KV_BOX, tmV, bar.kv_full(), bx * 64, w.j * BN, w.bhk);
     }
     ++units_issued;
     for (int s = 0; s < w.steps; ++s) {
@@ -182,17 +198,17 @@ __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const 
       if (!wait_phase(bar.q_empty(st), (use & 1u) ^ 1u, abort_flag, ERR_WAIT_BWD)) goto drain;
       int bh, i;
       step_coords(p, w, s, bh, i);
-      ptx::mbar_arrive_expect_tx(bar.q_full(st), 2 * Q_TILE + VEC_BYTES);
+      ptx::mbar_arrive_expect_tx(bar.q_full(st), 2 * C::Q_TILE + VEC_BYTES);
 #pragma unroll
-      for (int bx = 0; bx < 2; ++bx) {
-        ptx::tma_load_3d(smem + Q_OFF + st * Q_TILE + bx * Q_BOX, tmQ, bar.q_full(st), bx * 64,
+      for (int bx = 0; bx < C::NBOX; ++bx) {
+        ptx::tma_load_3d(smem + C::Q_OFF + st * C::Q_TILE + bx * Q_BOX, tmQ, bar.q_full(st), bx * 64,
                          i * BM, bh);
-        ptx::tma_load_3d(smem + DO_OFF + st * Q_TILE + bx * Q_BOX, tmDO, bar.q_full(st),
+        ptx::tma_load_3d(smem + C::DO_OFF + st * C::Q_TILE + bx * Q_BOX, tmDO, bar.q_full(st),
                          bx * 64, i * BM, bh);
       }
       const long long voff = static_cast<long long>(bh) * p.Npad + i * BM;
-      ptx::bulk_load(smem + VEC_OFF + st * VEC_BYTES, p.l2 + voff, BM * 4, bar.q_full(st));
-      ptx::bulk_load(smem + VEC_OFF + st * VEC_BYTES + BM * 4, p.dd + voff, BM * 4,
+      ptx::bulk_load(smem + C::VEC_OFF + st * VEC_BYTES, p.l2 + voff, BM * 4, bar.q_full(st));
+      ptx::bulk_load(smem + C::VEC_OFF + st * VEC_BYTES + BM * 4, p.dd + voff, BM * 4,
                      bar.q_full(st));
       ++steps_issued;
     }
@@ -210,8 +226,9 @@ drain:
 
 // ---------------------------------------------------------------------------- MMA issuer
 
-// S^T or dP^T: A = K_j or V_j (128 rows, two 128-byte column boxes, K-major), B = Q_i or
-// dO_i (64 rows, two boxes, K-major); K = 128 head dims in steps of 16.
+// S^T or dP^T: A = K_j or V_j (128 rows, D/64 128-byte column boxes, K-major), B = Q_i or
+// dO_i (64 rows, same boxes, K-major); K = D head dims in steps of 16.
+template <int D>
 __device__ __forceinline__ void issue_sdp(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
@@ -219,7 +236,8 @@ __device__ __forceinline__ void issue_sdp(uint32_t tmem_d, uint64_t a_desc, uint
     const uint32_t kb = kk * step;
     const uint32_t aoff = ((kb / 128) * KV_BOX + (kb % 128)) >> 4;
     const uint32_t boff = ((kb / 128) * Q_BOX + (kb % 128)) >> 4;
-    ptx::mma_bf16_ss_elect(tmem_d, a_desc + aoff, b_desc + boff, IDESC_S, kk > 0 ? 1u : 0u);
+    ptx::mma_bf16_ss_elect(tmem_d, a_desc + aoff, b_desc + boff, BCfg<D>::IDESC_S,
+                           kk > 0 ? 1u : 0u);
   }
 }
 
@@ -227,32 +245,38 @@ __device__ __forceinline__ void issue_sdp(uint32_t tmem_d, uint64_t a_desc, uint
 // bf16; queries 0-31 at columns 0-15 (+16 for dS), queries 32-63 at 32-47), B = dO_i or
 // Q_i read MN-major (64 query rows of 128-byte head-dim boxes); K = 64 queries in steps
 // of 16 (8 packed columns, 16 rows of 128 bytes).
+template <int D>
 __device__ __forceinline__ void issue_acc(uint32_t tmem_d, uint32_t tmem_a, uint64_t b_desc,
                                           uint32_t accumulate) {
 #pragma unroll
   for (int kk = 0; kk < BM / 16; ++kk) {
     const uint32_t a = tmem_a + (kk / 2) * 32 + (kk % 2) * 8;
     const uint32_t boff = (kk * 16 * 128) >> 4;
-    ptx::mma_bf16_ts_elect(tmem_d, a, b_desc + boff, IDESC_ACC, kk > 0 ? 1u : accumulate);
+    ptx::mma_bf16_ts_elect(tmem_d, a, b_desc + boff, BCfg<D>::IDESC_ACC,
+                           kk > 0 ? 1u : accumulate);
   }
 }
 
-// dQ^T = K_j^T dS^T: A = K_j read MN-major (M = head dims, two boxes 16 KB apart), B = dS^T
+// dQ^T = K_j^T dS^T: A = K_j read MN-major (M = 128 head dims: two boxes KT_LBO apart, the
+// second a tile of zeros at D = 64), B = dS^T
 // read MN-major (N = 64 queries in one 128-byte row); K = 128 keys in steps of 16 rows.
+template <int D>
 __device__ __forceinline__ void issue_dq(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc) {
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
     const uint32_t off = (kk * 16 * 128) >> 4;
-    ptx::mma_bf16_ss_elect(tmem_d, a_desc + off, b_desc + off, IDESC_DQ, kk > 0 ? 1u : 0u);
+    ptx::mma_bf16_ss_elect(tmem_d, a_desc + off, b_desc + off, BCfg<D>::IDESC_DQ,
+                           kk > 0 ? 1u : 0u);
   }
 }
 
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const BBars &bar,
                          volatile uint32_t *abort_flag) {
-  const uint64_t k_a = ptx::smem_desc_sw128(smem + K_OFF, 16, 1024);
-  const uint64_t v_a = ptx::smem_desc_sw128(smem + V_OFF, 16, 1024);
-  const uint64_t k_t = ptx::smem_desc_sw128(smem + K_OFF, KV_BOX, 1024);
+  using C = BCfg<D>;
+  const uint64_t k_a = ptx::smem_desc_sw128(smem + C::K_OFF, 16, 1024);
+  const uint64_t v_a = ptx::smem_desc_sw128(smem + C::V_OFF, 16, 1024);
+  const uint64_t k_t = ptx::smem_desc_sw128(smem + C::K_OFF, C::KT_LBO, 1024);
   auto wait = [&](uint32_t b, uint32_t parity) {
     const bool ok = wait_phase(b, parity, abort_flag, ERR_WAIT_BWD);
     return __all_sync(0xffffffffu, ok);
@@ -263,12 +287,12 @@ __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const
     const uint32_t use = g >> 1;
     if (!wait(bar.q_full(st), (g / QSTAGES) & 1u)) return false;
     ptx::tc_fence_after();
-    issue_sdp(tmem + s_col(b), k_a, ptx::smem_desc_sw128(smem + Q_OFF + st * Q_TILE, 16, 1024));
+    issue_sdp<D>(tmem + s_col(b), k_a, ptx::smem_desc_sw128(smem + C::Q_OFF + st * C::Q_TILE, 16, 1024));
     // dP^T lands where dQ^T of this buffer's previous step was: wait for its drain.
     if (!wait(bar.dq_empty(b), (use & 1u) ^ 1u)) return false;
     ptx::tc_fence_after();
-    issue_sdp(tmem + dp_col(b), v_a,
-              ptx::smem_desc_sw128(smem + DO_OFF + st * Q_TILE, 16, 1024));
+    issue_sdp<D>(tmem + dp_col(b), v_a,
+              ptx::smem_desc_sw128(smem + C::DO_OFF + st * C::Q_TILE, 16, 1024));
     ptx::mma_commit_elect(bar.sdp_full(b));
     return true;
   };
@@ -285,16 +309,16 @@ __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const
       const uint32_t use = g >> 1;
       if (!(ok = wait(bar.ds_full(b), use & 1u))) break;
       ptx::tc_fence_after();
-      issue_dq(tmem + dp_col(b), k_t, ptx::smem_desc_sw128(smem + DS_OFF, DS_TILE, 1024));
+      issue_dq<D>(tmem + dp_col(b), k_t, ptx::smem_desc_sw128(smem + C::DS_OFF, DS_TILE, 1024));
       ptx::mma_commit_elect(bar.dq_full(b));
       if (s == 0) {
         if (!(ok = wait(bar.acc_empty(), (unit_it & 1u) ^ 1u))) break;
         ptx::tc_fence_after();
       }
-      issue_acc(tmem + DV_COL, tmem + s_col(b),
-                ptx::smem_desc_sw128(smem + DO_OFF + st * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
-      issue_acc(tmem + DK_COL, tmem + s_col(b) + 16,
-                ptx::smem_desc_sw128(smem + Q_OFF + st * Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
+      issue_acc<D>(tmem + C::DV_COL, tmem + s_col(b),
+                ptx::smem_desc_sw128(smem + C::DO_OFF + st * C::Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
+      issue_acc<D>(tmem + C::DK_COL, tmem + s_col(b) + 16,
+                ptx::smem_desc_sw128(smem + C::Q_OFF + st * C::Q_TILE, Q_BOX, 1024), s > 0 ? 1u : 0u);
       ptx::mma_commit_elect(bar.q_empty(st));
       if (s == w.steps - 1) {
         ptx::mma_commit_elect(bar.acc_full());
@@ -315,11 +339,12 @@ __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const
 // q0 .. q0+31 (q0 = i*BM + 32h).  Writes P^T and dS^T as packed bf16 into its own 32
 // columns of the S^T buffer and dS^T into the shared-memory tile (128-byte swizzle: the
 // 16-byte chunk c of row r sits at chunk c ^ (r % 8)).
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ __forceinline__ bool softmax_step(const BwdParams &p, uint32_t tmem_row, uint32_t smem,
                                              const BBars &bar, uint32_t g, int h, int row,
                                              int key, int q0, bool need_mask,
                                              volatile uint32_t *abort_flag) {
+  using C = BCfg<D>;
   const int b = g & 1u, st = g % QSTAGES;
   uint32_t sr[2][16], dr[2][16];
   ptx::tmem_ld16(tmem_row + s_col(b) + h * 32, sr[0]);
@@ -332,7 +357,7 @@ __device__ __forceinline__ bool softmax_step(const BwdParams &p, uint32_t tmem_r
   ptx::reg_fence16(dr[0]);
   ptx::reg_fence16(dr[1]);
   const float *vec = reinterpret_cast<const float *>(
-      __cvta_shared_to_generic(smem + VEC_OFF + st * VEC_BYTES));
+      __cvta_shared_to_generic(smem + C::VEC_OFF + st * VEC_BYTES));
   const float4 *l2v = reinterpret_cast<const float4 *>(vec + h * 32);
   const float4 *ddv = reinterpret_cast<const float4 *>(vec + BM + h * 32);
   uint32_t pp[16], pd[16];
@@ -362,7 +387,7 @@ __device__ __forceinline__ bool softmax_step(const BwdParams &p, uint32_t tmem_r
   if (g > 0 && !wait_phase(bar.dq_full((g - 1) & 1u), ((g - 1) >> 1) & 1u, abort_flag,
                            ERR_WAIT_BWD))
     return false;
-  const uint32_t ds_row = smem + DS_OFF + row * 128;
+  const uint32_t ds_row = smem + C::DS_OFF + row * 128;
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     const uint32_t chunk = static_cast<uint32_t>(h * 4 + cc) ^ static_cast<uint32_t>(row & 7);
@@ -376,9 +401,10 @@ __device__ __forceinline__ bool softmax_step(const BwdParams &p, uint32_t tmem_r
   return true;
 }
 
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const BBars &bar,
                              volatile uint32_t *abort_flag) {
+  using C = BCfg<D>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = warp / 4;                     // query half of the step
   const int row = (warp % 4) * 32 + lane;     // key row within the block
@@ -398,7 +424,7 @@ __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, c
       // masking is needed on the key tail block and, causally, where the block of
       // queries starts before the last key of the block
       const bool need_mask = (w.j * BN + BN > p.Nk) || (CAUSAL && q0 < w.j * BN + BN - 1);
-      if (!softmax_step<CAUSAL>(p, tmem_row, smem, bar, g, h, row, key, q0, need_mask,
+      if (!softmax_step<D, CAUSAL>(p, tmem_row, smem, bar, g, h, row, key, q0, need_mask,
                                 abort_flag))
         return;
       ptx::mbar_arrive(bar.ds_full(b));
@@ -412,7 +438,7 @@ __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, c
 #pragma unroll 1
     for (int c = 0; c < D / 16; ++c) {
       uint32_t r[16];
-      ptx::tmem_ld16(tmem_row + (h == 0 ? DV_COL : DK_COL) + c * 16, r);
+      ptx::tmem_ld16(tmem_row + (h == 0 ? C::DV_COL : C::DK_COL) + c * 16, r);
       ptx::tmem_wait_ld();
       ptx::reg_fence16(r);
       uint32_t o[8];
@@ -438,13 +464,17 @@ __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, c
 // fp32 tile into the warp's staging buffer (one 128-byte row per query, so every store
 // instruction of the warp fills one row) and add the tile into the accumulator with one
 // bulk tensor reduce-add.  Queries past Nq fall outside the tensor and are not written.
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ void dq_role(const CUtensorMap *tmDQ, const BwdParams &p, uint32_t smem, uint32_t tmem,
                         const BBars &bar, volatile uint32_t *abort_flag) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int wq = warp % 4;
   const uint32_t tmem_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  const uint32_t stage = smem + DQS_OFF + wq * DQ_STAGE;
+  using C = BCfg<D>;
+  // warps whose head dims lie past D (D = 64: the zero rows of dQ^T) read and release
+  // the buffer but add nothing
+  const bool owner = wq < C::DRAIN_WARPS;
+  const uint32_t stage = smem + C::DQS_OFF + (owner ? wq : 0) * DQ_STAGE;
   if (lane == 0) ptx::prefetch_tmap(tmDQ);
   uint32_t gd = 0;
   bool pending = false;
@@ -464,6 +494,7 @@ __device__ void dq_role(const CUtensorMap *tmDQ, const BwdParams &p, uint32_t sm
       for (int c = 0; c < 4; ++c) ptx::reg_fence16(r[c]);
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.dq_empty(b));
+      if (!owner) continue;
       // the previous reduce must have read the staging tile before it is overwritten
       if (pending && lane == 0) ptx::bulk_wait_read_all();
       __syncwarp();
@@ -492,17 +523,18 @@ done:
 
 // ---------------------------------------------------------------------------- kernels
 
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+  using C = BCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t smem = (raw + 1023u) & ~1023u;  // 1024-aligned for 128-byte swizzle
   uint8_t *smem_gen = smem_raw + (smem - raw);
-  const BBars bar{smem + BAR_OFF};
-  uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + CTL_OFF);
+  const BBars bar{smem + C::BAR_OFF};
+  uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + C::CTL_OFF);
   volatile uint32_t *tmem_slot = ctl;
   volatile uint32_t *abort_flag = ctl + 1;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -530,20 +562,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tmem_alloc(ptx::smem_addr(ctl), TMEM_COLS);
     ptx::tmem_relinquish();
   }
+  if (C::Z_BYTES > 0) {
+    // the zero rows of the K^T operand (D = 64), visible to the tensor core
+    for (int o = threadIdx.x * 16; o < C::Z_BYTES; o += NUM_THREADS * 16)
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(smem + C::Z_OFF + o), "r"(0u)
+                   : "memory");
+    ptx::fence_proxy_async_smem();
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp < DRAIN_WARP0) {
-    softmax_role<CAUSAL>(p, smem, tmem, bar, abort_flag);
+    softmax_role<D, CAUSAL>(p, smem, tmem, bar, abort_flag);
   } else if (warp < MMA_WARP) {
-    dq_role<CAUSAL>(&tmDQ, p, smem, tmem, bar, abort_flag);
+    dq_role<D, CAUSAL>(&tmDQ, p, smem, tmem, bar, abort_flag);
   } else if (warp == MMA_WARP) {
-    mma_role<CAUSAL>(p, smem, tmem, bar, abort_flag);
+    mma_role<D, CAUSAL>(p, smem, tmem, bar, abort_flag);
     __syncwarp();
   } else if (warp == TMA_WARP) {
-    if (lane == 0) load_role<CAUSAL>(&tmQ, &tmK, &tmV, &tmDO, p, smem, bar, abort_flag);
+    if (lane == 0) load_role<D, CAUSAL>(&tmQ, &tmK, &tmV, &tmDO, p, smem, bar, abort_flag);
     __syncwarp();
   }
 
@@ -557,7 +596,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // Per query row: D = sum_t dO_t O_t (fp32 from bf16) and LSE * log2(e), into arrays
 // padded to Npad rows per (batch, head) (D = 0, LSE = +inf on the padding, so padded
-// queries contribute nothing).  One warp per row, 4 elements per lane (D = 128).
+// queries contribute nothing).  One warp per row, HD / 32 elements per lane.
+template <int HD>
 __global__ void fa_bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_t *__restrict__ dout,
                                    const float *__restrict__ lse, float *__restrict__ l2,
                                    float *__restrict__ dd, long long rows_padded, int Nq, int Npad) {
@@ -574,11 +614,15 @@ __global__ void fa_bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_
     return;
   }
   const long long row = bh * Nq + q;
-  const uint2 a = reinterpret_cast<const uint2 *>(o + row * D)[lane];
-  const uint2 g = reinterpret_cast<const uint2 *>(dout + row * D)[lane];
-  auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
-  auto hi = [](uint32_t x) { return __uint_as_float(x & 0xffff0000u); };
-  float s = lo(a.x) * lo(g.x) + hi(a.x) * hi(g.x) + lo(a.y) * lo(g.y) + hi(a.y) * hi(g.y);
+  constexpr int W = HD / 64;  // 32-bit words (bf16 pairs) per lane
+  const uint32_t *a = reinterpret_cast<const uint32_t *>(o + row * HD) + lane * W;
+  const uint32_t *g = reinterpret_cast<const uint32_t *>(dout + row * HD) + lane * W;
+  float s = 0.f;
+#pragma unroll
+  for (int n = 0; n < W; ++n) {
+    s += __uint_as_float(a[n] << 16) * __uint_as_float(g[n] << 16);
+    s += __uint_as_float(a[n] & 0xffff0000u) * __uint_as_float(g[n] & 0xffff0000u);
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) {

@@ -167,17 +167,19 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
  *   o, lse      the forward's outputs for these inputs (o bf16 [B,Hq,Nq,d], lse fp32)
  *   dout        bf16 [B,Hq,Nq,d], the gradient of the loss with respect to o
  *   dq          bf16 [B,Hq,Nq,d] out;  dk, dv  bf16 [B,Hkv,Nk,d] out
- *   B, Hq, Hkv, Nq, Nk, scale, causal   as for fa_fwd;  d must be 128; causal requires
- *   Nq == Nk
+ *   B, Hq, Hkv, Nq, Nk, scale, causal   as for fa_fwd;  d must be 64 or 128; causal
+ *   requires Nq == Nk
  *
  * All pointers 16-byte aligned (lse 4-byte).  The outputs must not overlap the inputs.
- * Scratch: the call allocates B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes on `stream` with
- * cudaMallocAsync (an fp32 dQ accumulator and two per-row vectors) and frees it on the
- * same stream with cudaFreeAsync.  dQ is summed with fp32 reduce-adds whose order varies,
- * so its last bits may differ between runs (dK and dV do not).  Enqueues a memset and three kernels.  Returns FA_OK once
- * enqueued; FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (d != 128, causal with Nq != Nk,
- * GPU not sm_100) with nothing enqueued; FA_ERR_CUDA if the scratch allocation or a launch
- * failed.
+ * Scratch: the call allocates B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes on `stream` (an
+ * fp32 dQ accumulator and two per-row vectors) from a stream-ordered memory pool that the
+ * library creates per device on first use, and frees it on the same stream.  The pool
+ * keeps up to 4 GiB of freed scratch for later calls for the life of the process.  dQ is
+ * summed with fp32 reduce-adds whose order varies, so its last bits may differ between
+ * runs (dK and dV do not).  Enqueues a memset and three kernels.  Returns FA_OK once
+ * enqueued; FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (d not 64 or 128, causal with
+ * Nq != Nk, GPU not sm_100) with nothing enqueued; FA_ERR_CUDA if the scratch allocation
+ * or a launch failed.
  */
 fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
                  const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv,

@@ -139,7 +139,8 @@ def test_bwd_invalid_arguments(kw):
     assert bwd_call(**kw) == fa.FA_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("kw", [dict(d=64), dict(d=256), dict(causal=1, Nq=128, Nk=256)])
+@pytest.mark.parametrize("kw", [dict(d=32), dict(d=96), dict(d=256),
+                                dict(causal=1, Nq=128, Nk=256)])
 def test_bwd_unsupported_configurations(kw):
     assert bwd_call(**kw) == fa.FA_ERR_UNSUPPORTED
 
@@ -150,7 +151,7 @@ def test_bwd_noalloc_validates_like_fa_bwd_and_rejects_oversize_scratch():
                                                     "dv", "B", "Hq", "Hkv", "Nq", "Nk", "d",
                                                     "scale", "causal")] + [None]
     assert fa.fa_bwd_noalloc(*args(q=0)) == fa.FA_ERR_INVALID_ARG
-    assert fa.fa_bwd_noalloc(*args(d=64)) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_bwd_noalloc(*args(d=256)) == fa.FA_ERR_UNSUPPORTED
     # B*Hq*Nq*d*4 = 128 MiB of dQ accumulator: more than the fixed 64 MiB scratch
     assert fa.fa_bwd_noalloc(*args(Hq=16, Hkv=16, Nq=16384, Nk=16384)) == fa.FA_ERR_UNSUPPORTED
 

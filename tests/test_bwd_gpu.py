@@ -45,9 +45,8 @@ def errors(got, ref, natural):
             float(np.abs(d).max() / max(np.abs(ref).max(), floor)))
 
 
-def check(shape, causal, seed=0, scale=None):
+def check(shape, causal, seed=0, scale=None, d=128):
     B, Hq, Hkv, Nq, Nk = shape
-    d = 128
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     scale = float(torch.tensor(scale, dtype=torch.float32))
     q = random_bf16((B, Hq, Nq, d), seed + 1)
@@ -81,6 +80,21 @@ def test_gradients_match_oracle(cuda_ok, shape, causal):
 @pytest.mark.parametrize("shape", [(1, 2, 2, 100, 300), (1, 2, 1, 300, 77)])
 def test_gradients_non_square(cuda_ok, shape):
     print(shape, check(shape, False))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [
+    (1, 1, 1, 1, 1), (1, 2, 2, 64, 64), (1, 2, 1, 200, 200), (2, 4, 2, 333, 333),
+    (1, 4, 1, 1000, 1000),
+])
+def test_gradients_head_dim_64(cuda_ok, shape, causal):
+    """d = 64: one 128-byte box per row; the dQ^T product runs on a zero-padded K^T."""
+    print(shape, causal, check(shape, causal, seed=7, d=64))
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 100, 300), (1, 4, 2, 300, 77)])
+def test_gradients_head_dim_64_non_square(cuda_ok, shape):
+    print(shape, check(shape, False, seed=9, d=64))
 
 
 def test_gradients_larger_scores(cuda_ok):

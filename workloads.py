@@ -118,6 +118,8 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("long_bwd", 1, 32, 32, 16384, 128, False, "bf16", "bf16", 1003, kind="bwd"),
     Workload("long_causal_bwd", 1, 32, 32, 16384, 128, True, "bf16", "bf16", 1003, kind="bwd"),
     Workload("gqa_causal_bwd", 4, 32, 8, 8192, 128, True, "bf16", "bf16", 1004, kind="bwd"),
+    Workload("gpt2_bwd", 16, 12, 12, 2048, 64, False, "bf16", "bf16", 1002, kind="bwd"),
+    Workload("gpt2_causal_bwd", 16, 12, 12, 2048, 64, True, "bf16", "bf16", 1002, kind="bwd"),
 ]}
 
 
