@@ -7,8 +7,8 @@
  * backward pass but computes it again ("Flash Attention" page, section "Zentrale
  * technische Innovationen", the bullet on recomputation, and its overview).  What the
  * backward pass computes is fixed by calculus: for O = P V with P = softmax(S) taken row
- * by row, S = scale * Q K^T over the admissible keys (j <= i under the causal mask), and an
- * upstream gradient dO,
+ * by row, S = scale * Q K^T over the admissible keys (j <= i + Nk - Nq under the causal
+ * mask, aligned at the bottom right as in the forward oracle), and an upstream gradient dO,
  *
  *   dV     = P^T dO
  *   dP     = dO V^T
@@ -17,7 +17,9 @@
  *   dK     = scale * dS^T Q
  *
  * With grouped heads (query head hq reads K/V head hq / (Hq / Hkv)), the dK and dV of a
- * K/V head are the sums over the query heads that read it.
+ * K/V head are the sums over the query heads that read it.  A query row without any
+ * admissible key (causal, Nq > Nk) has the constant output O = 0, so its dQ row is zero
+ * and it adds nothing to dK and dV.
  *
  * Evaluation, per (batch, K/V head) and all binary64: first the query rows (score row,
  * its maximum and sum, P row, dP row, the row term sum_k P_ik dP_ik, dQ row), keeping each
@@ -50,8 +52,7 @@ static double dot_rows(const void *a, int64_t ia, const void *b, int64_t ib, int
 /*
  * q, dout: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; all of one element type.
  * Outputs dq [B, Hq, Nq, d], dk and dv [B, Hkv, Nk, d] in fp64.
- * Causal masking requires Nq == Nk.  Returns 0, -1 on invalid arguments, -2 on
- * allocation failure.
+ * Returns 0, -1 on invalid arguments, -2 on allocation failure.
  */
 int oracle_attention_bwd(const void *q, const void *k, const void *v, const void *dout,
                          int elem_type, int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
@@ -60,7 +61,6 @@ int oracle_attention_bwd(const void *q, const void *k, const void *v, const void
     if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
     if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || d < 1 || Hq % Hkv != 0) return -1;
     if (elem_type != BWD_F64 && elem_type != BWD_BF16) return -1;
-    if (causal && Nq != Nk) return -1;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #else
@@ -91,7 +91,14 @@ int oracle_attention_bwd(const void *q, const void *k, const void *v, const void
                     for (int64_t gi = 0; gi < group * Nq; ++gi) {
                         const int64_t hq = hk * group + gi / Nq, i = gi % Nq;
                         const int64_t qoff = ((b * Hq + hq) * Nq + i) * d;
-                        const int64_t nkeys = causal ? i + 1 : Nk;
+                        const int64_t last = i + (Nk - Nq); /* last key the mask admits */
+                        const int64_t nkeys = !causal ? Nk : (last < Nk ? last + 1 : Nk);
+                        if (nkeys <= 0) {
+                            for (int64_t t = 0; t < d; ++t) dq[qoff + t] = 0.0;
+                            lse[gi] = -INFINITY;
+                            rowterm[gi] = 0.0;
+                            continue;
+                        }
                         double m = -INFINITY;
                         for (int64_t j = 0; j < nkeys; ++j) {
                             s[j] = scale * dot_rows(q, qoff, k, kvoff + j * d, elem_type, d);
@@ -126,7 +133,7 @@ int oracle_attention_bwd(const void *q, const void *k, const void *v, const void
                 for (int64_t t = 0; t < d; ++t) dvr[t] = dkr[t] = 0.0;
                 for (int64_t gi = 0; gi < group * Nq; ++gi) {
                     const int64_t hq = hk * group + gi / Nq, i = gi % Nq;
-                    if (causal && j > i) continue;
+                    if (causal && j > i + (Nk - Nq)) continue;
                     const int64_t qoff = ((b * Hq + hq) * Nq + i) * d;
                     const double sij = scale * dot_rows(q, qoff, k, kvoff + j * d, elem_type, d);
                     const double p = exp(sij - lse[gi]);

@@ -19,22 +19,31 @@ def rnd(shape, seed):
 
 
 def torch_grads(q, k, v, do, scale, causal):
+    """float64 autograd of the definition.  Causal masks align at the bottom right (query i
+    sees key j iff j <= i + Nk - Nq); a query row with no admissible key has O = 0."""
     group = q.shape[1] // k.shape[1]
+    Nq, Nk = q.shape[2], k.shape[2]
     tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
     kk, vv = tk.repeat_interleave(group, 1), tv.repeat_interleave(group, 1)
-    if q.shape[2] == k.shape[2] or not causal:
+    if Nq == Nk or not causal:
         o = torch.nn.functional.scaled_dot_product_attention(tq, kk, vv, is_causal=causal,
                                                              scale=scale)
+    else:
+        keep = torch.ones(Nq, Nk, dtype=torch.bool).tril(diagonal=Nk - Nq)
+        s = (scale * tq @ kk.transpose(-1, -2)).masked_fill(~keep, -np.inf)
+        m = s.amax(-1, keepdim=True).detach()
+        e = torch.exp(s - torch.where(torch.isfinite(m), m, torch.zeros_like(m)))
+        den = e.sum(-1, keepdim=True)
+        o = (e / torch.where(den > 0, den, torch.ones_like(den))) @ vv
     o.backward(torch.tensor(do))
     return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("shape", [(1, 2, 2, 17, 17, 8), (2, 4, 1, 9, 9, 16), (1, 3, 3, 5, 23, 4)])
+@pytest.mark.parametrize("shape", [(1, 2, 2, 17, 17, 8), (2, 4, 1, 9, 9, 16), (1, 3, 3, 5, 23, 4),
+                                   (1, 2, 1, 23, 5, 4)])
 def test_matches_torch_autograd(shape, causal):
     B, Hq, Hkv, Nq, Nk, d = shape
-    if causal and Nq != Nk:
-        pytest.skip("causal needs Nq == Nk")
     q, do = rnd((B, Hq, Nq, d), 1), rnd((B, Hq, Nq, d), 2)
     k, v = rnd((B, Hkv, Nk, d), 3), rnd((B, Hkv, Nk, d), 4)
     got = oracle.attention_bwd(q, k, v, do, 0.37, causal)
@@ -43,12 +52,14 @@ def test_matches_torch_autograd(shape, causal):
         assert np.abs(g - r).max() < 1e-12
 
 
-@pytest.mark.parametrize("causal", [False, True])
-def test_matches_finite_differences_of_the_forward_oracle(causal):
-    """d/dx of L = sum(dO * O) by central differences of the forward oracle."""
-    B, Hq, Hkv, N, d = 1, 2, 1, 5, 3
-    q, k, v = rnd((B, Hq, N, d), 5), rnd((B, Hkv, N, d), 6), rnd((B, Hkv, N, d), 7)
-    do = rnd((B, Hq, N, d), 8)
+@pytest.mark.parametrize("causal,nq,nk", [(False, 5, 5), (True, 5, 5), (True, 3, 6),
+                                           (True, 6, 3), (False, 6, 3)])
+def test_matches_finite_differences_of_the_forward_oracle(causal, nq, nk):
+    """d/dx of L = sum(dO * O) by central differences of the forward oracle (whose causal
+    mask is aligned at the bottom right when Nq != Nk)."""
+    B, Hq, Hkv, d = 1, 2, 1, 3
+    q, k, v = rnd((B, Hq, nq, d), 5), rnd((B, Hkv, nk, d), 6), rnd((B, Hkv, nk, d), 7)
+    do = rnd((B, Hq, nq, d), 8)
     scale, h = 0.6, 1e-6
     got = dict(zip("qkv", oracle.attention_bwd(q, k, v, do, scale, causal)))
 
@@ -100,7 +111,14 @@ def test_bf16_inputs_decode_exactly():
         assert np.array_equal(x, y)
 
 
-def test_rejects_causal_with_unequal_lengths():
-    with pytest.raises(ValueError):
-        oracle.attention_bwd(rnd((1, 1, 4, 2), 0), rnd((1, 1, 5, 2), 0), rnd((1, 1, 5, 2), 0),
-                             rnd((1, 1, 4, 2), 0), 1.0, True)
+def test_causal_rows_without_keys_have_zero_gradient():
+    """Causal with Nq = 7 > Nk = 3: query rows 0..3 see no key, so O is the constant 0 there;
+    their dQ rows vanish and they add nothing to dK and dV (the gradients of K and V equal
+    those of the problem restricted to rows 4..6, which is square and causal)."""
+    q, do = rnd((1, 2, 7, 4), 40), rnd((1, 2, 7, 4), 41)
+    k, v = rnd((1, 2, 3, 4), 42), rnd((1, 2, 3, 4), 43)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, 0.7, True)
+    assert not dq[:, :, :4].any()
+    dq2, dk2, dv2 = oracle.attention_bwd(q[:, :, 4:], k, v, do[:, :, 4:], 0.7, True)
+    assert np.array_equal(dq[:, :, 4:], dq2)
+    assert np.abs(dk - dk2).max() < 1e-14 and np.abs(dv - dv2).max() < 1e-14

@@ -143,14 +143,20 @@ def pin_quantise_rounding_bound(lib):
 
 
 def pin_bwd_autograd(lib):
-    for causal in (False, True):
-        q, do = rnd((1, 4, 7, 4), 30), rnd((1, 4, 7, 4), 31)
-        k, v = rnd((1, 2, 7, 4), 32), rnd((1, 2, 7, 4), 33)
+    for causal, nq, nk in ((False, 7, 7), (True, 7, 7), (True, 5, 9), (True, 9, 5)):
+        q, do = rnd((1, 4, nq, 4), 30), rnd((1, 4, nq, 4), 31)
+        k, v = rnd((1, 2, nk, 4), 32), rnd((1, 2, nk, 4), 33)
         got = oracle.attention_bwd(q, k, v, do, 0.45, causal, _library=lib)
         tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
-        o = torch.nn.functional.scaled_dot_product_attention(
-            tq, tk.repeat_interleave(2, 1), tv.repeat_interleave(2, 1), is_causal=causal,
-            scale=0.45)
+        # bottom-right causal mask; rows with no admissible key have O = 0
+        keep = torch.ones(nq, nk, dtype=torch.bool)
+        if causal:
+            keep = keep.tril(diagonal=nk - nq)
+        s = (0.45 * tq @ tk.repeat_interleave(2, 1).transpose(-1, -2)).masked_fill(~keep, -np.inf)
+        m = s.amax(-1, keepdim=True).detach()
+        e = torch.exp(s - torch.where(torch.isfinite(m), m, torch.zeros_like(m)))
+        den = e.sum(-1, keepdim=True)
+        o = (e / torch.where(den > 0, den, torch.ones_like(den))) @ tv.repeat_interleave(2, 1)
         o.backward(torch.tensor(do))
         for g, r in zip(got, (tq.grad, tk.grad, tv.grad)):
             assert np.abs(g - r.numpy()).max() < 1e-12
@@ -231,7 +237,11 @@ MUTANTS = {
     "bwd_dq_scale_dropped": ("dq[qoff + t] = scale * acc;", "dq[qoff + t] = acc;"),
     "bwd_dv_reads_q": ("dvr[t] += p * ld(dout, elem_type, qoff + t);",
                        "dvr[t] += p * ld(q, elem_type, qoff + t);"),
-    "bwd_causal_off_by_one": ("if (causal && j > i) continue;", "if (causal && j >= i) continue;"),
+    "bwd_causal_off_by_one": ("if (causal && j > i + (Nk - Nq)) continue;",
+                              "if (causal && j >= i + (Nk - Nq)) continue;"),
+    "bwd_key_pass_top_left": ("if (causal && j > i + (Nk - Nq)) continue;",
+                              "if (causal && j > i) continue;"),
+    "bwd_query_pass_top_left": ("const int64_t last = i + (Nk - Nq);", "const int64_t last = i;"),
     "bwd_lse_without_sum": ("lse[gi] = m + log(l);", "lse[gi] = m;"),
     "bwd_dp_reads_k": ("dp[j] = dot_rows(dout, qoff, v, kvoff + j * d, elem_type, d);",
                        "dp[j] = dot_rows(dout, qoff, k, kvoff + j * d, elem_type, d);"),
