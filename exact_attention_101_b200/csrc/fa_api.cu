@@ -562,7 +562,6 @@ fa_status check_bwd_args(const void *q, const void *k, const void *v, const void
       Nk > INT32_MAX - 2 * fa::bwd::BN)
     return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (causal && Nq != Nk) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -637,6 +636,7 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
   p.Nq = Nq;
   p.Nk = Nk;
   p.group = Hq / Hkv;
+  p.diag = Nk - Nq;
   p.num_qb = (Nq + fa::bwd::BM - 1) / fa::bwd::BM;
   p.Npad = p.num_qb * fa::bwd::BM;
   p.num_kb = (Nk + fa::bwd::BN - 1) / fa::bwd::BN;

@@ -115,6 +115,7 @@ struct BwdParams {
   const float *dd;     // [B*Hq, Npad]: D = rowsum(dO o O), 0 past Nq
   uint16_t *dk, *dv;   // bf16 [B*Hkv, Nk, D]
   int B, Hq, Hkv, Nq, Nk, Npad, group;
+  int diag;            // Nk - Nq: the causal mask admits key j for query i iff j <= i + diag
   int num_kb;          // ceil(Nk / BN)
   int num_qb;          // ceil(Nq / BM)
   int num_units;       // B * Hkv * num_kb
@@ -138,9 +139,11 @@ __device__ __forceinline__ BUnit decode_unit(const BwdParams &p, int u) {
   w.j = u % p.num_kb;
   w.b = w.bhk / p.Hkv;
   w.hk = w.bhk % p.Hkv;
-  // Under the causal mask query i sees key j only if j <= i: blocks of queries that end
-  // before the key block starts are skipped.
-  w.i0 = CAUSAL ? (w.j * BN) / BM : 0;
+  // Under the causal mask query i sees key j only if j <= i + diag: blocks of queries that
+  // end before the key block's first admitting query are skipped.  Query Nq - 1 admits
+  // every key, so no unit is left without steps.
+  const int first = w.j * BN - p.diag;  // first query that sees key j*BN
+  w.i0 = CAUSAL && first > 0 ? first / BM : 0;
   w.nq = p.num_qb - w.i0;
   w.steps = p.group * w.nq;
   return w;
@@ -372,7 +375,7 @@ __device__ __forceinline__ bool softmax_step(const BwdParams &p, uint32_t tmem_r
       const float s = __uint_as_float(sr[c / 16][c % 16]);
       const float dpv = __uint_as_float(dr[c / 16][c % 16]);
       float pe = ptx::ex2(fmaf(s, p.scale_log2, -lv[e]));
-      if (need_mask && (key >= p.Nk || (CAUSAL && key > q0 + c))) pe = 0.f;
+      if (need_mask && (key >= p.Nk || (CAUSAL && key > q0 + c + p.diag))) pe = 0.f;
       pv[e] = pe;
       sv[e] = pe * (dpv - dv[e]);
     }
@@ -421,9 +424,11 @@ __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, c
       int bh, i;
       step_coords(p, w, s, bh, i);
       const int q0 = i * BM + h * 32;
-      // masking is needed on the key tail block and, causally, where the block of
-      // queries starts before the last key of the block
-      const bool need_mask = (w.j * BN + BN > p.Nk) || (CAUSAL && q0 < w.j * BN + BN - 1);
+      // masking is needed on the key tail block and, causally, where the first query of
+      // the block does not admit the block's last key (this covers the rows that admit
+      // no key at all when Nq > Nk: their LSE is -inf and only the mask zeroes P)
+      const bool need_mask =
+          (w.j * BN + BN > p.Nk) || (CAUSAL && q0 + p.diag < w.j * BN + BN - 1);
       if (!softmax_step<D, CAUSAL>(p, tmem_row, smem, bar, g, h, row, key, q0, need_mask,
                                 abort_flag))
         return;

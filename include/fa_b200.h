@@ -167,8 +167,9 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
  *   o, lse      the forward's outputs for these inputs (o bf16 [B,Hq,Nq,d], lse fp32)
  *   dout        bf16 [B,Hq,Nq,d], the gradient of the loss with respect to o
  *   dq          bf16 [B,Hq,Nq,d] out;  dk, dv  bf16 [B,Hkv,Nk,d] out
- *   B, Hq, Hkv, Nq, Nk, scale, causal   as for fa_fwd;  d must be 64 or 128; causal
- *   requires Nq == Nk
+ *   B, Hq, Hkv, Nq, Nk, scale, causal   as for fa_fwd (the causal mask aligned at the
+ *   bottom right); d must be 64 or 128.  Query rows that admit no key (causal, Nq > Nk:
+ *   O = 0, LSE = -inf) get a zero dQ row and add nothing to dK and dV.
  *
  * All pointers 16-byte aligned (lse 4-byte).  The outputs must not overlap the inputs.
  * Scratch: the call allocates B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes on `stream` (an
@@ -177,9 +178,8 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float
  * keeps up to 4 GiB of freed scratch for later calls for the life of the process.  dQ is
  * summed with fp32 reduce-adds whose order varies, so its last bits may differ between
  * runs (dK and dV do not).  Enqueues a memset and three kernels.  Returns FA_OK once
- * enqueued; FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (d not 64 or 128, causal with
- * Nq != Nk, GPU not sm_100) with nothing enqueued; FA_ERR_CUDA if the scratch allocation
- * or a launch failed.
+ * enqueued; FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (d not 64 or 128, GPU not sm_100)
+ * with nothing enqueued; FA_ERR_CUDA if the scratch allocation or a launch failed.
  */
 fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
                  const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv,

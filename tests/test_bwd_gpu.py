@@ -77,9 +77,13 @@ def test_gradients_match_oracle(cuda_ok, shape, causal):
     print(shape, causal, check(shape, causal))
 
 
-@pytest.mark.parametrize("shape", [(1, 2, 2, 100, 300), (1, 2, 1, 300, 77)])
-def test_gradients_non_square(cuda_ok, shape):
-    print(shape, check(shape, False))
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [(1, 2, 2, 100, 300), (1, 2, 1, 300, 77), (1, 2, 2, 129, 513),
+                                   (2, 4, 2, 513, 129), (1, 1, 1, 1, 700), (1, 2, 1, 700, 1)])
+def test_gradients_non_square(cuda_ok, shape, causal):
+    """Nq != Nk; under the causal mask aligned at the bottom right, so with Nq > Nk the
+    first Nq - Nk query rows admit no key (zero dQ rows)."""
+    print(shape, causal, check(shape, causal))
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -92,9 +96,10 @@ def test_gradients_head_dim_64(cuda_ok, shape, causal):
     print(shape, causal, check(shape, causal, seed=7, d=64))
 
 
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("shape", [(1, 2, 2, 100, 300), (1, 4, 2, 300, 77)])
-def test_gradients_head_dim_64_non_square(cuda_ok, shape):
-    print(shape, check(shape, False, seed=9, d=64))
+def test_gradients_head_dim_64_non_square(cuda_ok, shape, causal):
+    print(shape, causal, check(shape, causal, seed=9, d=64))
 
 
 def test_gradients_larger_scores(cuda_ok):
