@@ -487,9 +487,9 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, fl
 }
 
 // One 64-column score row (sr) -> numerators in TMEM at t_p.  Adds the sum of the
-// numerators as rounded for the tensor core (bf16 only) to lr and of the unrounded
-// numerators to le.  NPOLY of every 8 column pairs use the polynomial exponential.
-// Numerators are packed and stored to TMEM 32 columns at a time (64 for e4m3).
+// unrounded numerators to le.  NPOLY of every 8 column pairs use the polynomial
+// exponential.  Numerators are packed and stored to TMEM 32 columns at a time (64 for
+// e4m3).
 // Keep masks of a 32-key block: bytes >= thr become 0xff (two keys per 16-bit mask half
 // below), from the four 64-bit Philox words.
 __device__ __forceinline__ void keep_bytes(const uint64_t (&r)[4], uint32_t thr4,
@@ -503,12 +503,11 @@ __device__ __forceinline__ void keep_bytes(const uint64_t (&r)[4], uint32_t thr4
 
 template <bool FP8, int NPOLY, bool DROPOUT = false>
 __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], float sl2,
-                                                   float neg_m, uint32_t t_p, float &lr,
-                                                   float &le, const uint32_t (*keep)[8] = nullptr) {
+                                                   float neg_m, uint32_t t_p, float &le,
+                                                   const uint32_t (*keep)[8] = nullptr) {
   const uint64_t scale2 = ptx::f2_pack(sl2, sl2);
   const uint64_t bias2 = ptx::f2_pack(neg_m, neg_m);
-  uint64_t acc_r[2] = {0ull, 0ull};  // packed (0.f, 0.f)
-  uint64_t acc_e[2] = {0ull, 0ull};
+  uint64_t acc_e[2] = {0ull, 0ull};  // packed (0.f, 0.f)
   constexpr int SCOLS = FP8 ? 64 : 32;  // score columns per 16-column TMEM store
 #pragma unroll
   for (int q = 0; q < 64 / SCOLS; ++q) {
@@ -533,13 +532,7 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], 
     if (!FP8) {
 #pragma unroll
       for (int e = 0; e < SCOLS; e += 2) {
-        const uint32_t pp = ptx::pack_bf16x2(pv[e], pv[e + 1]);
-        pk[e / 2] = pp;
-        // sum of the rounded values the tensor core multiplies with V, so that O stays a
-        // convex combination of value rows
-        acc_r[(e / 2) & 1] = ptx::f2_add(
-            acc_r[(e / 2) & 1],
-            ptx::f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u)));
+        pk[e / 2] = ptx::pack_bf16x2(pv[e], pv[e + 1]);
         if (DROPOUT) {
           // dropped keys leave the product (not the sum): key byte masks to 16-bit halves
           const uint32_t kb = keep[q][e / 4];
@@ -553,13 +546,9 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], 
     }
     ptx::tmem_st16(t_p + q * 16, pk);
   }
-  float a0, a1, b0, b1;
+  float a0, a1;
   ptx::f2_unpack(ptx::f2_add(acc_e[0], acc_e[1]), a0, a1);
   le += a0 + a1;
-  if (!FP8) {
-    ptx::f2_unpack(ptx::f2_add(acc_r[0], acc_r[1]), b0, b1);
-    lr += b0 + b1;
-  }
 }
 
 // Softmax warps: warpgroup x (warps 4x..4x+3) handles Q tile x, one thread per query row
@@ -593,8 +582,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
     // the row has none).
     const int key_lim = CAUSAL ? min(row + w.off, w.len_k - 1) : w.len_k - 1;
     float m_used = NEG_INF;  // running maximum in use, base-2 scaled domain
-    float l = 0.f;           // running sum of the numerators as rounded for the P V product
-    float l_exact = 0.f;     // running sum of the unrounded numerators (for the LSE)
+    float l = 0.f;           // running sum of the (unrounded, fp32) numerators
 
     for (int j = 0; j < nx; ++j) {
       const int b = j & 1;
@@ -658,7 +646,6 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       }
       if (resc) {
         l *= alpha;
-        l_exact *= alpha;
         m_used = xmax;
       }
       const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
@@ -666,7 +653,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       // Numerators p = 2^(s*sl2 - m_used), packed for the P V product.  Tiles without
       // masked entries send EXP2_POLY_PAIRS of every 8 column pairs to the FMA-pipe
       // polynomial and the rest to the MUFU unit.
-      float lr = 0.f, le = 0.f;
+      float le = 0.f;
       const uint32_t t_p = t_s + C::P_OFF;
       if (DROPOUT) {
         // two Philox blocks: keys kv0 .. kv0+31 and kv0+32 .. kv0+63 of this row
@@ -678,18 +665,17 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
                           static_cast<uint64_t>(w.bh), 0ull, p.seed, p.offset, r);
           keep_bytes(r, p.drop_thr4, keep[h]);
         }
-        softmax_numerators<FP8, 0, true>(sr, sl2, neg_m, t_p, lr, le, keep);
+        softmax_numerators<FP8, 0, true>(sr, sl2, neg_m, t_p, le, keep);
       } else if (EXP2_POLY_PAIRS == 0)   // one copy of the unrolled loop: smaller code, faster
-        softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, lr, le);
+        softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, le);
       else if (need_mask)
-        softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, lr, le);
+        softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, le);
       else
-        softmax_numerators<FP8, EXP2_POLY_PAIRS>(sr, sl2, neg_m, t_p, lr, le);
-      l_exact += le;
-      if (FP8)
-        l = l_exact;
-      else
-        l += lr;
+        softmax_numerators<FP8, EXP2_POLY_PAIRS>(sr, sl2, neg_m, t_p, le);
+      // O is normalised by the sum of the unrounded numerators: the bf16 (e4m3) values the
+      // tensor core multiplies with V then sum to 1 within one rounding (2^-9 relative for
+      // bf16), and the LSE comes from the same sum
+      l += le;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.p_full(x, b));
@@ -697,7 +683,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
     pv_base += nx;
 
     // Epilogue: O = O_acc / l (times the V descale for fp8),
-    // LSE = ln 2 * (m_used + log2 l_exact).
+    // LSE = ln 2 * (m_used + log2 l).
     {
       bool ok = wait_phase(bar.o_full(x), unit_it & 1u, abort_flag, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;
@@ -748,8 +734,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
         }
       }
       if (valid)
-        p.lse[lrow] = l_exact > 0.f ? (m_used + log2f(l_exact)) * 0.69314718055994530942f
-                                    : NEG_INF;
+        p.lse[lrow] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : NEG_INF;
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar.o_empty(x));
     }
