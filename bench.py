@@ -498,7 +498,25 @@ def run_ours(args):
     elif fp8:
         hds = [t.pin_memory() for t in (inp.descale_q, inp.descale_k, inp.descale_v)]
 
+    # Plain bf16 forward: the public host-memory entry point (fa_fwd_host), whose copies in
+    # both directions overlap the kernels chunk by chunk.  Other workloads: pinned copies on
+    # the stream around the device-memory call.
+    host_api = w.kind == "fwd" and not fp8 and not w.dropout
+    # kernels per end-to-end step: fa_fwd_host's default chunk count (about one wave of
+    # work units per chunk), else the device call's own launches
+    if host_api:
+        unit_rows = 128 if w.d > 128 else 256
+        units = w.B * w.Hq * (-(-w.N // unit_rows))
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        e2e_launches = e2e_steps * min(w.B * w.Hkv, max(1, units // sms))
+    else:
+        e2e_launches = e2e_steps * launches_per_step
+
     def e2e_step():
+        if host_api:
+            fa.forward_host(hq_, hk_, hv_, causal=w.causal, scale=w.scale, out_dtype=out_dtype,
+                            out=ho, lse=hl, device_buffers=(q, k, v, o, lse), stream=stream)
+            return
         q.copy_(hq_, non_blocking=True)
         k.copy_(hk_, non_blocking=True)
         v.copy_(hv_, non_blocking=True)
@@ -540,7 +558,9 @@ def run_ours(args):
             h2d += o.numel() * o.element_size() + lse.numel() * lse.element_size()
             d2h = sum(t.numel() * t.element_size() for t in (dq, dk, dv))
         e2e = {"value": w.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "api": ("fa_fwd_host: pinned host buffers, copies pipelined by head chunks"
+                       if host_api else "pinned copies on the stream around the device call")}
 
     if world > 1:
         import torch.distributed as dist
@@ -596,7 +616,7 @@ def run_ours(args):
                      "kernel": kernel_name},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * (args.steps + e2e_steps),
+        "gpu_launches": launches_per_step * args.steps + e2e_launches,
         "clocks": clk,
     }
     if quant is not None:

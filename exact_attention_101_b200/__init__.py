@@ -20,7 +20,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
-C_SYMBOLS = ("fa_fwd", "fa_fwd_dropout", "fa_fwd_varlen", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
+C_SYMBOLS = ("fa_fwd", "fa_fwd_host", "fa_fwd_dropout", "fa_fwd_varlen", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
              "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_string",
              "fa_version")
 
@@ -44,6 +44,8 @@ def lib() -> ctypes.CDLL:
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.fa_fwd.restype = i
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+        L.fa_fwd_host.restype = i
+        L.fa_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, i, f, i, i, i, vp]
         L.fa_fwd_dropout.restype = i
         L.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, f,
                                      ctypes.c_uint64, ctypes.c_uint64, i, vp]
@@ -75,6 +77,14 @@ def lib() -> ctypes.CDLL:
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
     """Raw ``fa_fwd``: pointers are ints (device addresses), stream an int handle."""
     return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream)
+
+
+def fa_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev,
+                B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, chunks, stream) -> int:
+    """Raw ``fa_fwd_host``: host and device addresses as ints."""
+    return lib().fa_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev,
+                             o_dev, lse_dev, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
+                             int(chunks), stream)
 
 
 def fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dropout_p, seed,
@@ -183,6 +193,50 @@ def forward(q, k, v, causal=False, scale=None, out_dtype=None, out=None, lse=Non
                 B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), dtype, _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def forward_host(q, k, v, causal=False, scale=None, out_dtype=None, out=None, lse=None,
+                 device_buffers=None, chunks=0, device=None, stream=None):
+    """``forward`` for bf16 [B, H, N, d] tensors in host memory (pinned memory lets the
+    copies overlap the kernel).  Returns host ``(o, lse)``, pinned when q is.
+    ``device_buffers`` = (q, k, v, o, lse) CUDA tensors of the right shapes to reuse;
+    otherwise they are allocated on ``device`` (default: the current CUDA device)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("%s must be a contiguous bf16 host tensor [B, H, N, d]" % name)
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError("q, k, v shapes do not match")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    pin = q.is_pinned()
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=out_dtype, pin_memory=pin)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, pin_memory=pin)
+    for name, t in (("out", out), ("lse", lse)):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous host tensor" % name)
+    if device_buffers is None:
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        device_buffers = (torch.empty(q.shape, dtype=q.dtype, device=dev),
+                          torch.empty(k.shape, dtype=k.dtype, device=dev),
+                          torch.empty(v.shape, dtype=v.dtype, device=dev),
+                          torch.empty(out.shape, dtype=out.dtype, device=dev),
+                          torch.empty(lse.shape, dtype=lse.dtype, device=dev))
+    qd, kd, vd, od, ld = device_buffers
+    dtype = FA_BF16_OUT_F32 if out_dtype == torch.float32 else FA_BF16
+    st = fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr(),
+                     B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), dtype, chunks,
+                     _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_host")
     return out, lse
 
 

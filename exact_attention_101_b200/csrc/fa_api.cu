@@ -750,6 +750,126 @@ fa_status bwd_noalloc(const void *q, const void *k, const void *v, const void *o
                     stream, ws);
 }
 
+// ---------------------------------------------------------------- host-memory forward
+
+// Per device: a stream for host-to-device copies, one for device-to-host copies, and the
+// events that order them against the caller's stream.  Created on first use, kept for
+// the life of the process; the mutex serialises the enqueueing of calls that share them.
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, in_done = nullptr, chunk_done = nullptr, out_done = nullptr;
+  std::mutex mu;
+  fa_status st = FA_ERR_CUDA;
+};
+
+HostPipe &host_pipe(int dev) {
+  static HostPipe pipes[kMaxDevices];
+  static std::once_flag once[kMaxDevices];
+  HostPipe &hp = pipes[dev];
+  std::call_once(once[dev], [&] {
+    const unsigned ef = cudaEventDisableTiming;
+    const bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.start, ef) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.in_done, ef) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.chunk_done, ef) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&hp.out_done, ef) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    hp.st = ok ? FA_OK : FA_ERR_CUDA;
+  });
+  return hp;
+}
+
+// The forward for Q, K, V, O and LSE in host memory, pipelined by chunks of heads.  A
+// chunk is a run of consecutive K/V heads (flattened over the batch) with the query heads
+// that read them: for every tensor that is one contiguous byte range, and on the device
+// it is an ordinary problem with B = 1.  Chunk c's inputs are copied on the input stream
+// while the kernel of chunk c-1 runs on `stream` and the outputs of chunk c-2 go back on
+// the output stream.
+fa_status fwd_host(const void *qh, const void *kh, const void *vh, void *oh, float *lseh,
+                   void *qd, void *kd, void *vd, void *od, float *lsed, int B, int Hq, int Hkv,
+                   int Nq, int Nk, int d, float scale, int causal, bool out_f32, int chunks,
+                   cudaStream_t stream) {
+  if (!qh || !kh || !vh || !oh || !lseh || chunks < 0) return FA_ERR_INVALID_ARG;
+  // the whole problem first, so that nothing is enqueued for an invalid request
+  fa_status st = check_args(qd, kd, vd, od, lsed, B, Hq, Hkv, Nq, Nk, d, scale, causal, false,
+                            nullptr, nullptr, nullptr);
+  if (st != FA_OK) return st;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  const uint64_t groups = static_cast<uint64_t>(B) * Hkv;  // K/V heads, flattened
+  const uint64_t g = static_cast<uint64_t>(Hq / Hkv);      // query heads per K/V head
+  const uint64_t q_head = static_cast<uint64_t>(Nq) * d * 2;
+  const uint64_t kv_head = static_cast<uint64_t>(Nk) * d * 2;
+  const uint64_t o_head = static_cast<uint64_t>(Nq) * d * (out_f32 ? 4 : 2);
+  const uint64_t lse_head = static_cast<uint64_t>(Nq) * 4;
+  if (!buffer_ok(qd, groups * g * q_head, dev) || !buffer_ok(kd, groups * kv_head, dev) ||
+      !buffer_ok(vd, groups * kv_head, dev) || !buffer_ok(od, groups * g * o_head, dev) ||
+      !buffer_ok(lsed, groups * g * lse_head, dev))
+    return FA_ERR_INVALID_ARG;
+  // default: about one wave of work units per chunk, so that a chunk's kernel takes about
+  // as long as its copies and the first copy and last kernel, which overlap nothing, are short
+  uint64_t n = static_cast<uint64_t>(chunks);
+  if (chunks == 0) {
+    DeviceInfo info;
+    st = device_info(dev, &info);
+    if (st != FA_OK) return st;
+    const uint64_t unit_rows = d > 128 ? fa::BM : fa::UNIT_ROWS;
+    const uint64_t units = groups * g * ((static_cast<uint64_t>(Nq) + unit_rows - 1) / unit_rows);
+    n = units / static_cast<uint64_t>(info.sms);
+    if (n < 1) n = 1;
+  }
+  if (n > groups) n = groups;
+  HostPipe &hp = host_pipe(dev);
+  if (hp.st != FA_OK) return hp.st;
+  std::lock_guard<std::mutex> lk(hp.mu);
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  auto bytes = [](const void *p, uint64_t off) {
+    return static_cast<const uint8_t *>(p) + off;
+  };
+  auto wbytes = [](void *p, uint64_t off) { return static_cast<uint8_t *>(p) + off; };
+  // nothing may overwrite the device buffers before the caller's earlier work is done
+  if (!ok(cudaEventRecord(hp.start, stream)) || !ok(cudaStreamWaitEvent(hp.in, hp.start, 0)) ||
+      !ok(cudaStreamWaitEvent(hp.out, hp.start, 0)))
+    st = FA_ERR_CUDA;
+  for (uint64_t c = 0; c < n && st == FA_OK; ++c) {
+    const uint64_t c0 = groups * c / n, c1 = groups * (c + 1) / n;  // K/V heads [c0, c1)
+    const uint64_t qo = c0 * g * q_head, qn = (c1 - c0) * g * q_head;
+    const uint64_t ko = c0 * kv_head, kn = (c1 - c0) * kv_head;
+    const uint64_t oo = c0 * g * o_head, on = (c1 - c0) * g * o_head;
+    const uint64_t lo = c0 * g * lse_head, ln = (c1 - c0) * g * lse_head;
+    if (!ok(cudaMemcpyAsync(wbytes(qd, qo), bytes(qh, qo), qn, cudaMemcpyHostToDevice, hp.in)) ||
+        !ok(cudaMemcpyAsync(wbytes(kd, ko), bytes(kh, ko), kn, cudaMemcpyHostToDevice, hp.in)) ||
+        !ok(cudaMemcpyAsync(wbytes(vd, ko), bytes(vh, ko), kn, cudaMemcpyHostToDevice, hp.in)) ||
+        !ok(cudaEventRecord(hp.in_done, hp.in)) ||
+        !ok(cudaStreamWaitEvent(stream, hp.in_done, 0))) {
+      st = FA_ERR_CUDA;
+      break;
+    }
+    st = fwd_common(bytes(qd, qo), bytes(kd, ko), bytes(vd, ko), wbytes(od, oo),
+                    reinterpret_cast<float *>(wbytes(lsed, lo)), 1,
+                    static_cast<int>((c1 - c0) * g), static_cast<int>(c1 - c0), Nq, Nk, d, scale,
+                    causal, out_f32, false, nullptr, nullptr, nullptr, stream);
+    if (st != FA_OK) break;
+    if (!ok(cudaEventRecord(hp.chunk_done, stream)) ||
+        !ok(cudaStreamWaitEvent(hp.out, hp.chunk_done, 0)) ||
+        !ok(cudaMemcpyAsync(wbytes(oh, oo), bytes(od, oo), on, cudaMemcpyDeviceToHost, hp.out)) ||
+        !ok(cudaMemcpyAsync(wbytes(lseh, lo), bytes(lsed, lo), ln, cudaMemcpyDeviceToHost,
+                            hp.out)))
+      st = FA_ERR_CUDA;
+  }
+  // whatever was enqueued, the caller's stream ends after all of it
+  if (!ok(cudaEventRecord(hp.in_done, hp.in)) || !ok(cudaStreamWaitEvent(stream, hp.in_done, 0)) ||
+      !ok(cudaEventRecord(hp.out_done, hp.out)) ||
+      !ok(cudaStreamWaitEvent(stream, hp.out_done, 0))) {
+    cudaGetLastError();
+    if (st == FA_OK) st = FA_ERR_CUDA;
+  }
+  if (st == FA_ERR_CUDA) cudaGetLastError();
+  return st;
+}
+
 }  // namespace
 
 extern "C" {
@@ -775,6 +895,16 @@ fa_status fa_quantize_e4m3(const void *x, const int8_t *signs, void *x8, float *
                            int H, int N, int d, fa_stream_t stream) {
   return quantize_common(x, signs, x8, descale, B, H, N, d,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
+                      float *lse_host, void *q_dev, void *k_dev, void *v_dev, void *o_dev,
+                      float *lse_dev, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                      int causal, fa_dtype dtype, int chunks, fa_stream_t stream) {
+  if (dtype != FA_BF16 && dtype != FA_BF16_OUT_F32) return FA_ERR_INVALID_ARG;
+  return fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev,
+                  B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype == FA_BF16_OUT_F32, chunks,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse, int B,

@@ -86,6 +86,42 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *ls
                  fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * fa_fwd for tensors that live in host memory.  The pages describe the kernel, whose
+ * inputs already sit in GPU memory; this call is a transfer pipeline around it for
+ * callers whose Q, K, V and results are in host memory.  The problem is cut into chunks of
+ * consecutive K/V heads (flattened over the batch) together with the query heads that read
+ * them; for every tensor a chunk is one contiguous byte range.  Chunk c's inputs are
+ * copied host -> device on an internal stream while the kernel of chunk c-1 runs on
+ * `stream` and the outputs of earlier chunks are copied device -> host on a second
+ * internal stream, so with pinned host memory the copies in both directions overlap the
+ * computation.  The result equals fa_fwd on the same data, bit for bit.
+ *
+ *   q_host, k_host, v_host   host pointers, bf16, layout as for fa_fwd; read
+ *   o_host, lse_host         host pointers, written (o bf16 or fp32 as dtype, lse fp32)
+ *   q_dev .. lse_dev         device buffers of fa_fwd's sizes and alignment, owned by the
+ *                            caller; they hold the copies and the device-side results
+ *   chunks                   number of chunks (clamped to B*Hkv); 0 picks about one wave
+ *                            of the kernel per chunk: (work units) / (SMs), at least 1
+ *   other arguments as for fa_fwd (dtype FA_BF16 or FA_BF16_OUT_F32)
+ *
+ * Ordering: nothing touches the buffers before the work already enqueued on `stream` has
+ * finished, and work enqueued on `stream` after this call starts only once every copy of
+ * it has finished; the call returns once everything is enqueued (with pageable host
+ * memory the CUDA runtime may block inside the copies).  The host buffers must stay valid
+ * and unmodified until then.  The library allocates no memory per call; it keeps two
+ * streams and four events per device, created on first use, and serialises the enqueueing
+ * of concurrent calls on one device.  Returns FA_OK; FA_ERR_INVALID_ARG for a null host
+ * pointer, chunks < 0 or any argument fa_fwd would reject, with nothing enqueued;
+ * FA_ERR_CUDA if a copy or launch could not be enqueued (the caller's stream still waits
+ * for what was).
+ */
+fa_status fa_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                      void *o_host, float *lse_host, void *q_dev, void *k_dev, void *v_dev,
+                      void *o_dev, float *lse_dev, int B, int Hq, int Hkv, int Nq, int Nk,
+                      int d, float scale, int causal, fa_dtype dtype, int chunks,
+                      fa_stream_t stream);
+
+/*
  * fa_fwd with dropout on the attention weights, fused into the kernel: the page "Flash
  * Attention" (section "Zentrale technische Innovationen", the fusion bullet) lists dropout
  * among the operations fused with the softmax.  With P the attention weights of a row,

@@ -80,6 +80,31 @@ def test_unsupported_configurations(kw):
     assert call(**kw) == fa.FA_ERR_UNSUPPORTED
 
 
+HOST_OK = dict(qh=A, kh=A, vh=A, oh=A, lh=A, qd=A, kd=A, vd=A, od=A, ld=A, B=1, Hq=4, Hkv=2,
+               Nq=256, Nk=256, d=128, scale=0.088, causal=0, dtype=fa.FA_BF16, chunks=0)
+
+
+def host_call(**kw):
+    a = dict(HOST_OK)
+    a.update(kw)
+    return fa.fa_fwd_host(*(a[n] for n in ("qh", "kh", "vh", "oh", "lh", "qd", "kd", "vd", "od",
+                                          "ld", "B", "Hq", "Hkv", "Nq", "Nk", "d", "scale",
+                                          "causal", "dtype", "chunks")), None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(qh=0), dict(kh=0), dict(vh=0), dict(oh=0), dict(lh=0), dict(chunks=-1),
+    dict(qd=0), dict(od=A + 4), dict(ld=A + 2), dict(Hq=3), dict(scale=0.0),
+    dict(dtype=fa.FA_E4M3), dict(B=0),
+])
+def test_host_entry_invalid_arguments(kw):
+    assert host_call(**kw) == fa.FA_ERR_INVALID_ARG
+
+
+def test_host_entry_unsupported_head_dim():
+    assert host_call(d=96) == fa.FA_ERR_UNSUPPORTED
+
+
 def test_fp8_entry_validation():
     args = (A, A, A, A, A, 1, 2, 2, 128, 128)
     # missing descales
