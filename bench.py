@@ -502,13 +502,14 @@ def run_ours(args):
     # both directions overlap the kernels chunk by chunk.  Other workloads: pinned copies on
     # the stream around the device-memory call.
     host_api = w.kind == "fwd" and not fp8 and not w.dropout
-    # kernels per end-to-end step: fa_fwd_host's default chunk count (about one wave of
-    # work units per chunk), else the device call's own launches
+    # kernels per end-to-end step: fa_fwd_host's default chunk count (as many K/V heads per
+    # chunk as fit one wave of work units), else the device call's own launches
     if host_api:
         unit_rows = 128 if w.d > 128 else 256
-        units = w.B * w.Hq * (-(-w.N // unit_rows))
+        group_units = (w.Hq // w.Hkv) * (-(-w.N // unit_rows))
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        e2e_launches = e2e_steps * min(w.B * w.Hkv, max(1, units // sms))
+        per = max(1, sms // group_units)
+        e2e_launches = e2e_steps * (-(-(w.B * w.Hkv) // per))
     else:
         e2e_launches = e2e_steps * launches_per_step
 

@@ -808,17 +808,21 @@ fa_status fwd_host(const void *qh, const void *kh, const void *vh, void *oh, flo
       !buffer_ok(vd, groups * kv_head, dev) || !buffer_ok(od, groups * g * o_head, dev) ||
       !buffer_ok(lsed, groups * g * lse_head, dev))
     return FA_ERR_INVALID_ARG;
-  // default: about one wave of work units per chunk, so that a chunk's kernel takes about
-  // as long as its copies and the first copy and last kernel, which overlap nothing, are short
-  uint64_t n = static_cast<uint64_t>(chunks);
+  // Chunk plan: chunk c covers K/V heads [c * per, min(groups, (c + 1) * per)) when the
+  // library picks the size (chunks == 0), else an even split into `chunks` pieces.  The
+  // library's size is as many K/V heads as fit one wave of work units (one CTA per SM),
+  // at least one: a chunk's kernel then takes about as long as its copies, and a chunk
+  // just over a wave, which would take two wave-times, never occurs.
+  uint64_t n = static_cast<uint64_t>(chunks), per = 0;
   if (chunks == 0) {
     DeviceInfo info;
     st = device_info(dev, &info);
     if (st != FA_OK) return st;
     const uint64_t unit_rows = d > 128 ? fa::BM : fa::UNIT_ROWS;
-    const uint64_t units = groups * g * ((static_cast<uint64_t>(Nq) + unit_rows - 1) / unit_rows);
-    n = units / static_cast<uint64_t>(info.sms);
-    if (n < 1) n = 1;
+    const uint64_t group_units = g * ((static_cast<uint64_t>(Nq) + unit_rows - 1) / unit_rows);
+    per = static_cast<uint64_t>(info.sms) / group_units;
+    if (per < 1) per = 1;
+    n = (groups + per - 1) / per;
   }
   if (n > groups) n = groups;
   HostPipe &hp = host_pipe(dev);
@@ -834,7 +838,9 @@ fa_status fwd_host(const void *qh, const void *kh, const void *vh, void *oh, flo
       !ok(cudaStreamWaitEvent(hp.out, hp.start, 0)))
     st = FA_ERR_CUDA;
   for (uint64_t c = 0; c < n && st == FA_OK; ++c) {
-    const uint64_t c0 = groups * c / n, c1 = groups * (c + 1) / n;  // K/V heads [c0, c1)
+    // K/V heads [c0, c1)
+    const uint64_t c0 = per ? c * per : groups * c / n;
+    const uint64_t c1 = per ? (c0 + per < groups ? c0 + per : groups) : groups * (c + 1) / n;
     const uint64_t qo = c0 * g * q_head, qn = (c1 - c0) * g * q_head;
     const uint64_t ko = c0 * kv_head, kn = (c1 - c0) * kv_head;
     const uint64_t oo = c0 * g * o_head, on = (c1 - c0) * g * o_head;

@@ -100,8 +100,9 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *ls
  *   o_host, lse_host         host pointers, written (o bf16 or fp32 as dtype, lse fp32)
  *   q_dev .. lse_dev         device buffers of fa_fwd's sizes and alignment, owned by the
  *                            caller; they hold the copies and the device-side results
- *   chunks                   number of chunks (clamped to B*Hkv); 0 picks about one wave
- *                            of the kernel per chunk: (work units) / (SMs), at least 1
+ *   chunks                   number of chunks (an even split, clamped to B*Hkv); 0 lets
+ *                            the library size them: as many K/V heads per chunk as fit
+ *                            one wave of the kernel's work units, at least one
  *   other arguments as for fa_fwd (dtype FA_BF16 or FA_BF16_OUT_F32)
  *
  * Ordering: nothing touches the buffers before the work already enqueued on `stream` has
