@@ -117,10 +117,13 @@ def test_dk_dv_deterministic(cuda_ok):
     assert (a[0].float() - b[0].float()).abs().max() <= 1e-2 * a[0].float().abs().max()
 
 
+@pytest.mark.parametrize("shape", [(1, 8, 8, 16384, 128), (16, 12, 12, 2048, 64)],
+                         ids=["long_h8", "gpt2"])
 @pytest.mark.parametrize("causal", [False, True])
-def test_full_size_gradient_identities(cuda_ok, causal):
-    """At the long-context size (too large for the full oracle) check what holds for any
-    input: sum_j dV_j = sum_i dO_i, and sum_j dK_j = 0 (rows of dS sum to zero).
+def test_full_size_gradient_identities(cuda_ok, causal, shape):
+    """At the long-context size and the GPT-2 backward workload's size (d = 64), too large
+    for the full oracle, check what holds for any input: sum_j dV_j = sum_i dO_i, and
+    sum_j dK_j = 0 (rows of dS sum to zero).
 
     Error budget (u = 2^-8), per component (head, t): in the dV identity the bf16
     rounding of the summed rows gives about u/sqrt(3) * sqrt(sum_j dV_jt^2), and rounding
@@ -132,7 +135,7 @@ def test_full_size_gradient_identities(cuda_ok, causal):
     is off by about scale * u * sqrt(N) * rms(O) rms(dO) sqrt(d) rms(q) per component;
     the bound takes 6 times that (the maximum over all components, and margin).  rms(O) is
     taken from 64 oracle rows per head."""
-    B, Hq, Hkv, N, d = 1, 8, 8, 16384, 128
+    B, Hq, Hkv, N, d = shape
     scale = float(torch.tensor(1.0 / np.sqrt(d), dtype=torch.float32))
     q, k, v, do = (random_bf16((B, Hq if s in (0, 3) else Hkv, N, d), 50 + s)
                    for s in range(4))

@@ -58,3 +58,25 @@ def test_threshold_zero_equals_fa_fwd_and_offset_changes_the_mask(cuda_ok):
     b = run(q, k, v, 0.25, 5, 0, False, 0.088)[0]
     c = run(q, k, v, 0.25, 5, 1, False, 0.088)[0]
     assert torch.equal(a, b) and not torch.equal(a, c)
+
+
+def test_dropout_full_size_sampled(cuda_ok):
+    """The dropout benchmark workload at full size (B1 H32 N16384 d128, p = 0.1, offset 0
+    as in the bench's first timed step), rows sampled over four heads, against the oracle."""
+    import workloads
+    from parity_util import sample_rows
+    w = workloads.WORKLOADS["long_dropout"]
+    inp = workloads.make_inputs(w)
+    o, lse = run(inp.q, inp.k, inp.v, w.dropout, w.seed, 0, w.causal, w.scale)
+    rows = sample_rows(w.B, w.Hq, w.N, n_heads=4, n_random=96, seed=w.seed)
+    thr = min(255, int(round(w.dropout * 256)))
+    ro, rl = oracle.attention_dropout_rows(inp.q, inp.k, inp.v, w.scale, w.causal, thr, w.seed,
+                                           0, rows=rows)
+    og = o.reshape(-1, w.d)[rows].double().numpy()
+    err = np.abs(og - ro)
+    grow = 1.0 / (1.0 - thr / 256.0)
+    stats = (float(err.max()), float(err.mean()),
+             float(np.abs(lse.reshape(-1)[rows].double().numpy() - rl).max()))
+    print(stats)
+    assert stats[0] <= BF16_MAX_ABS * grow and stats[1] <= BF16_MEAN_ABS * grow
+    assert stats[2] <= LSE_MAX_ABS

@@ -86,7 +86,8 @@ def test_deterministic(cuda_ok):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-@pytest.mark.parametrize("name", ["gpt2", "gpt2_causal", "long", "long_causal", "gqa_causal"])
+@pytest.mark.parametrize("name", ["gpt2", "gpt2_causal", "long", "long_causal", "gqa_causal",
+                                  "long_d256", "long_d256_causal"])
 def test_full_size_workloads_sampled(cuda_ok, name):
     w = W[name]
     inp = workloads.make_inputs(w)

@@ -116,3 +116,35 @@ def test_fixed_length_causal_bottom_right(cuda_ok, nq, nk):
     ro, rl = oracle.attention(q, k, v, D_SCALE[d], True)
     print(check_rows(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), ro.reshape(-1, d),
                      rl.reshape(-1)))
+
+
+def test_varlen_full_size_sampled(cuda_ok):
+    """The varlen benchmark workload at full size (16 sequences of 256 .. 8192 tokens,
+    H = 32, d = 128, causal) in the bench's launch configuration; rows sampled from the
+    shortest, the longest and a middle sequence (first, last and random rows of two heads
+    each) against the oracle on that sequence alone."""
+    import workloads
+    w = workloads.WORKLOADS["varlen_causal"]
+    inp = workloads.make_inputs(w)
+    lens = workloads.varlen_lengths(w)
+    dev = torch.device("cuda", 0)
+    cu_d = inp.cu_seqlens.to(dev)
+    o, lse = fa.forward_varlen(inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), cu_d, cu_d,
+                               max(lens), causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+    o, lse = o.cpu(), lse.cpu()
+    order = np.argsort(lens)
+    rng = np.random.default_rng(w.seed)
+    for b in (int(order[0]), int(order[len(order) // 2]), int(order[-1])):
+        t0, n = int(inp.cu_seqlens[b]), lens[b]
+        seq = lambda t: t[t0:t0 + n].transpose(0, 1).unsqueeze(0).contiguous()  # [1, H, n, d]
+        heads = [0, w.Hq - 1]
+        idx = sorted(set([0, 1, 127, 128, n // 2, n - 2, n - 1])
+                     | set(int(x) for x in rng.integers(0, n, size=48)))
+        rows = np.array([h * n + i for h in heads for i in idx])
+        ro, rl = oracle.attention_rows(seq(inp.q), seq(inp.k), seq(inp.v), w.scale, w.causal,
+                                       rows=rows)
+        go = torch.stack([o[t0 + i, h] for h in heads for i in idx])
+        gl = torch.stack([lse[h, t0 + i] for h in heads for i in idx])
+        print(b, n, compare_bf16(go, gl, ro, rl))
