@@ -22,18 +22,19 @@
 // useful K/V ring in shared memory, so a unit is one Q tile (NT = 1) and warps 4-7 and 10
 // stay idle.
 //
-// Key tiles are BN = 64 keys, and every Q tile has TWO score buffers in tensor memory:
-// while the softmax warps of a tile turn S(j) into P(j), the tensor core already
-// computes S(j+1) (and S(j+2) as soon as P(j) has been consumed).  So a tile's softmax
-// never waits for its own P.V product, and the two tiles' softmax warps -- one of each per
-// SM sub-partition -- can both be busy at once.  This matters on B200 because, at head
-// dim 128, the exponentials of one score tile take the SFU as long as the tensor core
-// takes for that tile's two products.
+// Key tiles are BN = 64 keys, and every Q tile has NBUF score buffers in tensor memory
+// (two; three at head dim 64, where the smaller O leaves room): while the softmax warps of
+// a tile turn S(j) into P(j), the tensor core already computes S(j+1) .. S(j+NBUF-1), and
+// S(j+NBUF) as soon as P(j) has been consumed.  So a tile's softmax never waits for its
+// own P.V product, and the two tiles' softmax warps -- one of each per SM sub-partition --
+// can both be busy at once.  This matters on B200 because, at head dim 128, the
+// exponentials of one score tile take the SFU as long as the tensor core takes for that
+// tile's two products.
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit), BN = 64:
-//   S(x, b) at x*128 + b*64, 64 fp32 columns (tile x, buffer b); the numerators P of
+//   S(x, b) at x*NBUF*64 + b*64, 64 fp32 columns (tile x, buffer b); the numerators P of
 //   that buffer (bf16 pairs or e4m3 quads packed in 32-bit columns) overwrite its upper
-//   32 columns; O_x accumulator at 256 + x*D.
+//   32 columns; O_x accumulator at O_COL0 + x*D (O_COL0 = 256, or 384 at head dim 64).
 //
 // Registers: the kernel is launched with LAUNCH_REGS per thread (384 threads); the third
 // warpgroup gives registers back (setmaxnreg.dec to OTHER_REGS) and the two softmax
@@ -52,8 +53,8 @@
 //   pv_done[x]              one P.V product of tile x finished (for the rare rescale)
 //   o_full[x] / o_empty[x]  O_x final for the unit / read out by the epilogue
 //
-// MMA order of tile x inside a unit (j = key tile): S(x, 0), S(x, 1), then for every j
-// PV(x, j), S(x, j+2).  S(x, j+2) reuses the buffer of P(x, j) and is issued after
+// MMA order of tile x inside a unit (j = key tile): S(x, 0) .. S(x, NBUF-1), then for
+// every j PV(x, j), S(x, j+NBUF).  S(x, j+NBUF) reuses the buffer of P(x, j) and is issued after
 // PV(x, j) by the same thread: tcgen05 operations from one thread run in issue order, so
 // the product reads P before the next scores overwrite it.
 //
@@ -132,22 +133,25 @@ struct TileCfg {
   static constexpr uint32_t AB_FORMAT = FP8 ? 0u : 1u;  // e4m3 : bf16
   static constexpr uint32_t IDESC_S = ptx::make_idesc(AB_FORMAT, BM, BN, 0);
   static constexpr uint32_t IDESC_O = ptx::make_idesc(AB_FORMAT, BM, D, 1);
-  // TMEM column map.
+  // TMEM column map.  Score buffers per Q tile: three at D = 64 (tensor memory then holds
+  // 3 x 64 score columns and a 64-column O per tile), so that the scores run two products
+  // ahead of the softmax; two otherwise.
+  static constexpr int NBUF = (D == 64 && !FP8) ? 3 : 2;
+  static constexpr uint32_t S_COLS = NBUF * 64;          // score columns of one Q tile
+  __host__ __device__ static constexpr uint32_t s_col(int x, int b) { return x * S_COLS + b * 64; }
   static constexpr uint32_t P_OFF = 32;                  // P inside a 64-column S buffer
-  static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
-  static_assert(256 + NT * D <= (int)TMEM_COLS, "TMEM budget");
+  static constexpr uint32_t O_COL0 = NT * S_COLS > 256 ? NT * S_COLS : 256, O_COL1 = O_COL0 + D;
+  static_assert(O_COL0 + NT * D <= TMEM_COLS, "TMEM budget");
   // Shared memory map (offsets from a 1024-aligned base).
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NT * Q_TILE_BYTES;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * KV_TILE_BYTES;
-  static constexpr int NUM_BARS = 2 * NSLOT + 18;
+  static constexpr int NUM_BARS = 2 * NSLOT + 22;
   static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// TMEM column of score buffer b of Q tile x.
-__host__ __device__ constexpr uint32_t s_col(int x, int b) { return x * 128 + b * 64; }
 
 struct FwdParams {
   void *o;
@@ -276,12 +280,13 @@ struct Bars {
   __device__ uint32_t slot_empty(int s) const { return base + 8u * (NSLOT + s); }
   __device__ uint32_t q_full() const { return base + 8u * (2 * NSLOT + 0); }
   __device__ uint32_t q_empty() const { return base + 8u * (2 * NSLOT + 1); }
-  __device__ uint32_t s_full(int x, int b) const { return base + 8u * (2 * NSLOT + 2 + 2 * x + b); }
-  __device__ uint32_t p_full(int x, int b) const { return base + 8u * (2 * NSLOT + 6 + 2 * x + b); }
-  __device__ uint32_t pv_done(int x) const { return base + 8u * (2 * NSLOT + 10 + x); }
-  __device__ uint32_t o_full(int x) const { return base + 8u * (2 * NSLOT + 12 + x); }
-  __device__ uint32_t o_empty(int x) const { return base + 8u * (2 * NSLOT + 14 + x); }
-  __device__ uint32_t drain(int x) const { return base + 8u * (2 * NSLOT + 16 + x); }
+  // three score buffers reserved per Q tile (TileCfg::NBUF of them used)
+  __device__ uint32_t s_full(int x, int b) const { return base + 8u * (2 * NSLOT + 2 + 3 * x + b); }
+  __device__ uint32_t p_full(int x, int b) const { return base + 8u * (2 * NSLOT + 8 + 3 * x + b); }
+  __device__ uint32_t pv_done(int x) const { return base + 8u * (2 * NSLOT + 14 + x); }
+  __device__ uint32_t o_full(int x) const { return base + 8u * (2 * NSLOT + 16 + x); }
+  __device__ uint32_t o_empty(int x) const { return base + 8u * (2 * NSLOT + 18 + x); }
+  __device__ uint32_t drain(int x) const { return base + 8u * (2 * NSLOT + 20 + x); }
 };
 
 // ---------------------------------------------------------------------------- producer
@@ -380,7 +385,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint6
 }
 
 // One MMA warp per Q tile x (warp 8 for tile 0, warp 10 for tile 1), so that each tile's
-// chain P(x, j) -> PV(x, j) -> S(x, j+2) waits only for its own softmax warps while the
+// chain P(x, j) -> PV(x, j) -> S(x, j+NBUF) waits only for its own softmax warps while the
 // other warp keeps the tensor core busy.  Runs on all 32 lanes of the warp; waits are
 // polled by every lane and made warp-uniform, MMAs and commits are issued by one elected
 // lane.  K/V ring slots and the Q tiles are shared by the two tiles: each is released by
@@ -413,8 +418,8 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
     if (also_tile0) ptx::mbar_arrive_elect(bar.slot_empty(idx % C::NSLOT));
   };
   auto scores = [&](const Unit &w, int nx, int j, uint32_t ki) {
-    issue_s<D, FP8>(tmem + s_col(x, j & 1), q_d, k_d0 + (ki % C::NSLOT) * SLOT_STEP);
-    ptx::mma_commit_elect(bar.s_full(x, j & 1));
+    issue_s<D, FP8>(tmem + C::s_col(x, j % C::NBUF), q_d, k_d0 + (ki % C::NSLOT) * SLOT_STEP);
+    ptx::mma_commit_elect(bar.s_full(x, j % C::NBUF));
     release(ki, x == 1 && j >= w.n0);
     if (j == nx - 1) ptx::mma_commit_elect(bar.q_empty());
   };
@@ -424,29 +429,29 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
     const int nx = x ? w.n1 : w.n0;
     if (!wait(bar.q_full(), unit_it & 1u)) break;
     bool ok = true;
-    for (int j = 0; j < 2 && j < nx; ++j) {
+    for (int j = 0; j < C::NBUF && j < nx; ++j) {
       if (!wait_slot(kv_base + 2 * j)) { ok = false; break; }
       ptx::tc_fence_after();
       scores(w, nx, j, kv_base + 2 * j);
     }
     for (int j = 0; j < nx && ok; ++j) {
-      const int b = j & 1;
+      const int b = j % C::NBUF;
       const uint32_t vi = kv_base + 2 * j + 1;    // V_j
       if (!wait_slot(vi)) { ok = false; break; }
       if (!wait(bar.p_full(x, b), (pph >> b) & 1u)) { ok = false; break; }
       pph ^= 1u << b;
       if (j == 0 && !wait(bar.o_empty(x), (unit_it & 1u) ^ 1u)) { ok = false; break; }
       ptx::tc_fence_after();
-      issue_pv<D, FP8>(t_o, tmem + s_col(x, b) + C::P_OFF, v_d0 + (vi % C::NSLOT) * SLOT_STEP,
+      issue_pv<D, FP8>(t_o, tmem + C::s_col(x, b) + C::P_OFF, v_d0 + (vi % C::NSLOT) * SLOT_STEP,
                        j > 0 ? 1u : 0u);
       ptx::mma_commit_elect(bar.pv_done(x));
       release(vi, x == 1 && j >= w.n0);
       if (j == nx - 1) ptx::mma_commit_elect(bar.o_full(x));
-      if (j + 2 < nx) {
-        const uint32_t ki = kv_base + 2 * (j + 2);  // K_{j+2}
+      if (j + C::NBUF < nx) {
+        const uint32_t ki = kv_base + 2 * (j + C::NBUF);  // K_{j+NBUF}, into P(j)'s buffer
         if (!wait_slot(ki)) { ok = false; break; }
         ptx::tc_fence_after();
-        scores(w, nx, j + 2, ki);
+        scores(w, nx, j + C::NBUF, ki);
       }
     }
     if (!ok) break;
@@ -585,13 +590,13 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
     float l = 0.f;           // running sum of the (unrounded, fp32) numerators
 
     for (int j = 0; j < nx; ++j) {
-      const int b = j & 1;
+      const int b = j % C::NBUF;
       bool ok = wait_phase(bar.s_full(x, b), (sph >> b) & 1u, abort_flag, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;
       sph ^= 1u << b;
       ptx::tc_fence_after();
 
-      const uint32_t t_s = tmem + lane_base + s_col(x, b);
+      const uint32_t t_s = tmem + lane_base + C::s_col(x, b);
       uint32_t sr[4][16];
 #pragma unroll
       for (int c = 0; c < 4; ++c) ptx::tmem_ld16(t_s + c * 16, sr[c]);
@@ -769,7 +774,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::mbar_init(bar.q_full(), 1);
     ptx::mbar_init(bar.q_empty(), C::NT);
     for (int x = 0; x < 2; ++x) {
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < C::NBUF; ++b) {
         ptx::mbar_init(bar.s_full(x, b), 1);
         ptx::mbar_init(bar.p_full(x, b), BM);
       }
