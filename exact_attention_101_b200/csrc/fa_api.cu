@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <map>
+#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -119,9 +120,31 @@ bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_
   return r == CUDA_SUCCESS;
 }
 
+// The next slot of the forward kernel's work counters (fa::g_fa_sched) on device `dev`,
+// round-robin over the slots: launches in flight at the same time get different slots as
+// long as fewer than SCHED_SLOTS of them are.  The slots start at zero (static device
+// memory) and every launch leaves its slot at zero.
+fa_status sched_slot(int dev, unsigned int **out) {
+  static std::once_flag once[kMaxDevices];
+  static unsigned int *base[kMaxDevices];
+  static fa_status st[kMaxDevices];
+  static std::atomic<uint32_t> cursor[kMaxDevices];
+  std::call_once(once[dev], [&] {
+    void *a = nullptr;
+    st[dev] = cudaGetSymbolAddress(&a, fa::g_fa_sched) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    if (st[dev] != FA_OK) cudaGetLastError();
+    base[dev] = static_cast<unsigned int *>(a);
+  });
+  if (st[dev] != FA_OK) return st[dev];
+  *out = base[dev] + 2 * (cursor[dev].fetch_add(1u) % fa::SCHED_SLOTS);
+  return FA_OK;
+}
+
 template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN = false, bool DROPOUT = false>
 fa_status launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                 const fa::FwdParams &p, int grid, int dev, cudaStream_t stream) {
+                 const fa::FwdParams &params, int grid, int dev, cudaStream_t stream) {
+  fa::FwdParams p = params;
+  if (sched_slot(dev, &p.sched) != FA_OK) return FA_ERR_CUDA;
   using C = fa::TileCfg<D, FP8>;
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, OUT_F32, FP8, VARLEN, DROPOUT>;
   static std::once_flag attr_once[kMaxDevices];

@@ -110,6 +110,17 @@ constexpr uint32_t ERR_WAIT_DRAIN = 1u << 3;
 constexpr uint32_t ERR_WAIT_SELFTEST = 1u << 4;
 
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait
+
+// Work distribution: every CTA starts with unit blockIdx.x; after that its TMA warp claims
+// the next unit from a counter shared by the launch (one atomic per unit), so CTAs that
+// drew short units (causal, variable lengths) take more of them.  Each launch owns one
+// slot of g_fa_sched, chosen round-robin by the host: word 0 counts the units claimed,
+// word 1 the CTAs that have finished; the last CTA to finish sets both back to zero for
+// the slot's next launch.  (Launches that share a slot while both are in flight would
+// share the counter: the host cycles through SCHED_SLOTS slots per device.)
+constexpr int SCHED_SLOTS = 4096;
+__device__ unsigned int g_fa_sched[SCHED_SLOTS][2];
+constexpr int UNIT_RING = 4;  // units the TMA warp publishes ahead to the consumer warps
 constexpr uint32_t WAIT_MAX_ITERS = 1u << 28;
 
 template <int D, bool FP8>
@@ -146,9 +157,10 @@ struct TileCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NT * Q_TILE_BYTES;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * KV_TILE_BYTES;
-  static constexpr int NUM_BARS = 2 * NSLOT + 22;
+  static constexpr int NUM_BARS = 2 * NSLOT + 22 + 2 * UNIT_RING;
   static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
+  // control words: TMEM base, abort flag, 2 spare, then the ring of published units
+  static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16 + 4 * UNIT_RING;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -173,6 +185,7 @@ struct FwdParams {
   uint64_t seed, offset;
   uint32_t drop_thr4;  // drop_thr in every byte
   float keep_scale;
+  unsigned int *sched;  // this launch's slot of g_fa_sched (two words, zero at launch)
 };
 
 struct Unit {
@@ -287,23 +300,62 @@ struct Bars {
   __device__ uint32_t o_full(int x) const { return base + 8u * (2 * NSLOT + 16 + x); }
   __device__ uint32_t o_empty(int x) const { return base + 8u * (2 * NSLOT + 18 + x); }
   __device__ uint32_t drain(int x) const { return base + 8u * (2 * NSLOT + 20 + x); }
+  // ring of published work units: written (full) by the TMA warp, read (empty) by the
+  // MMA and softmax warps
+  __device__ uint32_t unit_full(int s) const { return base + 8u * (2 * NSLOT + 22 + s); }
+  __device__ uint32_t unit_empty(int s) const {
+    return base + 8u * (2 * NSLOT + 22 + UNIT_RING + s);
+  }
 };
+
+// The next work unit for a consumer warp (all 32 lanes): the one the TMA warp published
+// at ring position `taken`; a value >= num_units ends the list.  False if the wait was
+// aborted or ran out.
+template <int NSLOT>
+__device__ __forceinline__ bool take_unit(const Bars<NSLOT> &bar, volatile uint32_t *ring,
+                                          uint32_t &taken, volatile uint32_t *abort_flag,
+                                          uint32_t who, uint32_t &u) {
+  const int s = taken % UNIT_RING;
+  const bool ok = wait_phase(bar.unit_full(s), (taken / UNIT_RING) & 1u, abort_flag, who);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+  u = ring[s];
+  __syncwarp();
+  ptx::mbar_arrive_elect(bar.unit_empty(s));
+  ++taken;
+  return true;
+}
 
 // ---------------------------------------------------------------------------- producer
 
 template <int D, bool CAUSAL, bool FP8, bool VARLEN>
 __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                           const FwdParams &p, uint32_t smem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
-                          volatile uint32_t *abort_flag) {
+                          volatile uint32_t *unit_ring, volatile uint32_t *abort_flag) {
   using C = TileCfg<D, FP8>;
   ptx::prefetch_tmap(tmQ);
   ptx::prefetch_tmap(tmK);
   ptx::prefetch_tmap(tmV);
-  uint32_t issued = 0;    // K/V slot loads issued so far
-  uint32_t q_issued = 0;  // Q loads issued so far
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, u);
-    if (VARLEN && w.empty) continue;
+  uint32_t issued = 0;     // K/V slot loads issued so far
+  uint32_t q_issued = 0;   // Q loads issued so far
+  uint32_t published = 0;  // units published to the consumer warps
+  const uint32_t num_units = static_cast<uint32_t>(p.num_units);
+  auto claim = [&]() { return gridDim.x + atomicAdd(p.sched, 1u); };
+  for (uint32_t u = blockIdx.x;; u = claim()) {
+    Unit w;
+    if (u < num_units) {
+      w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, static_cast<int>(u));
+      if (VARLEN && w.empty) continue;  // past the end of its sequence: never published
+    }
+    {  // publish u (or, past the last unit, the end of the list)
+      const int s = published % UNIT_RING;
+      if (!wait_phase(bar.unit_empty(s), ((published / UNIT_RING) & 1u) ^ 1u, abort_flag,
+                      ERR_WAIT_LOAD))
+        goto drain;
+      unit_ring[s] = u;
+      ptx::mbar_arrive(bar.unit_full(s));
+      ++published;
+    }
+    if (u >= num_units) break;
     if (!wait_phase(bar.q_empty(), (q_issued & 1u) ^ 1u, abort_flag, ERR_WAIT_LOAD)) goto drain;
     ptx::mbar_arrive_expect_tx(bar.q_full(), C::NT * C::Q_TILE_BYTES);
 #pragma unroll
@@ -395,7 +447,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint6
 template <int D, bool CAUSAL, bool FP8, bool VARLEN>
 __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
                          const Bars<TileCfg<D, FP8>::NSLOT> &bar, const int x,
-                         volatile uint32_t *abort_flag) {
+                         volatile uint32_t *unit_ring, volatile uint32_t *abort_flag) {
   using C = TileCfg<D, FP8>;
   const uint64_t q_d = ptx::smem_desc_sw128(smem + C::Q_OFF + x * C::Q_TILE_BYTES, 16, 1024);
   const uint64_t k_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, 16, 1024);
@@ -423,9 +475,13 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
     release(ki, x == 1 && j >= w.n0);
     if (j == nx - 1) ptx::mma_commit_elect(bar.q_empty());
   };
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, u);
-    if (VARLEN && w.empty) continue;
+  uint32_t taken = 0;
+  for (;;) {
+    uint32_t u;
+    if (!take_unit(bar, unit_ring, taken, abort_flag, ERR_WAIT_MMA, u) ||
+        u >= static_cast<uint32_t>(p.num_units))
+      break;
+    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, static_cast<int>(u));
     const int nx = x ? w.n1 : w.n0;
     if (!wait(bar.q_full(), unit_it & 1u)) break;
     bool ok = true;
@@ -562,7 +618,7 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], 
 // row statistics are carried from tile to tile.
 template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN, bool DROPOUT>
 __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
-                             volatile uint32_t *abort_flag) {
+                             volatile uint32_t *unit_ring, volatile uint32_t *abort_flag) {
   using C = TileCfg<D, FP8>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int x = warp / 4;              // Q tile handled by this warpgroup
@@ -574,10 +630,14 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
   uint32_t sph = 0;      // phase bits of s_full(x, b), bit b
   uint32_t pv_base = 0;  // P.V products of this tile in earlier units
   uint32_t unit_it = 0;
+  uint32_t taken = 0;
 
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, u);
-    if (VARLEN && w.empty) continue;
+  for (;;) {
+    uint32_t u;
+    if (!take_unit(bar, unit_ring, taken, abort_flag, ERR_WAIT_SOFTMAX, u) ||
+        u >= static_cast<uint32_t>(p.num_units))
+      return;
+    const Unit w = decode_unit<CAUSAL, VARLEN, C::UNIT>(p, static_cast<int>(u));
     const int nx = x ? w.n1 : w.n0;
     const int row = w.r0 + x * BM + row_in_tile;     // query row of this thread
     const int tile_row0 = w.r0 + x * BM;
@@ -762,6 +822,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + C::CTL_OFF);
   volatile uint32_t *tmem_slot = ctl;
   volatile uint32_t *abort_flag = ctl + 1;
+  volatile uint32_t *unit_ring = ctl + 4;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -784,6 +845,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     ptx::mbar_init(bar.drain(0), 1);
     ptx::mbar_init(bar.drain(1), 1);
+    for (int s = 0; s < UNIT_RING; ++s) {
+      ptx::mbar_init(bar.unit_full(s), 1);
+      ptx::mbar_init(bar.unit_empty(s), 5 * C::NT);  // MMA warps + softmax warps
+    }
     *abort_flag = 0u;
     ptx::fence_mbar_init();
   }
@@ -802,12 +867,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::setmaxnreg_dec<OTHER_REGS>();
 
   if (warp < 4 * C::NT) {
-    softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN, DROPOUT>(p, tmem, bar, abort_flag);
+    softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN, DROPOUT>(p, tmem, bar, unit_ring, abort_flag);
   } else if (warp == MMA_WARP || (C::NT == 2 && warp == MMA_WARP + 2)) {
-    mma_role<D, CAUSAL, FP8, VARLEN>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, abort_flag);
+    mma_role<D, CAUSAL, FP8, VARLEN>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, unit_ring,
+                                     abort_flag);
     __syncwarp();
   } else if (warp == TMA_WARP) {
-    if (lane == 0) load_role<D, CAUSAL, FP8, VARLEN>(&tmQ, &tmK, &tmV, p, smem, bar, abort_flag);
+    if (lane == 0)
+      load_role<D, CAUSAL, FP8, VARLEN>(&tmQ, &tmK, &tmV, p, smem, bar, unit_ring, abort_flag);
     __syncwarp();
   }
 
@@ -816,6 +883,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == MMA_WARP) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
+  // every claim of this CTA is done (its TMA warp has left its loop): count the CTA out;
+  // the last one resets the launch's counters
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
   }
 }
 
