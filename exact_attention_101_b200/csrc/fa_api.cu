@@ -707,6 +707,7 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
                                      static_cast<long long>(rows_padded), Nq, p.Npad);
     if (cudaGetLastError() != cudaSuccess) st = FA_ERR_CUDA;
   }
+  if (st == FA_OK && sched_slot(dev, &p.sched) != FA_OK) st = FA_ERR_CUDA;
   if (st == FA_OK) {
     const int grid = p.num_units < info.sms ? p.num_units : info.sms;
     if (d == 64)

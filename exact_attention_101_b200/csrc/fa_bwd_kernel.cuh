@@ -68,7 +68,7 @@ constexpr int DS_TILE = BN * BM * 2;     // dS^T [keys][queries] bf16, 128-byte 
 constexpr int VEC_BYTES = 2 * BM * 4;    // per step: LSE*log2(e) and D for BM queries
 constexpr int QSTAGES = 3;               // ring of Q, dO and vector stages
 constexpr int DQ_STAGE = 32 * BM * 4;    // per drain warp: 64 queries x 32 head dims fp32
-constexpr int NUM_BARS = 2 + 2 * QSTAGES + 2 * 4 + 3;
+constexpr int NUM_BARS = 2 + 2 * QSTAGES + 2 * 4 + 3 + 2 * UNIT_RING;
 
 // Tensor-memory columns of the step buffers.
 __host__ __device__ constexpr uint32_t s_col(int b) { return b * 128; }
@@ -97,7 +97,8 @@ struct BCfg {
   static constexpr int VEC_OFF = DQS_OFF + DRAIN_WARPS * DQ_STAGE;
   static constexpr int BAR_OFF = VEC_OFF + QSTAGES * VEC_BYTES;
   static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16;
+  // control words: TMEM base, abort flag, 2 spare, then the ring of published units
+  static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16 + 4 * UNIT_RING;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // Tensor memory: step buffers at 0..255, dV at 256, dK after it.
   static constexpr uint32_t DV_COL = 256, DK_COL = 256 + D;
@@ -119,6 +120,7 @@ struct BwdParams {
   int num_kb;          // ceil(Nk / BN)
   int num_qb;          // ceil(Nq / BM)
   int num_units;       // B * Hkv * num_kb
+  unsigned int *sched; // this launch's work counters (see g_fa_sched)
   float scale_log2;    // scale * log2(e)
   float scale;
 };
@@ -170,6 +172,9 @@ struct BBars {
   __device__ uint32_t acc_full() const { return base + 8u * (B0 + 8); }
   __device__ uint32_t acc_empty() const { return base + 8u * (B0 + 9); }
   __device__ uint32_t drain() const { return base + 8u * (B0 + 10); }
+  // ring of published work units (TMA warp -> MMA, softmax and dQ warps)
+  __device__ uint32_t unit_full(int s) const { return base + 8u * (B0 + 11 + s); }
+  __device__ uint32_t unit_empty(int s) const { return base + 8u * (B0 + 11 + UNIT_RING + s); }
 };
 
 // ---------------------------------------------------------------------------- producer
@@ -177,15 +182,28 @@ struct BBars {
 template <int D, bool CAUSAL>
 __device__ void load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                           const CUtensorMap *tmDO, const BwdParams &p, uint32_t smem,
-                          const BBars &bar, volatile uint32_t *abort_flag) {
+                          const BBars &bar, volatile uint32_t *unit_ring,
+                          volatile uint32_t *abort_flag) {
   using C = BCfg<D>;
   ptx::prefetch_tmap(tmQ);
   ptx::prefetch_tmap(tmK);
   ptx::prefetch_tmap(tmV);
   ptx::prefetch_tmap(tmDO);
-  uint32_t units_issued = 0, steps_issued = 0;
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const BUnit w = decode_unit<CAUSAL>(p, u);
+  uint32_t units_issued = 0, steps_issued = 0, published = 0;
+  const uint32_t num_units = static_cast<uint32_t>(p.num_units);
+  // first unit blockIdx.x, then units claimed from the launch's counter (see the forward)
+  for (uint32_t u = blockIdx.x;; u = gridDim.x + atomicAdd(p.sched, 1u)) {
+    {  // publish u (or, past the last unit, the end of the list)
+      const int s = published % UNIT_RING;
+      if (!wait_phase(bar.unit_empty(s), ((published / UNIT_RING) & 1u) ^ 1u, abort_flag,
+                      ERR_WAIT_BWD))
+        goto drain;
+      unit_ring[s] = u;
+      ptx::mbar_arrive(bar.unit_full(s));
+      ++published;
+    }
+    if (u >= num_units) break;
+    const BUnit w = decode_unit<CAUSAL>(p, static_cast<int>(u));
     if (!wait_phase(bar.kv_empty(), (units_issued & 1u) ^ 1u, abort_flag, ERR_WAIT_BWD))
       goto drain;
     ptx::mbar_arrive_expect_tx(bar.kv_full(), 2 * C::KV_TILE);
@@ -275,7 +293,7 @@ __device__ __forceinline__ void issue_dq(uint32_t tmem_d, uint64_t a_desc, uint6
 
 template <int D, bool CAUSAL>
 __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const BBars &bar,
-                         volatile uint32_t *abort_flag) {
+                         volatile uint32_t *unit_ring, volatile uint32_t *abort_flag) {
   using C = BCfg<D>;
   const uint64_t k_a = ptx::smem_desc_sw128(smem + C::K_OFF, 16, 1024);
   const uint64_t v_a = ptx::smem_desc_sw128(smem + C::V_OFF, 16, 1024);
@@ -299,10 +317,14 @@ __device__ void mma_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const
     ptx::mma_commit_elect(bar.sdp_full(b));
     return true;
   };
-  uint32_t gm = 0, unit_it = 0;
+  uint32_t gm = 0, unit_it = 0, taken = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++unit_it) {
-    const BUnit w = decode_unit<CAUSAL>(p, u);
+  for (; ok; ++unit_it) {
+    uint32_t u;
+    if (!take_unit(bar, unit_ring, taken, abort_flag, ERR_WAIT_BWD, u) ||
+        u >= static_cast<uint32_t>(p.num_units))
+      break;
+    const BUnit w = decode_unit<CAUSAL>(p, static_cast<int>(u));
     if (!wait(bar.kv_full(), unit_it & 1u)) break;
     ptx::tc_fence_after();
     for (int s = 0; s < 2 && s < w.steps && ok; ++s) ok = start_step(gm + s);
@@ -406,15 +428,19 @@ __device__ __forceinline__ bool softmax_step(const BwdParams &p, uint32_t tmem_r
 
 template <int D, bool CAUSAL>
 __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, const BBars &bar,
-                             volatile uint32_t *abort_flag) {
+                             volatile uint32_t *unit_ring, volatile uint32_t *abort_flag) {
   using C = BCfg<D>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = warp / 4;                     // query half of the step
   const int row = (warp % 4) * 32 + lane;     // key row within the block
   const uint32_t tmem_row = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-  uint32_t gs = 0, unit_it = 0;
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++unit_it) {
-    const BUnit w = decode_unit<CAUSAL>(p, u);
+  uint32_t gs = 0, unit_it = 0, taken = 0;
+  for (;; ++unit_it) {
+    uint32_t u;
+    if (!take_unit(bar, unit_ring, taken, abort_flag, ERR_WAIT_BWD, u) ||
+        u >= static_cast<uint32_t>(p.num_units))
+      return;
+    const BUnit w = decode_unit<CAUSAL>(p, static_cast<int>(u));
     const int key = w.j * BN + row;
     for (int s = 0; s < w.steps; ++s) {
       const uint32_t g = gs + s;
@@ -471,7 +497,8 @@ __device__ void softmax_role(const BwdParams &p, uint32_t smem, uint32_t tmem, c
 // bulk tensor reduce-add.  Queries past Nq fall outside the tensor and are not written.
 template <int D, bool CAUSAL>
 __device__ void dq_role(const CUtensorMap *tmDQ, const BwdParams &p, uint32_t smem, uint32_t tmem,
-                        const BBars &bar, volatile uint32_t *abort_flag) {
+                        const BBars &bar, volatile uint32_t *unit_ring,
+                        volatile uint32_t *abort_flag) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int wq = warp % 4;
   const uint32_t tmem_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
@@ -481,10 +508,14 @@ __device__ void dq_role(const CUtensorMap *tmDQ, const BwdParams &p, uint32_t sm
   const bool owner = wq < C::DRAIN_WARPS;
   const uint32_t stage = smem + C::DQS_OFF + (owner ? wq : 0) * DQ_STAGE;
   if (lane == 0) ptx::prefetch_tmap(tmDQ);
-  uint32_t gd = 0;
+  uint32_t gd = 0, taken = 0;
   bool pending = false;
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-    const BUnit w = decode_unit<CAUSAL>(p, u);
+  for (;;) {
+    uint32_t u;
+    if (!take_unit(bar, unit_ring, taken, abort_flag, ERR_WAIT_BWD, u) ||
+        u >= static_cast<uint32_t>(p.num_units))
+      break;
+    const BUnit w = decode_unit<CAUSAL>(p, static_cast<int>(u));
     for (int s = 0; s < w.steps; ++s) {
       const uint32_t g = gd + s;
       const int b = g & 1u;
@@ -542,6 +573,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + C::CTL_OFF);
   volatile uint32_t *tmem_slot = ctl;
   volatile uint32_t *abort_flag = ctl + 1;
+  volatile uint32_t *unit_ring = ctl + 4;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
@@ -560,6 +592,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::mbar_init(bar.acc_full(), 1);
     ptx::mbar_init(bar.acc_empty(), 256);
     ptx::mbar_init(bar.drain(), 1);
+    for (int s = 0; s < UNIT_RING; ++s) {
+      ptx::mbar_init(bar.unit_full(s), 1);
+      ptx::mbar_init(bar.unit_empty(s), 13);  // MMA warp, 8 softmax warps, 4 dQ warps
+    }
     *abort_flag = 0u;
     ptx::fence_mbar_init();
   }
@@ -580,14 +616,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < DRAIN_WARP0) {
-    softmax_role<D, CAUSAL>(p, smem, tmem, bar, abort_flag);
+    softmax_role<D, CAUSAL>(p, smem, tmem, bar, unit_ring, abort_flag);
   } else if (warp < MMA_WARP) {
-    dq_role<D, CAUSAL>(&tmDQ, p, smem, tmem, bar, abort_flag);
+    dq_role<D, CAUSAL>(&tmDQ, p, smem, tmem, bar, unit_ring, abort_flag);
   } else if (warp == MMA_WARP) {
-    mma_role<D, CAUSAL>(p, smem, tmem, bar, abort_flag);
+    mma_role<D, CAUSAL>(p, smem, tmem, bar, unit_ring, abort_flag);
     __syncwarp();
   } else if (warp == TMA_WARP) {
-    if (lane == 0) load_role<D, CAUSAL>(&tmQ, &tmK, &tmV, &tmDO, p, smem, bar, abort_flag);
+    if (lane == 0)
+      load_role<D, CAUSAL>(&tmQ, &tmK, &tmV, &tmDO, p, smem, bar, unit_ring, abort_flag);
     __syncwarp();
   }
 
@@ -596,6 +633,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == MMA_WARP) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
+  // every claim of this CTA is done: count the CTA out; the last one resets the counters
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
   }
 }
 

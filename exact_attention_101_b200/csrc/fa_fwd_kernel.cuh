@@ -311,8 +311,8 @@ struct Bars {
 // The next work unit for a consumer warp (all 32 lanes): the one the TMA warp published
 // at ring position `taken`; a value >= num_units ends the list.  False if the wait was
 // aborted or ran out.
-template <int NSLOT>
-__device__ __forceinline__ bool take_unit(const Bars<NSLOT> &bar, volatile uint32_t *ring,
+template <class BarsT>
+__device__ __forceinline__ bool take_unit(const BarsT &bar, volatile uint32_t *ring,
                                           uint32_t &taken, volatile uint32_t *abort_flag,
                                           uint32_t who, uint32_t &u) {
   const int s = taken % UNIT_RING;
