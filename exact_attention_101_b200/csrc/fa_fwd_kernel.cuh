@@ -212,24 +212,27 @@ __device__ __forceinline__ int key_tiles(int last_row, int len_k, int off) {
   return last_key < 0 ? 1 : last_key / BN + 1;
 }
 
-// Work list: groups of HEAD_GROUP consecutive (batch, query head) pairs, so that the CTAs
-// running at the same time share the K/V of a few heads in L2 (and query heads that share
-// a K/V head are neighbours).  Inside a group the query blocks run last-first across its
-// heads: longest-first under the causal mask, so that the units claimed last, at the end
-// of the list, are short ones.  With variable lengths every sequence gets num_qb blocks
-// (those of the longest sequence); the blocks past the end of a shorter sequence are
-// empty and never published.
-constexpr int HEAD_GROUP = 8;
+// Work list: groups of consecutive (batch, query head) pairs, so that the CTAs running at
+// the same time share the K/V of a few heads in L2 (and query heads that share a K/V head
+// are neighbours).  Inside a group the query blocks run last-first across its heads.
+// Under the causal mask that is longest-first over CAUSAL_HEAD_GROUP heads, so that the
+// units claimed last, at the end of the list, are short ones.  Without the mask every
+// unit costs the same and a group is one head: fewer heads in flight read less K/V from
+// DRAM (8 heads of 8 MB each did not stay in L2).  With variable lengths every sequence
+// gets num_qb blocks (those of the longest sequence); the blocks past the end of a
+// shorter sequence are empty and never published.
+constexpr int CAUSAL_HEAD_GROUP = 8;
 
 template <bool CAUSAL, bool VARLEN, int UNIT = UNIT_ROWS>
 __device__ __forceinline__ Unit decode_unit(const FwdParams &p, int u) {
-  const int BH = p.num_units / p.num_qb;              // (batch, query head) pairs
-  const int g = u / (HEAD_GROUP * p.num_qb);           // head group
-  const int r = u - g * HEAD_GROUP * p.num_qb;
-  const int heads = min(HEAD_GROUP, BH - g * HEAD_GROUP);  // the last group may be smaller
+  constexpr int HG = CAUSAL ? CAUSAL_HEAD_GROUP : 1;
+  const int BH = p.num_units / p.num_qb;      // (batch, query head) pairs
+  const int g = u / (HG * p.num_qb);          // head group
+  const int r = u - g * HG * p.num_qb;
+  const int heads = min(HG, BH - g * HG);     // the last group may be smaller
   const int qb = p.num_qb - 1 - r / heads;
   Unit w;
-  w.bh = g * HEAD_GROUP + r % heads;
+  w.bh = g * HG + r % heads;
   const int b = w.bh / p.Hq, hq = w.bh % p.Hq;
   w.bhk = b * p.Hkv + hq / p.group;
   w.r0 = qb * UNIT;
