@@ -29,6 +29,13 @@
  * after a call returns and allocates no device memory, except fa_bwd, which allocates
  * and frees its scratch in stream order on the caller's stream (see there).
  *
+ * Work distribution: the forward and backward kernels run one persistent CTA per SM, and
+ * the CTAs claim work units from a counter of their launch.  The counters are 4096 pairs
+ * of 32-bit words per device in the library's static device memory.  Every launch takes
+ * the next pair (round-robin per device) and leaves it at zero when it ends.  So at most
+ * 4096 of these launches may be in flight on one device at the same time; more, on
+ * different streams, would share counters.
+ *
  * Execution: every call validates its arguments on the host first; on a validation error
  * it returns without touching the GPU.  Otherwise it enqueues its kernels on `stream`
  * and returns immediately (asynchronous).  A device-side wait that gave up (see
