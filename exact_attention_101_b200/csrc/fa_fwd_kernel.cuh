@@ -1,8 +1,9 @@
 // fa_fwd_kernel.cuh -- fused exact-attention forward kernel for B200 (sm_100a).
 //
-// One persistent CTA per SM walks a static list of work units.  A unit is 256 query
-// rows (two 128-row Q tiles) of one (batch, query head); the two tiles share every K/V
-// tile that is streamed through shared memory.  The method is the IO-aware tiled
+// One persistent CTA per SM claims work units from a list shared by the launch (see
+// "Work distribution" below).  A unit is 256 query rows (two 128-row Q tiles) of one
+// (batch, query head); the two tiles share every K/V tile that is streamed through
+// shared memory.  The method is the IO-aware tiled
 // attention of the page "FlashAttention (DE)" (sections "Tiling und blockweise
 // Verarbeitung", "Online-Softmax-Berechnung", "Zusammenfassen von Operationen in einem
 // CUDA-Kernel"): S = Q K^T, the mask, the online softmax and O += P V all happen on chip;
