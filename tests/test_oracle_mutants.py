@@ -242,6 +242,8 @@ MUTANTS = {
     "bwd_key_pass_top_left": ("if (causal && j > i + (Nk - Nq)) continue;",
                               "if (causal && j > i) continue;"),
     "bwd_query_pass_top_left": ("const int64_t last = i + (Nk - Nq);", "const int64_t last = i;"),
+    "bwd_row_without_keys_nonzero_dq": ("for (int64_t t = 0; t < d; ++t) dq[qoff + t] = 0.0;",
+                                        "for (int64_t t = 0; t < d; ++t) dq[qoff + t] = 1.0;"),
     "bwd_lse_without_sum": ("lse[gi] = m + log(l);", "lse[gi] = m;"),
     "bwd_dp_reads_k": ("dp[j] = dot_rows(dout, qoff, v, kvoff + j * d, elem_type, d);",
                        "dp[j] = dot_rows(dout, qoff, k, kvoff + j * d, elem_type, d);"),
