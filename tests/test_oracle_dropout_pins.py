@@ -55,18 +55,25 @@ def test_threshold_zero_is_plain_attention():
         assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
-@pytest.mark.parametrize("causal", [False, True])
-def test_bruteforce_with_numpy_bytes(causal):
-    B, H, N, d, thr, seed, off = 1, 2, 40, 3, 77, 2024, 3
-    q, k, v = rnd((B, H, N, d), 4), rnd((B, H, N, d), 5), rnd((B, H, N, d), 6)
+@pytest.mark.parametrize("causal,nq,nk", [(False, 40, 40), (True, 40, 40), (False, 25, 40),
+                                           (True, 25, 40), (True, 40, 25)])
+def test_bruteforce_with_numpy_bytes(causal, nq, nk):
+    """Causal masks align at the bottom right (key j admissible for query i iff
+    j <= i + nk - nq); a row without admissible keys has O = 0 and LSE = -inf."""
+    B, H, d, thr, seed, off = 1, 2, 3, 77, 2024, 3
+    q, k, v = rnd((B, H, nq, d), 4), rnd((B, H, nk, d), 5), rnd((B, H, nk, d), 6)
     o, lse = oracle.attention_dropout_rows(q, k, v, 0.5, causal, thr, seed, off)
-    o = o.reshape(B, H, N, d)
+    o, lse = o.reshape(B, H, nq, d), lse.reshape(B, H, nq)
     for h in range(H):
-        for i in range(N):
-            keys = range(i + 1) if causal else range(N)
+        for i in range(nq):
+            keys = range(max(0, min(nk, i + 1 + nk - nq))) if causal else range(nk)
+            if len(keys) == 0:
+                assert np.all(o[0, h, i] == 0.0) and np.isneginf(lse[0, h, i])
+                continue
             e = [math.exp(0.5 * math.fsum(q[0, h, i, t] * k[0, h, j, t] for t in range(d)))
                  for j in keys]
             z = math.fsum(e)
+            assert abs(lse[0, h, i] - math.log(z)) < 1e-12
             blocks = {}
             out = [0.0] * d
             for n, j in enumerate(keys):

@@ -176,15 +176,18 @@ def pin_philox_numpy(lib):
 def pin_dropout_bruteforce(lib):
     q, k, v = rnd((1, 2, 5, 3), 40), rnd((1, 2, 40, 3), 41), rnd((1, 2, 40, 3), 42)
     thr, seed, off = 90, 7, 1
-    o, _ = oracle.attention_dropout_rows(q, k, v, 0.5, False, thr, seed, off, _library=lib)
-    o = o.reshape(2, 5, 3)
-    for h in range(2):
-        for i in range(5):
-            e = np.exp(0.5 * (k[0, h] @ q[0, h, i]))
-            keep = np.array([((int(_np_block([j // 32, i, h, 0], [seed, off])[(j % 32) // 8])
-                               >> (8 * (j % 8))) & 0xFF) >= thr for j in range(40)])
-            ref = (e * keep) @ v[0, h] / e.sum() / (1 - thr / 256)
-            assert np.abs(o[h, i] - ref).max() < 1e-12
+    for causal in (False, True):   # causal: bottom-right, query i sees keys j <= i + 35
+        o, _ = oracle.attention_dropout_rows(q, k, v, 0.5, causal, thr, seed, off,
+                                             _library=lib)
+        o = o.reshape(2, 5, 3)
+        for h in range(2):
+            for i in range(5):
+                adm = np.arange(40) <= (i + 35 if causal else 39)
+                e = np.exp(0.5 * (k[0, h] @ q[0, h, i])) * adm
+                keep = np.array([((int(_np_block([j // 32, i, h, 0], [seed, off])[(j % 32) // 8])
+                                   >> (8 * (j % 8))) & 0xFF) >= thr for j in range(40)])
+                ref = (e * keep) @ v[0, h] / e.sum() / (1 - thr / 256)
+                assert np.abs(o[h, i] - ref).max() < 1e-12
 
 
 PINS = [pin_sdpa, pin_bruteforce_lse, pin_bottom_right, pin_gqa, pin_decoders, pin_e4m3_descales,
@@ -242,6 +245,9 @@ MUTANTS = {
     "bwd_key_pass_top_left": ("if (causal && j > i + (Nk - Nq)) continue;",
                               "if (causal && j > i) continue;"),
     "bwd_query_pass_top_left": ("const int64_t last = i + (Nk - Nq);", "const int64_t last = i;"),
+    "dropout_causal_top_left": (
+        "if (causal && i + 1 + (Nk - Nq) < n_adm) n_adm = i + 1 + (Nk - Nq);",
+        "if (causal && i + 1 < n_adm) n_adm = i + 1;"),
     "bwd_row_without_keys_nonzero_dq": ("for (int64_t t = 0; t < d; ++t) dq[qoff + t] = 0.0;",
                                         "for (int64_t t = 0; t < d; ++t) dq[qoff + t] = 1.0;"),
     "bwd_lse_without_sum": ("lse[gi] = m + log(l);", "lse[gi] = m;"),
