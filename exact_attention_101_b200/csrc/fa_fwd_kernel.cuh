@@ -23,19 +23,18 @@
 // useful K/V ring in shared memory, so a unit is one Q tile (NT = 1) and warps 4-7 and 10
 // stay idle.
 //
-// Key tiles are BN = 64 keys, and every Q tile has NBUF score buffers in tensor memory
-// (two; three at head dim 64, where the smaller O leaves room): while the softmax warps of
-// a tile turn S(j) into P(j), the tensor core already computes S(j+1) .. S(j+NBUF-1), and
-// S(j+NBUF) as soon as P(j) has been consumed.  So a tile's softmax never waits for its
-// own P.V product, and the two tiles' softmax warps -- one of each per SM sub-partition --
-// can both be busy at once.  This matters on B200 because, at head dim 128, the
+// Key tiles are BN = 64 keys, and every Q tile has NBUF = 2 score buffers in tensor
+// memory: while the softmax warps of a tile turn S(j) into P(j), the tensor core already
+// computes S(j+1), and S(j+2) as soon as P(j) has been consumed.  So a tile's softmax
+// never waits for its own P.V product, and the two tiles' softmax warps -- one of each
+// per SM sub-partition -- can both be busy at once.  This matters on B200 because, at head dim 128, the
 // exponentials of one score tile take the SFU as long as the tensor core takes for that
 // tile's two products.
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit), BN = 64:
 //   S(x, b) at x*NBUF*64 + b*64, 64 fp32 columns (tile x, buffer b); the numerators P of
 //   that buffer (bf16 pairs or e4m3 quads packed in 32-bit columns) overwrite its upper
-//   32 columns; O_x accumulator at O_COL0 + x*D (O_COL0 = 256, or 384 at head dim 64).
+//   32 columns; O_x accumulator at O_COL0 + x*D (O_COL0 = 256).
 //
 // Registers: the kernel is launched with LAUNCH_REGS per thread (384 threads); the third
 // warpgroup gives registers back (setmaxnreg.dec to OTHER_REGS) and the two softmax
@@ -145,10 +144,12 @@ struct TileCfg {
   static constexpr uint32_t AB_FORMAT = FP8 ? 0u : 1u;  // e4m3 : bf16
   static constexpr uint32_t IDESC_S = ptx::make_idesc(AB_FORMAT, BM, BN, 0);
   static constexpr uint32_t IDESC_O = ptx::make_idesc(AB_FORMAT, BM, D, 1);
-  // TMEM column map.  Score buffers per Q tile: three at D = 64 (tensor memory then holds
-  // 3 x 64 score columns and a 64-column O per tile), so that the scores run two products
-  // ahead of the softmax; two otherwise.
-  static constexpr int NBUF = (D == 64 && !FP8) ? 3 : 2;
+  // TMEM column map.  Two score buffers per Q tile.  (At D = 64 tensor memory would hold a
+  // third, but the rescale's wait for the previous P.V product is a parity wait on one
+  // pv_done barrier, exact only while at most one product is outstanding: with S(j)
+  // issued after P.V(j-2), at most P.V(j-1) is.  A third buffer would need one pv_done
+  // barrier per product parity.)
+  static constexpr int NBUF = 2;
   static constexpr uint32_t S_COLS = NBUF * 64;          // score columns of one Q tile
   __host__ __device__ static constexpr uint32_t s_col(int x, int b) { return x * S_COLS + b * 64; }
   static constexpr uint32_t P_OFF = 32;                  // P inside a 64-column S buffer

@@ -1,0 +1,167 @@
+"""A model of one Q tile's score buffers, P.V products and lazy rescaling in the forward
+kernel, run under random interleavings on the CPU.
+
+Per unit the tile visits nx key tiles j (buffer b = j % NBUF):
+- MMA warp (its products run on the tensor core in issue order; a commit arrives when
+  the products before it have finished): S(0) .. S(NBUF-1), each followed by a commit to
+  s_full(b); then per j: wait p_full(b) (parity from a per-buffer phase bit), at j = 0
+  wait o_empty, P.V(j) (reads P from buffer b, accumulates into O; j = 0 overwrites O),
+  commit pv_done, at the last j commit o_full, then S(j+NBUF) into buffer b.
+- softmax warps: per j wait s_full(b), read S(j); sometimes (data-dependent in the
+  kernel, random here) rescale O, which first waits pv_done with parity
+  (pv_base + j - 1) & 1, pv_base being the P.V products of earlier units, so that
+  P.V(j-1) and everything before it has finished; write P(j) into buffer b; arrive
+  p_full(b).  Per unit: wait o_full, read O, arrive o_empty.
+
+Every read checks what it needs when it happens: the softmax reads S(j); P.V(j) reads
+P(j); a rescale finds O holding exactly the products up to j-1 with none in flight; the
+epilogue finds all nx products; P.V(0) of the next unit runs only after the epilogue has
+read O.  Random schedules with NBUF 2 (the kernel's) must finish without a failed check or
+deadlock.  (Random schedules with NBUF 3 and this single pv_done barrier do fail: see
+the last test.)"""
+import random
+
+import pytest
+
+
+class MBarrier:
+    def __init__(self, count=1):
+        self.count, self.pending, self.phase = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        assert self.pending >= 0
+        if self.pending == 0:
+            self.phase ^= 1
+            self.pending = self.count
+
+    def try_wait(self, parity):
+        return self.phase != parity
+
+
+class Tile:
+    def __init__(self, units, nbuf, seed, rescale_p=0.3, mutant=None):
+        self.units, self.nbuf, self.mutant = units, nbuf, mutant
+        self.rng = random.Random(seed)
+        self.rescale_p = rescale_p
+        self.s_full = [MBarrier() for _ in range(nbuf)]
+        self.p_full = [MBarrier() for _ in range(nbuf)]
+        self.pv_done, self.o_full, self.o_empty = MBarrier(), MBarrier(), MBarrier()
+        self.buf = [None] * nbuf
+        self.o = None                  # (unit, products accumulated)
+        self.o_read = -1               # last unit whose O the epilogue has read
+        self.tc = []
+        self.agents = {"mma": self._mma(), "soft": self._softmax()}
+        self.waiting = {k: None for k in self.agents}
+        self.finished = set()
+
+    def _mma(self):
+        pph = 0
+        for u, nx in enumerate(self.units):
+            for j in range(min(self.nbuf, nx)):
+                self.tc += [("S", u, j), ("commit", self.s_full[j % self.nbuf])]
+            for j in range(nx):
+                b = j % self.nbuf
+                yield lambda b=b, ph=(pph >> b) & 1: self.p_full[b].try_wait(ph)
+                pph ^= 1 << b
+                if j == 0:
+                    yield lambda u=u: self.o_empty.try_wait((u & 1) ^ 1)
+                self.tc += [("PV", u, j), ("commit", self.pv_done)]
+                if j == nx - 1:
+                    self.tc.append(("commit", self.o_full))
+                if j + self.nbuf < nx:
+                    self.tc += [("S", u, j + self.nbuf), ("commit", self.s_full[b])]
+
+    def _softmax(self):
+        sph, pv_base = 0, 0
+        for u, nx in enumerate(self.units):
+            for j in range(nx):
+                b = j % self.nbuf
+                yield lambda b=b, ph=(sph >> b) & 1: self.s_full[b].try_wait(ph)
+                sph ^= 1 << b
+                assert self.buf[b] == ("S", u, j), ("softmax reads S", self.buf[b], u, j)
+                if j > 0 and self.rng.random() < self.rescale_p:
+                    parity = (pv_base + j - 1) & 1
+                    if self.mutant == "rescale_parity_off_by_one":
+                        parity = (pv_base + j) & 1
+                    if self.mutant != "rescale_without_wait":
+                        yield lambda p=parity: self.pv_done.try_wait(p)
+                    assert self.o == (u, j), ("rescale finds O", self.o, u, j)
+                    assert not any(op[0] == "PV" for op in self.tc), "a product in flight"
+                self.buf[b] = ("P", u, j)
+                self.p_full[b].arrive()
+            pv_base += nx
+            yield lambda u=u: self.o_full.try_wait(u & 1)
+            assert self.o == (u, nx), ("epilogue reads O", self.o, u, nx)
+            self.o_read = u
+            self.o_empty.arrive()
+
+    def _run(self):
+        op = self.tc.pop(0)
+        if op[0] == "commit":
+            op[1].arrive()
+            return
+        kind, u, j = op
+        b = j % self.nbuf
+        if kind == "S":
+            self.buf[b] = ("S", u, j)
+        else:
+            assert self.buf[b] == ("P", u, j), ("P.V reads P", self.buf[b], u, j)
+            if j == 0:
+                assert self.o_read == u - 1, "O overwritten before the epilogue read it"
+                self.o = (u, 1)
+            else:
+                assert self.o == (u, j), ("accumulation order", self.o, u, j)
+                self.o = (u, j + 1)
+
+    def run(self):
+        while len(self.finished) < len(self.agents) or self.tc:
+            moves = [("tc", None)] if self.tc else []
+            for k in self.agents:
+                if k not in self.finished and (self.waiting[k] is None or self.waiting[k]()):
+                    moves.append(("agent", k))
+            assert moves, "deadlock"
+            kind, k = self.rng.choice(moves)
+            if kind == "tc":
+                self._run()
+                continue
+            try:
+                self.waiting[k] = next(self.agents[k])
+            except StopIteration:
+                self.finished.add(k)
+                self.waiting[k] = None
+
+
+def mix(rng):
+    return [rng.randint(1, 9) for _ in range(rng.randint(1, 6))]
+
+
+def test_score_buffers_and_rescale_are_race_free():
+    """The kernel's configuration: two score buffers per Q tile."""
+    for seed in range(300):
+        Tile(mix(random.Random(seed)), 2, seed).run()
+
+
+def test_three_buffers_need_more_than_one_pv_done_barrier():
+    """With three buffers, S(j) follows P.V(j-3), so P.V(j-2) and P.V(j-1) can both be
+    outstanding when the softmax of step j rescales; pv_done is then two phases behind,
+    its parity matches the one awaited, and the wait returns early.  The model finds that
+    schedule, which is why the kernel keeps two buffers."""
+    caught = 0
+    for seed in range(100):
+        try:
+            Tile(mix(random.Random(seed)), 3, seed, rescale_p=0.5).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+@pytest.mark.parametrize("mutant", ["rescale_without_wait", "rescale_parity_off_by_one"])
+def test_model_catches_a_wrong_rescale_wait(mutant):
+    caught = 0
+    for seed in range(100):
+        try:
+            Tile(mix(random.Random(seed)), 2, seed, rescale_p=0.5, mutant=mutant).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, mutant
