@@ -40,13 +40,15 @@ class MBarrier:
 
 
 class Tile:
-    def __init__(self, units, nbuf, seed, rescale_p=0.3, mutant=None):
+    def __init__(self, units, nbuf, seed, rescale_p=0.3, mutant=None, pv_barriers=1):
         self.units, self.nbuf, self.mutant = units, nbuf, mutant
+        self.pv_barriers = pv_barriers  # 2: P.V product n commits to pv_done[n & 1]
         self.rng = random.Random(seed)
         self.rescale_p = rescale_p
         self.s_full = [MBarrier() for _ in range(nbuf)]
         self.p_full = [MBarrier() for _ in range(nbuf)]
-        self.pv_done, self.o_full, self.o_empty = MBarrier(), MBarrier(), MBarrier()
+        self.pv_done = [MBarrier() for _ in range(pv_barriers)]
+        self.o_full, self.o_empty = MBarrier(), MBarrier()
         self.buf = [None] * nbuf
         self.o = None                  # (unit, products accumulated)
         self.o_read = -1               # last unit whose O the epilogue has read
@@ -56,7 +58,7 @@ class Tile:
         self.finished = set()
 
     def _mma(self):
-        pph = 0
+        pph, pv_issued = 0, 0
         for u, nx in enumerate(self.units):
             for j in range(min(self.nbuf, nx)):
                 self.tc += [("S", u, j), ("commit", self.s_full[j % self.nbuf])]
@@ -66,7 +68,9 @@ class Tile:
                 pph ^= 1 << b
                 if j == 0:
                     yield lambda u=u: self.o_empty.try_wait((u & 1) ^ 1)
-                self.tc += [("PV", u, j), ("commit", self.pv_done)]
+                self.tc += [("PV", u, j),
+                            ("commit", self.pv_done[pv_issued % self.pv_barriers])]
+                pv_issued += 1
                 if j == nx - 1:
                     self.tc.append(("commit", self.o_full))
                 if j + self.nbuf < nx:
@@ -81,11 +85,13 @@ class Tile:
                 sph ^= 1 << b
                 assert self.buf[b] == ("S", u, j), ("softmax reads S", self.buf[b], u, j)
                 if j > 0 and self.rng.random() < self.rescale_p:
-                    parity = (pv_base + j - 1) & 1
+                    n = pv_base + j - 1            # the P.V product to wait for
                     if self.mutant == "rescale_parity_off_by_one":
-                        parity = (pv_base + j) & 1
+                        n += 1
+                    bar = self.pv_done[n % self.pv_barriers]
+                    parity = (n // self.pv_barriers) & 1
                     if self.mutant != "rescale_without_wait":
-                        yield lambda p=parity: self.pv_done.try_wait(p)
+                        yield lambda bar=bar, p=parity: bar.try_wait(p)
                     assert self.o == (u, j), ("rescale finds O", self.o, u, j)
                     assert not any(op[0] == "PV" for op in self.tc), "a product in flight"
                 self.buf[b] = ("P", u, j)
@@ -165,3 +171,12 @@ def test_model_catches_a_wrong_rescale_wait(mutant):
         except AssertionError:
             caught += 1
     assert caught > 0, mutant
+
+
+def test_three_buffers_with_a_pv_done_barrier_per_product_parity():
+    """The fix a third buffer would need: P.V product n commits to pv_done[n & 1] and the
+    rescale waits on pv_done[(n) & 1] with parity (n >> 1) & 1 for n = the previous
+    product.  Each barrier then has at most one product outstanding, and the model finds
+    no race."""
+    for seed in range(300):
+        Tile(mix(random.Random(seed)), 3, seed, rescale_p=0.5, pv_barriers=2).run()
