@@ -37,20 +37,21 @@ class MBarrier:
 
 
 class Model:
-    def __init__(self, units, nslot, nbuf, seed, tile0_arrive=True, release_at_issue=False):
-        self.units, self.nslot, self.nbuf = units, nslot, nbuf
+    def __init__(self, units, nslot, nbuf, seed, tile0_arrive=True, release_at_issue=False,
+                 nt=2):
+        self.units, self.nslot, self.nbuf, self.nt = units, nslot, nbuf, nt
         self.rng = random.Random(seed)
         self.slot_full = [MBarrier(1) for _ in range(nslot)]
-        self.slot_empty = [MBarrier(2) for _ in range(nslot)]
-        self.q_full, self.q_empty = MBarrier(1), MBarrier(2)
+        self.slot_empty = [MBarrier(nt) for _ in range(nslot)]   # one arrival per Q tile
+        self.q_full, self.q_empty = MBarrier(1), MBarrier(nt)
         self.content = [None] * nslot
         self.q_content = None
         self.tile0_arrive = tile0_arrive
         self.release_at_issue = release_at_issue
         self.loader = self._loader()
-        self.mma = [self._mma(x) for x in range(2)]
+        self.mma = [self._mma(x) for x in range(nt)]
         self.tc = [[], []]              # per warp: issued operations, retired in order
-        self.done = [False, False, False]
+        self.done = [False, nt < 2, False]     # a missing tile 1 counts as done
 
     # ---- agents are generators that yield a predicate to wait on, or None to move on
     def _loader(self):
@@ -118,7 +119,9 @@ class Model:
             rest[0].arrive()
 
     def run(self):
-        gens = {"load": self.loader, "mma0": self.mma[0], "mma1": self.mma[1]}
+        gens = {"load": self.loader, "mma0": self.mma[0]}
+        if self.nt == 2:
+            gens["mma1"] = self.mma[1]
         waiting = {k: None for k in gens}
         while not (all(self.done) and not self.tc[0] and not self.tc[1]):
             moves = []
@@ -182,3 +185,12 @@ def test_model_catches_a_release_before_the_product_ran():
         except AssertionError:
             caught += 1
     assert caught >= 30
+
+
+@pytest.mark.parametrize("nslot", [2, 4])
+def test_kv_ring_with_one_q_tile_per_unit(nslot):
+    """Head dim 256: one Q tile per unit (n0 = n1), one arrival per slot and per Q tile."""
+    for seed in range(40):
+        rng = random.Random(seed)
+        units = [(n, n) for n in (rng.randint(1, 9) for _ in range(rng.randint(1, 6)))]
+        Model(units, nslot, 2, seed, nt=1).run()
