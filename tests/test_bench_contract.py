@@ -55,3 +55,18 @@ def test_warmup_below_three_is_rejected():
                           "reference", "--warmup", "2"], cwd=ROOT, capture_output=True,
                          text=True, timeout=120)
     assert res.returncode != 0 and "warmup" in res.stderr
+
+
+def test_traffic_is_reported_only_for_the_kernel_it_was_measured_on(monkeypatch):
+    """roofline.traffic comes from profiles/traffic.json only while the forward kernel's
+    source hash matches the hash stored with the capture; otherwise it is null."""
+    import io
+    import bench
+    stored = json.dumps({"long": {"kernel_source_sha": "abc", "dram_bytes_per_launch": 123}})
+    monkeypatch.setattr(bench, "open", lambda path, *a, **k: io.StringIO(stored),
+                        raising=False)
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "abc")
+    assert bench.profiled_traffic("long") == 123
+    assert bench.profiled_traffic("gpt2") is None
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "def")
+    assert bench.profiled_traffic("long") is None

@@ -6,6 +6,7 @@ while the real oracle passes them all.  The mistakes are planted on the CPU only
 temporary builds."""
 import math
 import os
+import shutil
 
 import numpy as np
 import pytest
@@ -270,19 +271,34 @@ MUTANTS = {
 }
 
 
-def _build_mutant(tmp_path, name, old, new):
+# Mutant builds go to a git-ignored directory inside the repository, one per mutant,
+# removed after the test.
+BUILD_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), ".mutant_build")
+
+
+@pytest.fixture
+def build_dir(request):
+    path = os.path.join(BUILD_DIR, request.node.callspec.id if hasattr(request.node,
+                                                                       "callspec") else "x")
+    os.makedirs(path, exist_ok=True)
+    yield path
+    shutil.rmtree(path, ignore_errors=True)
+
+
+def _build_mutant(build_dir, name, old, new):
     hits = [src for src in SOURCES if open(src).read().count(old) == 1]
     assert len(hits) == 1 and sum(open(src).read().count(old) for src in SOURCES) == 1, \
         "mutation anchor not found exactly once: %s" % name
     sources = []
     for src in SOURCES:
         text = open(src).read()
-        path = tmp_path / os.path.basename(src)
-        path.write_text(text.replace(old, new) if src == hits[0] else text)
-        sources.append(str(path))
-    lib = tmp_path / ("lib" + name + ".so")
-    oracle_build.compile_library(str(lib), sources, opt="-O1")
-    return oracle.load_library(str(lib))
+        path = os.path.join(build_dir, os.path.basename(src))
+        with open(path, "w") as f:
+            f.write(text.replace(old, new) if src == hits[0] else text)
+        sources.append(path)
+    lib = os.path.join(build_dir, "lib" + name + ".so")
+    oracle_build.compile_library(lib, sources, opt="-O1")
+    return oracle.load_library(lib)
 
 
 def test_real_oracle_passes_every_compact_pin():
@@ -291,8 +307,8 @@ def test_real_oracle_passes_every_compact_pin():
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_every_planted_mistake_is_caught(tmp_path, name):
-    lib = _build_mutant(tmp_path, name, *MUTANTS[name])
+def test_every_planted_mistake_is_caught(build_dir, name):
+    lib = _build_mutant(build_dir, name, *MUTANTS[name])
     failed = []
     for pin in PINS:
         try:
