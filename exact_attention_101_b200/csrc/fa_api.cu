@@ -589,10 +589,14 @@ fa_status check_bwd_args(const void *q, const void *k, const void *v, const void
 }
 
 // Bytes of backward scratch: the fp32 dQ accumulator and two padded per-row vectors,
-// each rounded up to 256 bytes.
-uint64_t bwd_scratch_bytes(int B, int Hq, int Nq, int d, uint64_t *acc_bytes, uint64_t *vec_bytes) {
+// each rounded up to 256 bytes.  *acc_used is the accumulator's own size (before the
+// rounding): the bytes every call clears.
+uint64_t bwd_scratch_bytes(int B, int Hq, int Nq, int d, uint64_t *acc_bytes, uint64_t *vec_bytes,
+                           uint64_t *acc_used = nullptr) {
   const uint64_t npad = (static_cast<uint64_t>(Nq) + fa::bwd::BM - 1) / fa::bwd::BM * fa::bwd::BM;
-  *acc_bytes = (static_cast<uint64_t>(B) * Hq * Nq * d * 4 + 255) / 256 * 256;
+  const uint64_t used = static_cast<uint64_t>(B) * Hq * Nq * d * 4;
+  if (acc_used) *acc_used = used;
+  *acc_bytes = (used + 255) / 256 * 256;
   *vec_bytes = (static_cast<uint64_t>(B) * Hq * npad * 4 + 255) / 256 * 256;
   return *acc_bytes + 2 * *vec_bytes;
 }
@@ -679,8 +683,8 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
   // Scratch, stream-ordered: the fp32 dQ accumulator and the padded per-row LSE * log2(e)
   // and D arrays.
   const uint64_t rows_padded = static_cast<uint64_t>(B) * Hq * p.Npad;
-  uint64_t acc_bytes = 0, vec_bytes = 0;
-  const uint64_t ws_bytes = bwd_scratch_bytes(B, Hq, Nq, d, &acc_bytes, &vec_bytes);
+  uint64_t acc_bytes = 0, vec_bytes = 0, acc_used = 0;
+  const uint64_t ws_bytes = bwd_scratch_bytes(B, Hq, Nq, d, &acc_bytes, &vec_bytes, &acc_used);
   void *ws = fixed_ws;
   if (ws == nullptr) {
     cudaMemPool_t pool;
@@ -696,7 +700,7 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
   CUtensorMap tdq;
   st = encode_tmap_dq(&tdq, dq_acc, d, Nq, static_cast<uint64_t>(B) * Hq) ? FA_OK
                                                                            : FA_ERR_INVALID_ARG;
-  if (st == FA_OK && cudaMemsetAsync(dq_acc, 0, q_bytes * 2, stream) != cudaSuccess)
+  if (st == FA_OK && cudaMemsetAsync(dq_acc, 0, acc_used, stream) != cudaSuccess)
     st = FA_ERR_CUDA;
   if (st == FA_OK) {
     const unsigned blocks = static_cast<unsigned>((rows_padded + 7) / 8);
@@ -718,7 +722,7 @@ fa_status bwd_common(const void *q, const void *k, const void *v, const void *o,
                   : bwd_launch<128, false>(tq, tk, tv, tdo, tdq, p, grid, dev, stream);
   }
   if (st == FA_OK) {
-    const long long n4 = static_cast<long long>(q_bytes / 2 / 4);
+    const long long n4 = static_cast<long long>(acc_used / 16);  // float4 groups of dQ
     fa::bwd::fa_bwd_dq_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
         dq_acc, static_cast<uint16_t *>(dq), n4, scale);
     if (cudaGetLastError() != cudaSuccess) st = FA_ERR_CUDA;

@@ -26,15 +26,22 @@
  * LSE = -inf.
  *
  * Ownership: the caller allocates and owns every buffer.  The library keeps no pointer
- * after a call returns and allocates no device memory, except fa_bwd, which allocates
- * and frees its scratch in stream order on the caller's stream (see there).
+ * after a call returns and allocates no device memory at call time, except fa_bwd, which
+ * allocates and frees its scratch in stream order on the caller's stream (see there).
+ * The library's static device memory -- the work counters below and fa_bwd_noalloc's
+ * fixed 64 MiB scratch -- is part of its kernels' module: it is resident on every device
+ * where the library's kernels are loaded, from the first call on that device until the
+ * process exits, whichever entry points are used.
  *
  * Work distribution: the forward and backward kernels run one persistent CTA per SM, and
  * the CTAs claim work units from a counter of their launch.  The counters are 4096 pairs
  * of 32-bit words per device in the library's static device memory.  Every launch takes
  * the next pair (round-robin per device) and leaves it at zero when it ends.  So at most
  * 4096 of these launches may be in flight on one device at the same time; more, on
- * different streams, would share counters.
+ * different streams, would share counters.  A launch captured into a CUDA graph keeps
+ * the pair it was given at capture for every replay: a replay must not run at the same
+ * time as any other call of this library on the same device (that call may hold the same
+ * pair), or units are skipped or computed twice.
  *
  * Execution: every call validates its arguments on the host first; on a validation error
  * it returns without touching the GPU.  Otherwise it enqueues its kernels on `stream`
@@ -235,9 +242,14 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, con
  * per call (a framework whose own caching allocator holds nearly all of the device's
  * memory, or a service that must keep a fixed footprint).  Arguments, results and errors
  * are those of fa_bwd, except for the scratch: instead of allocating it on `stream`, the
- * call uses one fixed 64 MiB buffer that the library holds per device.  A problem whose
- * scratch, B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes (each part rounded up to 256 bytes),
- * does not fit returns FA_ERR_UNSUPPORTED with nothing enqueued.  Calls on the same stream
+ * call uses one fixed 64 MiB buffer that the library holds per device.  The buffer is a
+ * static device array of the library's module, so those 64 MiB are taken on every device
+ * where the library's kernels are loaded, by any entry point, until the process exits.
+ * The first fa_bwd_noalloc call on a device looks up the buffer's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.  A problem
+ * whose scratch, B*Hq*(Nq*d + 2*ceil(Nq/64)*64) * 4 bytes (each part rounded up to 256
+ * bytes), does not fit returns FA_ERR_UNSUPPORTED with nothing enqueued.  Every call
+ * clears the dQ accumulator part of the buffer before using it.  Calls on the same stream
  * are ordered; calls that may overlap in time on the same device (other streams, other
  * host threads) share the buffer and race, so the caller must serialise them.
  */
@@ -268,8 +280,8 @@ fa_status fa_bwd_noalloc(const void *q, const void *k, const void *v, const void
  *   B, H, N  >= 1
  *   d        128 (the head dimension of fa_fwd_fp8)
  *
- * The call enqueues a memset of descale (used as the amax accumulator) and three kernels
- * on `stream`.  Returns FA_OK once enqueued; FA_ERR_INVALID_ARG (null, misaligned or
+ * The call enqueues one kernel on `stream` (the CTAs that share a slice combine their
+ * maxima on chip, so nothing is cleared beforehand).  Returns FA_OK once enqueued; FA_ERR_INVALID_ARG (null, misaligned or
  * undersized buffer, bad size) or FA_ERR_UNSUPPORTED (d != 128, GPU not sm_100) with
  * nothing enqueued; FA_ERR_CUDA if a launch failed.
  */
