@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa_b200.so")
 SOURCES = [os.path.join(CSRC, "fa_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_bwd_kernel.cuh",
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_fwd_pair.cuh", "fa_bwd_kernel.cuh",
                                                   "fa_quant.cuh", "sm100.cuh")] + [
     os.path.join(ROOT, "include", "fa_b200.h")]
 

@@ -19,6 +19,7 @@
 #include "fa_b200.h"
 #include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
+#include "fa_fwd_pair.cuh"
 #include "fa_quant.cuh"
 
 namespace {
@@ -29,11 +30,11 @@ using PFN_encodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint3
                                      const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                      const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-using PFN_addressRange = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+using PFN_pointerAttrs = CUresult (*)(unsigned int, CUpointer_attribute *, void **, CUdeviceptr);
 
 struct DriverFns {
   PFN_encodeTiled encode = nullptr;
-  PFN_addressRange range = nullptr;
+  PFN_pointerAttrs attrs = nullptr;
   bool ok = false;
 };
 
@@ -48,11 +49,11 @@ const DriverFns &driver_fns() {
         q == cudaDriverEntryPointSuccess)
       fns.encode = reinterpret_cast<PFN_encodeTiled>(fn);
     fn = nullptr;
-    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) ==
+    if (cudaGetDriverEntryPoint("cuPointerGetAttributes", &fn, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fns.range = reinterpret_cast<PFN_addressRange>(fn);
-    fns.ok = fns.encode && fns.range;
+      fns.attrs = reinterpret_cast<PFN_pointerAttrs>(fn);
+    fns.ok = fns.encode && fns.attrs;
   });
   return fns;
 }
@@ -85,28 +86,71 @@ fa_status device_info(int dev, DeviceInfo *out) {
   return FA_OK;
 }
 
-// Device or managed memory of device `dev`, and the allocation holding `p` extends at
-// least `bytes` past it.
+// Device memory of device `dev` (or managed memory), and the allocation holding `p`
+// extends at least `bytes` past it.  One driver query per buffer: memory type, managed
+// flag, device and the allocation's address range together.  (A pointer the driver does
+// not know gets zeroed attributes and is refused.)
 bool buffer_ok(const void *p, size_t bytes, int dev) {
-  cudaPointerAttributes a;
-  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
-  }
-  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return false;
-  if (a.type == cudaMemoryTypeDevice && a.device != dev) return false;
-  CUdeviceptr base = 0;
+  CUpointer_attribute which[5] = {CU_POINTER_ATTRIBUTE_MEMORY_TYPE, CU_POINTER_ATTRIBUTE_IS_MANAGED,
+                                  CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL,
+                                  CU_POINTER_ATTRIBUTE_RANGE_START_ADDR,
+                                  CU_POINTER_ATTRIBUTE_RANGE_SIZE};
+  unsigned int type = 0;
+  uint64_t managed = 0;  // written as a boolean of at most 4 bytes
+  int ordinal = -1;
+  CUdeviceptr start = 0;
   size_t size = 0;
-  if (driver_fns().range(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS)
+  void *data[5] = {&type, &managed, &ordinal, &start, &size};
+  if (driver_fns().attrs(5, which, data, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS)
     return false;
+  const bool is_managed = (managed & 0xffffffffull) != 0;
+  if (!is_managed && (type != CU_MEMORYTYPE_DEVICE || ordinal != dev)) return false;
+  if (size == 0) return false;
   const uint64_t end = static_cast<uint64_t>(reinterpret_cast<uintptr_t>(p)) + bytes;
-  return end <= static_cast<uint64_t>(base) + size;
+  return end <= static_cast<uint64_t>(start) + size;
+}
+
+// Tensor maps are pure functions of (address, shape, box, format): a call looks them up in
+// a small per-thread cache before encoding one, so repeated calls on the same buffers skip
+// the encoding.  The buffer checks above still run on every call.
+struct TmapKey {
+  const void *base;
+  uint64_t d, rows, heads;
+  uint32_t box_rows, kind;  // kind: 0 bf16 [heads, rows, d], 1 e4m3, 2 packed bf16, 3 fp32 dQ
+  bool operator==(const TmapKey &o) const {
+    return base == o.base && d == o.d && rows == o.rows && heads == o.heads &&
+           box_rows == o.box_rows && kind == o.kind;
+  }
+};
+struct TmapEntry {
+  CUtensorMap map;
+  TmapKey key;
+  bool valid;
+};
+constexpr int kTmapCache = 32;
+thread_local TmapEntry t_tmap_cache[kTmapCache];
+thread_local unsigned t_tmap_next = 0;
+
+template <class Encode>
+bool cached_tmap(CUtensorMap *m, const TmapKey &key, Encode encode) {
+  for (int i = 0; i < kTmapCache; ++i) {
+    if (t_tmap_cache[i].valid && t_tmap_cache[i].key == key) {
+      *m = t_tmap_cache[i].map;
+      return true;
+    }
+  }
+  if (!encode(m)) return false;
+  TmapEntry &e = t_tmap_cache[t_tmap_next++ % kTmapCache];
+  e.map = *m;
+  e.key = key;
+  e.valid = true;
+  return true;
 }
 
 // 3-D tensor map over a [heads, rows, d] tensor, box = [1, box_rows, 128 bytes of d],
 // 128-byte swizzle, out-of-bounds elements read as zero.
-bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_t rows,
-                 uint64_t heads, uint32_t box_rows) {
+bool encode_tmap_now(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_t rows,
+                     uint64_t heads, uint32_t box_rows) {
   const uint64_t eb = fp8 ? 1 : 2;
   cuuint64_t dims[3] = {d, rows, heads};
   cuuint64_t strides[2] = {d * eb, rows * d * eb};
@@ -118,6 +162,14 @@ bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_
       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap(CUtensorMap *m, const void *base, bool fp8, uint64_t d, uint64_t rows,
+                 uint64_t heads, uint32_t box_rows) {
+  const TmapKey key{base, d, rows, heads, box_rows, fp8 ? 1u : 0u};
+  return cached_tmap(m, key, [&](CUtensorMap *out) {
+    return encode_tmap_now(out, base, fp8, d, rows, heads, box_rows);
+  });
 }
 
 // The next slot of the forward kernel's work counters (fa::g_fa_sched) on device `dev`,
@@ -170,6 +222,95 @@ fa_status launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap
   if (attr_st[dev] != FA_OK) return attr_st[dev];
   kern<<<grid, fa::NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// The bf16 forward at head dimension 128 without dropout runs on CTA pairs
+// (fa_fwd_pair.cuh) unless the library is built with FA_NO_PAIR_KERNEL.
+bool pair_path(int d, bool fp8, int drop_thr) {
+#ifdef FA_NO_PAIR_KERNEL
+  (void)d; (void)fp8; (void)drop_thr;
+  return false;
+#else
+  return d == fa::pair::D && !fp8 && drop_thr == 0;
+#endif
+}
+
+// Query rows per work unit, and CTAs per unit, of the forward instance for (d, path).
+int fwd_unit_rows(int d, bool pair) {
+  return pair ? fa::pair::UNIT_ROWS : (d > 128 ? fa::BM : fa::UNIT_ROWS);
+}
+
+// Clusters of the pair kernel that fit on device `dev` at once (0 if none), asked once per
+// device and instance.
+template <bool CAUSAL, bool OUT_F32>
+fa_status pair_setup(int dev, int sms, int *clusters) {
+  auto kern = fa::pair::fa_fwd_pair_kernel<CAUSAL, OUT_F32>;
+  static std::once_flag once[kMaxDevices];
+  static fa_status st[kMaxDevices];
+  static int n[kMaxDevices];
+  std::call_once(once[dev], [&] {
+    st[dev] = FA_ERR_CUDA;
+    n[dev] = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::pair::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      return;
+    }
+    cudaFuncAttributes fa_attr;
+    if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess) {
+      cudaGetLastError();
+      return;
+    }
+    // setmaxnreg.inc would wait forever if the launch pool could not cover the split
+    if (fa_attr.numRegs * fa::pair::NUM_THREADS <
+        256 * fa::pair::SOFTMAX_REGS + 128 * fa::pair::OTHER_REGS) {
+      st[dev] = FA_ERR_UNSUPPORTED;
+      return;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2), 1, 1);
+    cfg.blockDim = dim3(fa::pair::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = fa::pair::SMEM_BYTES;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      return;
+    }
+    n[dev] = c;
+    st[dev] = FA_OK;
+  });
+  *clusters = n[dev];
+  return st[dev];
+}
+
+template <bool CAUSAL, bool OUT_F32>
+fa_status launch_pair(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                      const fa::FwdParams &params, int clusters, int dev, cudaStream_t stream) {
+  fa::FwdParams p = params;
+  if (sched_slot(dev, &p.sched) != FA_OK) return FA_ERR_CUDA;
+  const int n = p.num_units < clusters ? p.num_units : clusters;
+  fa::pair::fa_fwd_pair_kernel<CAUSAL, OUT_F32>
+      <<<2 * n, fa::pair::NUM_THREADS, fa::pair::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <bool CAUSAL, bool OUT_F32>
+fa_status run_pair(const void *q, const void *k, const void *v, int B, int Hq, int Hkv, int Nq,
+                   int Nk, fa::FwdParams &p, const DeviceInfo &info, int dev, cudaStream_t stream,
+                   bool *ran) {
+  *ran = false;
+  int clusters = 0;
+  const fa_status st = pair_setup<CAUSAL, OUT_F32>(dev, info.sms, &clusters);
+  if (st != FA_OK || clusters < 1) return FA_OK;  // not resident here: the one-CTA kernel runs
+  CUtensorMap tq, tk, tv;
+  if (!encode_tmap(&tq, q, false, fa::pair::D, Nq, static_cast<uint64_t>(B) * Hq, fa::pair::BM) ||
+      !encode_tmap(&tk, k, false, fa::pair::D, Nk, static_cast<uint64_t>(B) * Hkv, 64) ||
+      !encode_tmap(&tv, v, false, fa::pair::D, Nk, static_cast<uint64_t>(B) * Hkv, fa::pair::BN))
+    return FA_ERR_INVALID_ARG;
+  p.num_qb = (Nq + fa::pair::UNIT_ROWS - 1) / fa::pair::UNIT_ROWS;
+  p.num_units = B * Hq * p.num_qb;
+  *ran = true;
+  return launch_pair<CAUSAL, OUT_F32>(tq, tk, tv, p, clusters, dev, stream);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -239,12 +380,6 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
               !buffer_ok(dv, static_cast<size_t>(B) * Hkv * 4, dev)))
     return FA_ERR_INVALID_ARG;
 
-  CUtensorMap tq, tk, tv;
-  if (!encode_tmap(&tq, q, fp8, d, Nq, static_cast<uint64_t>(B) * Hq, fa::BM) ||
-      !encode_tmap(&tk, k, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::BN) ||
-      !encode_tmap(&tv, v, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::BN))
-    return FA_ERR_INVALID_ARG;
-
   fa::FwdParams p;
   p.o = o;
   p.lse = lse;
@@ -267,6 +402,24 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
   p.num_qb = (Nq + unit_rows - 1) / unit_rows;
   p.num_units = B * Hq * p.num_qb;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+
+  if (pair_path(d, fp8, drop_thr)) {
+    bool ran = false;
+    const fa_status ps =
+        causal ? (out_f32 ? run_pair<true, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
+                          : run_pair<true, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran))
+               : (out_f32 ? run_pair<false, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
+                          : run_pair<false, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran));
+    if (ran || ps != FA_OK) return ps;
+    p.num_qb = (Nq + unit_rows - 1) / unit_rows;
+    p.num_units = B * Hq * p.num_qb;
+  }
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_tmap(&tq, q, fp8, d, Nq, static_cast<uint64_t>(B) * Hq, fa::BM) ||
+      !encode_tmap(&tk, k, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::BN) ||
+      !encode_tmap(&tv, v, fp8, d, Nk, static_cast<uint64_t>(B) * Hkv, fa::BN))
+    return FA_ERR_INVALID_ARG;
   const int grid = p.num_units < info.sms ? p.num_units : info.sms;
 
   if (fp8) {
@@ -311,8 +464,8 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
 
 // 3-D tensor map over a packed [tokens, heads, d] bf16 tensor, box = [128 bytes of d,
 // 1 head, box_rows tokens], 128-byte swizzle: the same shared-memory tile as encode_tmap.
-bool encode_tmap_packed(CUtensorMap *m, const void *base, uint64_t d, uint64_t heads,
-                        uint64_t tokens, uint32_t box_rows) {
+bool encode_tmap_packed_now(CUtensorMap *m, const void *base, uint64_t d, uint64_t heads,
+                            uint64_t tokens, uint32_t box_rows) {
   cuuint64_t dims[3] = {d, heads, tokens};
   cuuint64_t strides[2] = {d * 2, heads * d * 2};
   cuuint32_t box[3] = {64, 1, box_rows};
@@ -322,6 +475,14 @@ bool encode_tmap_packed(CUtensorMap *m, const void *base, uint64_t d, uint64_t h
       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_packed(CUtensorMap *m, const void *base, uint64_t d, uint64_t heads,
+                        uint64_t tokens, uint32_t box_rows) {
+  const TmapKey key{base, d, tokens, heads, box_rows, 2u};
+  return cached_tmap(m, key, [&](CUtensorMap *out) {
+    return encode_tmap_packed_now(out, base, d, heads, tokens, box_rows);
+  });
 }
 
 fa_status fwd_varlen_common(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -846,9 +1007,10 @@ fa_status fwd_host(const void *qh, const void *kh, const void *vh, void *oh, flo
     DeviceInfo info;
     st = device_info(dev, &info);
     if (st != FA_OK) return st;
-    const uint64_t unit_rows = d > 128 ? fa::BM : fa::UNIT_ROWS;
+    const bool pair = pair_path(d, false, 0);
+    const uint64_t unit_rows = static_cast<uint64_t>(fwd_unit_rows(d, pair));
     const uint64_t group_units = g * ((static_cast<uint64_t>(Nq) + unit_rows - 1) / unit_rows);
-    per = static_cast<uint64_t>(info.sms) / group_units;
+    per = static_cast<uint64_t>(pair ? info.sms / 2 : info.sms) / group_units;
     if (per < 1) per = 1;
     n = (groups + per - 1) / per;
   }

@@ -1,0 +1,704 @@
+// fa_fwd_pair.cuh -- the bf16 head-dimension-128 attention forward on CTA pairs (sm_100a).
+//
+// Same method as fa_fwd_kernel.cuh (the IO-aware tiled attention of the page "FlashAttention
+// (DE)", sections "Tiling und blockweise Verarbeitung", "Online-Softmax-Berechnung" and
+// "Zusammenfassen von Operationen in einem CUDA-Kernel"; the warp roles of the page
+// "FlashAttention 4: Praxisleitfaden ...", section "Was ist neu in FlashAttention 4?"), laid
+// out for the tensor core's two-SM products.
+//
+// Why pairs.  A one-SM S = Q K^T product with M = 128 reads A (Q) and B (K) from shared
+// memory: at N = 64 keys that is 6 KB per 32 tensor-core cycles, above the 128 bytes per
+// cycle that shared memory delivers, so the one-SM kernel is bound by shared-memory
+// bandwidth (about 160 KB per 64-key step against 1024 tensor cycles).  A pair of CTAs on
+// two SMs issues tcgen05 products with M = 256 (.cta_group::2): each SM holds 128 rows of A
+// and half of B's N columns, and computes its own 128 rows of D.  With 128-key blocks a
+// K-step reads 4 KB of Q and 2 KB of K per SM for 64 cycles; V is split the same way, and
+// each CTA loads only its halves of K and V.  Per 128-key block an SM moves about 80 KB
+// through shared memory for 1024 tensor cycles.
+//
+// Geometry.  A cluster of two CTAs (ranks 0 and 1) processes a unit of 256 query rows of
+// one (batch, query head), rows [128 r, 128 r + 128) in CTA r (its 128 tensor-memory
+// lanes).  Keys come in blocks of BN = 128; CTA r holds keys [64 r, 64 r + 64) of every K
+// block (all 128 dimensions) and dimensions [64 r, 64 r + 64) of every V block (all 128
+// keys).  Per CTA:
+//
+//   warps 0-3   softmax of the even key blocks (key stream 0), and the epilogue of O's
+//               dimensions 0-63 (thread = query row = TMEM lane)
+//   warps 4-7   the odd key blocks (stream 1), and dimensions 64-127
+//   warp  8     tensor-memory allocator; in CTA 0 the MMA issuer
+//   warp  9     TMA producer (lane 0); in CTA 0 also the claimer of work units
+//   warps 10-11 idle (complete the third warpgroup)
+//
+// Two key streams.  At head dim 128 the exponentials of a block take the SFU as long as the
+// tensor core takes for the block's two products (16 exponentials and 16 x 512 MMA FLOPs
+// per SM per cycle), so the softmax must never wait for its scores and the two softmax
+// warps of an SM sub-partition must not hit the SFU in step.  Each warpgroup runs its own
+// online softmax over every other key block -- its own running maximum, row sum and O
+// accumulator -- so while one warpgroup exponentiates block j, the other loads block j+1
+// and the tensor core multiplies.  The two partial results are merged once per unit in
+// the epilogue, the same way blocks are merged inside a stream:
+//   m = max(m_0, m_1), O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1).
+//
+// Tensor memory (512 columns, allocated for the pair): score buffer S(s) of stream s at
+// s * 128 (128 fp32 columns, its bf16 numerators P over the first 64 once read), and the
+// accumulator O_s at 256 + s * 128.
+//
+// MMA order inside a unit (one warp of CTA 0): S(0), S(1), then for every block j:
+// P(j) V_j into O_(j mod 2), S(j+2) into P(j)'s buffer (tcgen05 operations of one thread run
+// in issue order, so the product reads P(j) before S(j+2) overwrites it).  The commit that
+// signals S(j) covers P(j-2) V, the last product into the stream's accumulator, so a lazy
+// rescale of O_s needs no other wait.
+//
+// Synchronisation.  Barriers sit at the same offsets in both CTAs.  Those the MMA warp waits
+// on live in CTA 0 (slot_full, q_full, p_full, o_empty, unit_empty): both CTAs' copies signal
+// CTA 0's slot_full/q_full (.cta_group::2 copies), and CTA 1's softmax warps arrive on CTA
+// 0's p_full/o_empty remotely.  Those the producers and softmax warps wait on are signalled
+// in both CTAs at once by the MMA commits (slot_empty, q_empty, s_full, o_full).  CTA 0's
+// producer claims units and writes each into both CTAs' unit rings.
+#pragma once
+
+#include "fa_fwd_kernel.cuh"
+
+namespace fa {
+namespace pair {
+
+constexpr int D = 128;
+constexpr int BM = 128;                     // query rows of a unit held by one CTA
+constexpr int BN = 128;                     // keys per block (N of S over the pair)
+constexpr int UNIT_ROWS = 2 * BM;           // query rows per unit (MMA M)
+constexpr int NUM_THREADS = 384;
+constexpr int MMA_WARP = 8;
+constexpr int TMA_WARP = 9;
+constexpr int LAUNCH_REGS = 168;
+constexpr int SOFTMAX_REGS = 208;
+constexpr int OTHER_REGS = (NUM_THREADS * LAUNCH_REGS - 256 * SOFTMAX_REGS) / 128 / 8 * 8;
+static_assert(OTHER_REGS >= 64, "register split leaves too few for the MMA/TMA warps");
+static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS <= NUM_THREADS * LAUNCH_REGS,
+              "register split exceeds the launch pool");
+#ifndef FA_PAIR_POLY_PAIRS
+#define FA_PAIR_POLY_PAIRS 0
+#endif
+// Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial instead of the
+// SFU, on blocks without masked entries.
+constexpr int POLY_PAIRS = FA_PAIR_POLY_PAIRS;
+static_assert(POLY_PAIRS >= 0 && POLY_PAIRS <= 8, "pairs per 16-column chunk");
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int Q_BOX_BYTES = BM * 128;       // 128 rows x 128 bytes (64 dims)
+constexpr int Q_TILE_BYTES = 2 * Q_BOX_BYTES;
+constexpr int K_BOX_BYTES = 64 * 128;       // 64 keys x 128 bytes
+constexpr int SLOT_BYTES = 16384;           // K half: 2 boxes; V half: 128 keys x 64 dims
+constexpr int NSLOT = 8;
+constexpr int S_KSTEPS = D / 16;
+constexpr int PV_KSTEPS = BN / 16;
+constexpr uint32_t IDESC_S = ptx::make_idesc(1u, 256, BN, 0);
+constexpr uint32_t IDESC_O = ptx::make_idesc(1u, 256, D, 1);
+constexpr uint32_t O_COL0 = 256;            // O_0; O_1 follows at O_COL0 + D
+constexpr int UNIT_RING_P = 4;
+// consumers of a published unit: CTA 0's MMA warp and eight softmax warps, CTA 1's eight
+// softmax warps and its producer
+constexpr uint32_t UNIT_CONSUMERS = 1 + 8 + 8 + 1;
+constexpr uint32_t SOFTMAX_WARPS_PAIR = 16;  // softmax warps of both CTAs (o_empty)
+constexpr uint16_t BOTH = 0x3;              // CTA mask of the pair
+
+// shared memory: two Q buffers (unit parity), the K/V ring, the exchange of the streams'
+// row statistics [2 unit parities][maximum, sum][2 streams][128 rows] (fp32), the mbarriers
+// and the control words
+constexpr int Q_OFF = 0;
+constexpr int RING_OFF = 2 * Q_TILE_BYTES;
+constexpr int XCH_OFF = RING_OFF + NSLOT * SLOT_BYTES;
+constexpr int XCH_BYTES = 2 * 2 * 2 * BM * 4;
+constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
+constexpr int NUM_BARS = 2 * NSLOT + 18 + 2 * UNIT_RING_P;
+constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
+// control words: TMEM base, abort flag, 2 spare, then the unit ring
+constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16 + 4 * UNIT_RING_P;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct PBars {
+  uint32_t base;
+  __device__ uint32_t slot_full(int s) const { return base + 8u * s; }
+  __device__ uint32_t slot_empty(int s) const { return base + 8u * (NSLOT + s); }
+  __device__ uint32_t q_full(int q) const { return base + 8u * (2 * NSLOT + q); }
+  __device__ uint32_t q_empty(int q) const { return base + 8u * (2 * NSLOT + 2 + q); }
+  __device__ uint32_t s_full(int b) const { return base + 8u * (2 * NSLOT + 4 + b); }
+  __device__ uint32_t p_full(int b) const { return base + 8u * (2 * NSLOT + 6 + b); }
+  __device__ uint32_t o_full() const { return base + 8u * (2 * NSLOT + 8); }
+  __device__ uint32_t o_empty() const { return base + 8u * (2 * NSLOT + 10); }
+  __device__ uint32_t drain() const { return base + 8u * (2 * NSLOT + 13); }
+  // row-statistics exchange of warp pair (wq, wq + 4), wq = 0..3
+  __device__ uint32_t xchg(int wq) const { return base + 8u * (2 * NSLOT + 14 + wq); }
+  __device__ uint32_t unit_full(int s) const { return base + 8u * (2 * NSLOT + 18 + s); }
+  __device__ uint32_t unit_empty(int s) const {
+    return base + 8u * (2 * NSLOT + 18 + UNIT_RING_P + s);
+  }
+};
+
+// The CTA's abort flag and its address in the peer CTA: a wait that gives up raises both,
+// so that the peer stops waiting for work this CTA will not do.
+struct Abort {
+  volatile uint32_t *flag;
+  uint32_t peer;  // shared::cluster address of the peer's flag
+};
+
+template <bool CLUSTER>
+__device__ __forceinline__ bool pwait_slow(uint32_t bar, uint32_t parity, const Abort &ab,
+                                           uint32_t who) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1; it < WAIT_MAX_ITERS; ++it) {
+    if (CLUSTER ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity))
+      return true;
+    if ((it & 255u) == 0) {
+      if (*ab.flag) return false;
+      if (ptx::globaltimer_ns() - t0 > WAIT_LIMIT_NS) break;
+    }
+  }
+  *ab.flag = 1u;
+  ptx::st_cluster_u32(ab.peer, 1u);
+  atomicOr(&g_fa_error, who);
+  return false;
+}
+
+// Bounded wait on a phase of one of this CTA's mbarriers.  The per-block handshakes use
+// the default (CTA-scope acquire) semantics: what they hand over is tensor memory or MMA
+// operands, ordered by tcgen05 fences and the async proxy.  The unit ring, whose value is
+// an ordinary shared-memory word written by the other CTA, waits with cluster-scope
+// acquire (CLUSTER).
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, const Abort &ab,
+                                      uint32_t who) {
+  if (CLUSTER ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity))
+    return true;
+  return pwait_slow<CLUSTER>(bar, parity, ab, who);
+}
+
+// Key blocks that query rows up to `last_row` visit (at least one; see key_tiles).
+template <bool CAUSAL>
+__device__ __forceinline__ int key_blocks(int last_row, int len_k, int off) {
+  const int last_key = CAUSAL ? min(len_k - 1, last_row + off) : len_k - 1;
+  return last_key < 0 ? 1 : last_key / BN + 1;
+}
+
+struct PUnit {
+  int bh;    // b * Hq + hq
+  int bhk;   // b * Hkv + hq / group
+  int r0;    // first query row of the unit
+  int off;   // causal diagonal: query i sees keys j <= i + off
+  int n;     // key blocks the unit visits
+};
+
+// Work list as in decode_unit: head by head without the mask; under the causal mask groups
+// of CAUSAL_HEAD_GROUP heads, longest units first.
+template <bool CAUSAL>
+__device__ __forceinline__ PUnit pair_decode(const FwdParams &p, int u) {
+  constexpr int HG = CAUSAL ? CAUSAL_HEAD_GROUP : 1;
+  const int BH = p.num_units / p.num_qb;
+  const int g = u / (HG * p.num_qb);
+  const int r = u - g * HG * p.num_qb;
+  const int heads = min(HG, BH - g * HG);
+  const int qb = p.num_qb - 1 - r / heads;
+  PUnit w;
+  w.bh = g * HG + r % heads;
+  const int b = w.bh / p.Hq, hq = w.bh % p.Hq;
+  w.bhk = b * p.Hkv + hq / p.group;
+  w.r0 = qb * UNIT_ROWS;
+  w.off = p.Nk - p.Nq;
+  w.n = key_blocks<CAUSAL>(w.r0 + UNIT_ROWS - 1, p.Nk, w.off);
+  return w;
+}
+
+// ---------------------------------------------------------------------------- producer
+
+// Lane 0 of warp 9 in both CTAs.  CTA 0 claims units (its first is its cluster index, then
+// one atomic per unit) and publishes each in both CTAs' rings; CTA 1 takes them from its
+// ring.  Each CTA copies its own 128 rows of Q (into the buffer of the unit's parity) and
+// its halves of every K and V block; all copies complete on CTA 0's barriers, which CTA 0
+// arms with the bytes of both.
+template <bool CAUSAL>
+__device__ void pair_load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                               const CUtensorMap *tmV, const FwdParams &p, uint32_t smem,
+                               const PBars &bar, volatile uint32_t *ring, const Abort &ab,
+                               uint32_t rank) {
+  ptx::prefetch_tmap(tmQ);
+  ptx::prefetch_tmap(tmK);
+  ptx::prefetch_tmap(tmV);
+  const uint32_t num_units = static_cast<uint32_t>(p.num_units);
+  uint32_t issued = 0, q_issued = 0, units = 0;
+  uint32_t u = ptx::cluster_id_x();
+  for (;;) {
+    const int s = units % UNIT_RING_P;
+    const uint32_t ph = (units / UNIT_RING_P) & 1u;
+    if (rank == 0) {  // publish u (or, past the last unit, the end of the list)
+      if (!pwait<true>(bar.unit_empty(s), ph ^ 1u, ab, ERR_WAIT_LOAD)) goto drain;
+      ring[s] = u;
+      ptx::st_cluster_u32(ptx::mapa(ptx::smem_addr(const_cast<uint32_t *>(ring + s)), 1), u);
+      ptx::mbar_arrive(bar.unit_full(s));
+      ptx::mbar_arrive_cluster(ptx::mapa(bar.unit_full(s), 1));
+    } else {
+      if (!pwait<true>(bar.unit_full(s), ph, ab, ERR_WAIT_LOAD)) goto drain;
+      u = ring[s];
+      ptx::mbar_arrive_cluster(ptx::mapa(bar.unit_empty(s), 0));
+    }
+    ++units;
+    if (u >= num_units) break;
+    {
+      const PUnit w = pair_decode<CAUSAL>(p, static_cast<int>(u));
+      const int qb = q_issued & 1;
+      if (!pwait(bar.q_empty(qb), ((q_issued >> 1) & 1u) ^ 1u, ab, ERR_WAIT_LOAD)) goto drain;
+      if (rank == 0) ptx::mbar_arrive_expect_tx(bar.q_full(qb), 2 * Q_TILE_BYTES);
+      const uint32_t qf = ptx::mapa(bar.q_full(qb), 0);
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx)
+        ptx::tma_load_3d_pair(smem + Q_OFF + qb * Q_TILE_BYTES + bx * Q_BOX_BYTES, tmQ, qf,
+                              bx * 64, w.r0 + static_cast<int>(rank) * BM, w.bh);
+      ++q_issued;
+      for (int j = 0; j < w.n; ++j) {
+        // K half: keys j*BN + 64 rank .. + 63, all dimensions (two 64-dimension boxes)
+        {
+          const int sl = issued % NSLOT;
+          if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
+            goto drain;
+          if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
+          const uint32_t sf = ptx::mapa(bar.slot_full(sl), 0);
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx)
+            ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES + bx * K_BOX_BYTES, tmK, sf,
+                                  bx * 64, j * BN + static_cast<int>(rank) * 64, w.bhk);
+          ++issued;
+        }
+        // V half: keys j*BN .. + 127, dimensions 64 rank .. + 63
+        {
+          const int sl = issued % NSLOT;
+          if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
+            goto drain;
+          if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
+          ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES, tmV,
+                                ptx::mapa(bar.slot_full(sl), 0), static_cast<int>(rank) * 64,
+                                j * BN, w.bhk);
+          ++issued;
+        }
+      }
+    }
+    if (rank == 0) u = ptx::num_clusters_x() + atomicAdd(p.sched, 1u);
+  }
+drain:
+  if (rank == 0) {
+    // every phase this CTA armed completes once both CTAs' copies have landed
+    for (int s = 0; s < NSLOT; ++s) {
+      if (issued > static_cast<uint32_t>(s)) {
+        const uint32_t last = s + NSLOT * ((issued - 1 - s) / NSLOT);
+        drain_wait(bar.slot_full(s), (last / NSLOT) & 1u);
+      }
+    }
+    for (uint32_t qb = 0; qb < 2; ++qb) {
+      if (q_issued > qb) {
+        const uint32_t last = qb + 2 * ((q_issued - 1 - qb) / 2);
+        drain_wait(bar.q_full(qb), (last >> 1) & 1u);
+      }
+    }
+  } else if (*ab.flag) {
+    // After an abort CTA 1 cannot see CTA 0's barriers: give copies it issued for phases
+    // CTA 0 never armed time to land before the CTAs leave (bounded, 200 us).
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 0; it < WAIT_MAX_ITERS && ptx::globaltimer_ns() - t0 < 200000ull; ++it) {
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- MMA issuer
+
+__device__ __forceinline__ void pair_issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
+#pragma unroll
+  for (int kk = 0; kk < S_KSTEPS; ++kk) {
+    const uint32_t kb = kk * 32;  // bytes along the head dimension
+    const uint32_t qoff = ((kb / 128) * Q_BOX_BYTES + (kb % 128)) >> 4;
+    const uint32_t koff = ((kb / 128) * K_BOX_BYTES + (kb % 128)) >> 4;
+    ptx::mma2_bf16_ss_elect(tmem_s, q_desc + qoff, k_desc + koff, IDESC_S, kk > 0 ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void pair_issue_pv(uint32_t tmem_o, uint32_t tmem_s, uint64_t v_desc,
+                                              uint32_t accumulate) {
+  // V half is [128 keys x 64 dims], dims contiguous: an MN-major B operand of one 128-byte
+  // swizzle atom across N; 16 key rows of 128 bytes per K-step.
+#pragma unroll
+  for (int kk = 0; kk < PV_KSTEPS; ++kk) {
+    const uint32_t off = (kk * 16 * 128) >> 4;
+    ptx::mma2_bf16_ts_elect(tmem_o, tmem_s + kk * 8, v_desc + off, IDESC_O,
+                            kk > 0 ? 1u : accumulate);
+  }
+}
+
+// Warp 8 of CTA 0.  Every commit that frees a resource or signals a result arrives on the
+// barrier in both CTAs.
+template <bool CAUSAL>
+__device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, const PBars &bar,
+                              volatile uint32_t *ring, const Abort &ab) {
+  const uint64_t q_d0 = ptx::smem_desc_sw128(smem + Q_OFF, 16, 1024);
+  const uint64_t k_d0 = ptx::smem_desc_sw128(smem + RING_OFF, 16, 1024);
+  const uint64_t v_d0 = ptx::smem_desc_sw128(smem + RING_OFF, SLOT_BYTES, 1024);
+  constexpr uint32_t SLOT_STEP = SLOT_BYTES >> 4;
+  constexpr uint32_t QBUF_STEP = Q_TILE_BYTES >> 4;
+  uint32_t kv_base = 0, pph = 0, unit_it = 0, taken = 0;
+  auto wait = [&](uint32_t b, uint32_t parity) {
+    const bool ok = pwait(b, parity, ab, ERR_WAIT_MMA);
+    return __all_sync(0xffffffffu, ok);
+  };
+  auto wait_slot = [&](uint32_t idx) {
+    return wait(bar.slot_full(idx % NSLOT), (idx / NSLOT) & 1u);
+  };
+  for (;;) {
+    const int s = taken % UNIT_RING_P;
+    if (!__all_sync(0xffffffffu, pwait<true>(bar.unit_full(s), (taken / UNIT_RING_P) & 1u, ab,
+                                             ERR_WAIT_MMA)))
+      break;
+    const uint32_t u = ring[s];
+    __syncwarp();
+    ptx::mbar_arrive_elect(bar.unit_empty(s));
+    ++taken;
+    if (u >= static_cast<uint32_t>(p.num_units)) break;
+    const PUnit w = pair_decode<CAUSAL>(p, static_cast<int>(u));
+    const int n = w.n;
+    const int qb = unit_it & 1;
+    const uint64_t q_d = q_d0 + qb * QBUF_STEP;
+    auto scores = [&](int j, uint32_t ki) {
+      pair_issue_s(tmem + (j & 1) * BN, q_d, k_d0 + (ki % NSLOT) * SLOT_STEP);
+      ptx::mma2_commit_mc_elect(bar.s_full(j & 1), BOTH);
+      ptx::mma2_commit_mc_elect(bar.slot_empty(ki % NSLOT), BOTH);
+      if (j == n - 1) ptx::mma2_commit_mc_elect(bar.q_empty(qb), BOTH);
+    };
+    if (!wait(bar.q_full(qb), (unit_it >> 1) & 1u)) break;
+    bool ok = true;
+    for (int j = 0; j < 2 && j < n; ++j) {
+      if (!wait_slot(kv_base + 2 * j)) { ok = false; break; }
+      ptx::tc_fence_after();
+      scores(j, kv_base + 2 * j);
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const int b = j & 1;  // key stream
+      const uint32_t vi = kv_base + 2 * j + 1;
+      if (!wait_slot(vi)) { ok = false; break; }
+      if (!wait(bar.p_full(b), (pph >> b) & 1u)) { ok = false; break; }
+      pph ^= 1u << b;
+      // the previous unit's epilogue has read both accumulators
+      if (j == 0 && !wait(bar.o_empty(), (unit_it & 1u) ^ 1u)) { ok = false; break; }
+      ptx::tc_fence_after();
+      pair_issue_pv(tmem + O_COL0 + b * D, tmem + b * BN, v_d0 + (vi % NSLOT) * SLOT_STEP,
+                    j >= 2 ? 1u : 0u);
+      ptx::mma2_commit_mc_elect(bar.slot_empty(vi % NSLOT), BOTH);
+      if (j == n - 1) ptx::mma2_commit_mc_elect(bar.o_full(), BOTH);
+      if (j + 2 < n) {
+        const uint32_t ki = kv_base + 2 * (j + 2);
+        if (!wait_slot(ki)) { ok = false; break; }
+        ptx::tc_fence_after();
+        scores(j + 2, ki);
+      }
+    }
+    if (!ok) break;
+    kv_base += 2 * n;
+    ++unit_it;
+  }
+  // every product this warp issued has finished before tensor memory is freed
+  ptx::mma2_commit_elect(bar.drain());
+  drain_wait(bar.drain(), 0);
+}
+
+// ---------------------------------------------------------------------------- softmax
+
+// A 128-score row (sr) -> bf16 numerators at t_p (64 columns); adds the sum of the
+// unrounded numerators to le.  NPOLY of every 8 column pairs use the FMA-pipe exponential.
+template <int NPOLY>
+__device__ __forceinline__ void pair_numerators(const uint32_t (&sr)[4][32], float sl2,
+                                                float neg_m, uint32_t t_p, float &le) {
+  const uint64_t scale2 = ptx::f2_pack(sl2, sl2);
+  const uint64_t bias2 = ptx::f2_pack(neg_m, neg_m);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const uint64_t xx = ptx::f2_fma(
+          ptx::f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, bias2);
+      float x0, x1, p0, p1;
+      ptx::f2_unpack(xx, x0, x1);
+      if (((e % 16) / 2) < NPOLY) {
+        exp2_poly_pair(x0, x1, p0, p1);
+      } else {
+        p0 = ptx::ex2(x0);
+        p1 = ptx::ex2(x1);
+      }
+      acc[(e / 2) & 3] = ptx::f2_add(acc[(e / 2) & 3], ptx::f2_pack(p0, p1));
+      pk[e / 2] = ptx::pack_bf16x2(p0, p1);
+    }
+    ptx::tmem_st16(t_p + c * 16, pk);
+  }
+  float a0, a1;
+  ptx::f2_unpack(ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])), a0, a1);
+  le += a0 + a1;
+}
+
+template <bool CAUSAL, bool OUT_F32>
+__device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars &bar,
+                                  volatile uint32_t *ring, const Abort &ab, uint32_t rank,
+                                  volatile float *xch) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = warp / 4;        // key stream (blocks j with j mod 2 == h); O dims [64 h, 64 h + 64)
+  const int wq = warp % 4;       // TMEM lane quarter
+  const int r_cta = wq * 32 + lane;  // row inside the CTA's 128
+  const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+  const uint32_t t_s = tmem + lane_base + h * BN;
+  const uint32_t t_o = tmem + lane_base + O_COL0;  // O_0; O_1 is D columns further
+  const uint32_t p_full_c = ptx::mapa(bar.p_full(h), 0);
+  const uint32_t o_empty_c = ptx::mapa(bar.o_empty(), 0);
+  const uint32_t xbar = bar.xchg(wq);
+
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  uint32_t sph = 0, xph = 0, unit_it = 0, taken = 0;
+
+  for (;;) {
+    uint32_t u;
+    {
+      const int s = taken % UNIT_RING_P;
+      const bool ok =
+          pwait<true>(bar.unit_full(s), (taken / UNIT_RING_P) & 1u, ab, ERR_WAIT_SOFTMAX);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      u = ring[s];
+      __syncwarp();
+      ptx::mbar_arrive_cluster_elect(ptx::mapa(bar.unit_empty(s), 0));
+      ++taken;
+    }
+    if (u >= static_cast<uint32_t>(p.num_units)) return;
+    const PUnit w = pair_decode<CAUSAL>(p, static_cast<int>(u));
+    const int row0 = w.r0 + static_cast<int>(rank) * BM;  // first row of this CTA
+    const int row = row0 + r_cta;
+    const float sl2 = p.scale_log2;
+    const int key_lim = CAUSAL ? min(row + w.off, p.Nk - 1) : p.Nk - 1;
+    float m_used = NEG_INF;  // this stream's running maximum (base-2 scaled domain)
+    float l = 0.f;           // this stream's row sum
+
+    for (int j = h; j < w.n; j += 2) {
+      bool ok = pwait(bar.s_full(h), sph, ab, ERR_WAIT_SOFTMAX);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      sph ^= 1u;
+      ptx::tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::tmem_ld32(t_s + c * 32, sr[c]);
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::reg_fence32(sr[c]);
+
+      const int kv0 = j * BN;
+      const bool need_mask = (CAUSAL && kv0 + BN - 1 > row0 + w.off) || (kv0 + BN > p.Nk);
+      if (need_mask) {
+        const int lim = key_lim - kv0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e > lim) sr[c][e] = __float_as_uint(NEG_INF);
+      }
+      float mx[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float m = ptx::max3(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]),
+                            __uint_as_float(sr[c][2]));
+#pragma unroll
+        for (int e = 3; e < 31; e += 2)
+          m = ptx::max3(m, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+        mx[c] = fmaxf(m, __uint_as_float(sr[c][31]));
+      }
+      const float xmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      const bool resc = xmax > m_used + RESCALE_THRESHOLD;
+      const float alpha = resc ? ptx::ex2(m_used - xmax) : 1.f;  // 0 on the stream's first block
+      if (__any_sync(0xffffffffu, resc && j >= 2)) {
+        // O_h is quiescent: the commit that signalled S(j) covered P(j-2) V
+        const uint32_t t_oh = t_o + h * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t o[16];
+          ptx::tmem_ld16(t_oh + c * 16, o);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence16(o);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          ptx::tmem_st16(t_oh + c * 16, o);
+        }
+      }
+      if (resc) {
+        l *= alpha;
+        m_used = xmax;
+      }
+      const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
+      float le = 0.f;
+      if (POLY_PAIRS == 0 || need_mask)
+        pair_numerators<0>(sr, sl2, neg_m, t_s, le);
+      else
+        pair_numerators<POLY_PAIRS>(sr, sl2, neg_m, t_s, le);
+      l += le;
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      ptx::mbar_arrive_remote_elect(p_full_c);
+    }
+
+    // Epilogue: merge the two streams, O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1) with
+    // a_s = 2^(m_s - m), m = max(m_0, m_1); LSE = ln 2 * (m + log2 l).  A stream without
+    // admissible keys for this row (l_s = 0: no block, or all masked) adds nothing; its
+    // accumulator may hold stale values and is not read into the result.
+    {
+      // [stream][row] maxima and sums of this unit's parity: a stream that finishes its next
+      // unit early cannot overwrite values its partner has not read yet
+      volatile float *xm = xch + (unit_it & 1) * 4 * BM;
+      volatile float *xl = xm + 2 * BM;
+      xm[h * BM + r_cta] = m_used;
+      xl[h * BM + r_cta] = l;
+      __syncwarp();
+      ptx::mbar_arrive_elect(xbar);
+      bool ok = pwait(xbar, xph, ab, ERR_WAIT_SOFTMAX);
+      xph ^= 1u;
+      if (!__all_sync(0xffffffffu, ok)) return;
+      const float m0 = xm[r_cta], m1 = xm[BM + r_cta];
+      const float l0 = xl[r_cta], l1 = xl[BM + r_cta];
+      const float m = fmaxf(m0, m1);
+      const float a0 = l0 > 0.f ? ptx::ex2(m0 - m) : 0.f;
+      const float a1 = l1 > 0.f ? ptx::ex2(m1 - m) : 0.f;
+      const float lt = a0 * l0 + a1 * l1;
+      ok = pwait(bar.o_full(), unit_it & 1u, ab, ERR_WAIT_SOFTMAX);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      ptx::tc_fence_after();
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float f0 = a0 * inv, f1 = a1 * inv;
+      const bool valid = row < p.Nq;
+      const size_t orow = static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t col = h * 64 + c * 32;
+        uint32_t a[32], bq[32];
+        ptx::tmem_ld32(t_o + col, a);
+        ptx::tmem_ld32(t_o + D + col, bq);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence32(a);
+        ptx::reg_fence32(bq);
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          v[e] = (f0 != 0.f ? __uint_as_float(a[e]) * f0 : 0.f) +
+                 (f1 != 0.f ? __uint_as_float(bq[e]) * f1 : 0.f);
+        if (valid) {
+          if (OUT_F32) {
+            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          } else {
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + col);
+            uint32_t hh[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) hh[e] = ptx::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
+          }
+        }
+      }
+      if (valid && h == 0)
+        p.lse[orow] = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994530942f : NEG_INF;
+      ptx::tc_fence_before();
+      __syncwarp();
+      ptx::mbar_arrive_remote_elect(o_empty_c);
+    }
+    ++unit_it;
+  }
+}
+
+// ---------------------------------------------------------------------------- kernel
+
+template <bool CAUSAL, bool OUT_F32>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_addr(smem_raw);
+  const uint32_t smem = (raw + 1023u) & ~1023u;  // 1024-aligned for 128-byte swizzle
+  uint8_t *smem_gen = smem_raw + (smem - raw);
+  const PBars bar{smem + BAR_OFF};
+  uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + CTL_OFF);
+  volatile uint32_t *tmem_slot = ctl;
+  volatile uint32_t *abort_flag = ctl + 1;
+  volatile uint32_t *ring = ctl + 4;
+  volatile float *xch = reinterpret_cast<volatile float *>(smem_gen + XCH_OFF);
+  const uint32_t rank = ptx::cluster_ctarank();
+  const Abort ab{abort_flag, ptx::mapa(ptx::smem_addr(ctl + 1), rank ^ 1u)};
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSLOT; ++s) {
+      ptx::mbar_init(bar.slot_full(s), 1);
+      ptx::mbar_init(bar.slot_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar.q_full(b), 1);
+      ptx::mbar_init(bar.q_empty(b), 1);
+      ptx::mbar_init(bar.s_full(b), 1);
+      ptx::mbar_init(bar.p_full(b), SOFTMAX_WARPS_PAIR / 2);  // one stream's warps, both CTAs
+    }
+    ptx::mbar_init(bar.o_full(), 1);
+    ptx::mbar_init(bar.o_empty(), SOFTMAX_WARPS_PAIR);
+    ptx::mbar_init(bar.drain(), 1);
+    for (int wq = 0; wq < 4; ++wq) ptx::mbar_init(bar.xchg(wq), 2);  // warps wq and wq + 4
+    for (int s = 0; s < UNIT_RING_P; ++s) {
+      ptx::mbar_init(bar.unit_full(s), 1);
+      ptx::mbar_init(bar.unit_empty(s), UNIT_CONSUMERS);
+    }
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+  }
+  if (warp == MMA_WARP) {
+    ptx::tmem_alloc_pair(ptx::smem_addr(ctl), TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  // both CTAs' barriers are initialised and the pair's tensor memory allocated before
+  // either CTA signals the other
+  ptx::tc_fence_before();
+  ptx::cluster_sync();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 8)
+    ptx::setmaxnreg_inc<SOFTMAX_REGS>();
+  else
+    ptx::setmaxnreg_dec<OTHER_REGS>();
+
+  if (warp < 8) {
+    pair_softmax_role<CAUSAL, OUT_F32>(p, tmem, bar, ring, ab, rank, xch);
+  } else if (rank == 0 && warp == MMA_WARP) {
+    pair_mma_role<CAUSAL>(p, smem, tmem, bar, ring, ab);
+    __syncwarp();
+  } else if (warp == TMA_WARP) {
+    if (lane == 0) pair_load_role<CAUSAL>(&tmQ, &tmK, &tmV, p, smem, bar, ring, ab, rank);
+    __syncwarp();
+  }
+
+  // neither CTA leaves (or frees the pair's tensor memory) while the other may still
+  // signal it or run products on it
+  ptx::tc_fence_before();
+  ptx::cluster_sync();
+  if (warp == MMA_WARP) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
+  }
+}
+
+}  // namespace pair
+}  // namespace fa

@@ -90,18 +90,28 @@ def test_varlen_fp32_output(cuda_ok):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_varlen_equal_lengths_equal_fixed_length_bits(cuda_ok, causal):
-    """Packed sequences of one length run the same tiles as the [B, H, N, d] path."""
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_varlen_equal_lengths_equal_fixed_length(cuda_ok, causal, d):
+    """Packed sequences of one length against the [B, H, N, d] path.  At head dims 64 and
+    256 both run the same tiles of the one-CTA kernel: equal bits.  At 128 the fixed-length
+    path runs the CTA-pair kernel (another summation order): equal within the bf16 bar."""
     dev = torch.device("cuda", 0)
-    B, H, N, d = 3, 4, 385, 128
+    B, H, N = 3, 4, 385
     q, k, v = (random_bf16((B, H, N, d), 400 + s) for s in range(3))
     o1, l1 = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal=causal, scale=D_SCALE[d])
     pk = lambda t: t.permute(0, 2, 1, 3).reshape(B * N, H, d).contiguous().to(dev)
     c = cu([N] * B).to(dev)
     o2, l2 = fa.forward_varlen(pk(q), pk(k), pk(v), c, c, N, causal=causal, scale=D_SCALE[d])
     torch.cuda.synchronize()
-    assert torch.equal(o1.permute(0, 2, 1, 3).reshape(B * N, H, d), o2)
-    assert torch.equal(l1.permute(1, 0, 2).reshape(H, B * N), l2)
+    o1 = o1.permute(0, 2, 1, 3).reshape(B * N, H, d)
+    l1 = l1.permute(1, 0, 2).reshape(H, B * N)
+    if d != 128:
+        assert torch.equal(o1, o2)
+        assert torch.equal(l1, l2)
+    else:
+        e = (o1.float() - o2.float()).abs()
+        assert e.max().item() <= 2e-2 and e.mean().item() <= 2e-3
+        assert (l1 - l2).abs().max().item() <= 1e-3
 
 
 @pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (129, 513), (513, 129), (1, 700)])
