@@ -31,30 +31,33 @@
 //
 // Two key streams.  At head dim 128 the exponentials of a block take the SFU as long as the
 // tensor core takes for the block's two products (16 exponentials and 16 x 512 MMA FLOPs
-// per SM per cycle), so the softmax must never wait for its scores and the two softmax
-// warps of an SM sub-partition must not hit the SFU in step.  Each warpgroup runs its own
-// online softmax over every other key block -- its own running maximum, row sum and O
-// accumulator -- so while one warpgroup exponentiates block j, the other loads block j+1
-// and the tensor core multiplies.  The two partial results are merged once per unit in
-// the epilogue, the same way blocks are merged inside a stream:
-//   m = max(m_0, m_1), O = (2^(m_0-m) O_0 + 2^(m_1-m) O_1) / (2^(m_0-m) l_0 + 2^(m_1-m) l_1).
+// per SM per cycle), and one warp's softmax of a 128-key block also waits on tensor-memory
+// loads and stores.  So the two softmax warpgroups take turns: warpgroup s handles the
+// blocks j with j mod 2 == s, full 128-key rows, while the other loads and exponentiates its
+// own block.  Both use one running maximum: block j's maximum in use is handed to block
+// j+1 through shared memory right after block j's row maximum is known (lazy rescaling: it
+// only moves when the block maximum exceeds it by more than RESCALE_THRESHOLD), so the
+// numerators of every block are relative to the maximum O holds.  Each warpgroup keeps its
+// own part of the row sum, brought to the final maximum and added in the epilogue.
 //
-// Tensor memory (512 columns, allocated for the pair): score buffer S(s) of stream s at
-// s * 128 (128 fp32 columns, its bf16 numerators P over the first 64 once read), and the
-// accumulator O_s at 256 + s * 128.
+// Tensor memory (512 columns, allocated for the pair): score buffers S(b) at b * 128 (128
+// fp32 columns), the accumulator O at 256, numerator buffers P(b) at 384 + b * 64 (bf16
+// pairs).  P does not overwrite S, so S(j+2) is computed into S(j mod 2) as soon as the
+// softmax has read S(j), while block j's numerators are still being formed: the softmax
+// then finds its next scores ready.
 //
-// MMA order inside a unit (one warp of CTA 0): S(0), S(1), then for every block j:
-// P(j) V_j into O_(j mod 2), S(j+2) into P(j)'s buffer (tcgen05 operations of one thread run
-// in issue order, so the product reads P(j) before S(j+2) overwrites it).  The commit that
-// signals S(j) covers P(j-2) V, the last product into the stream's accumulator, so a lazy
-// rescale of O_s needs no other wait.
+// MMA order inside a unit (one warp of CTA 0): S(0), S(1), then for every block j: S(j+2)
+// once S(j) has been read, then P(j) V_j into O once P(j) is written.  O is rescaled (by
+// the softmax of block j, rarely) only after P(j-1) V has completed (pv_done) and before
+// P(j) V is issued.
 //
 // Synchronisation.  Barriers sit at the same offsets in both CTAs.  Those the MMA warp waits
-// on live in CTA 0 (slot_full, q_full, p_full, o_empty, unit_empty): both CTAs' copies signal
-// CTA 0's slot_full/q_full (.cta_group::2 copies), and CTA 1's softmax warps arrive on CTA
-// 0's p_full/o_empty remotely.  Those the producers and softmax warps wait on are signalled
-// in both CTAs at once by the MMA commits (slot_empty, q_empty, s_full, o_full).  CTA 0's
-// producer claims units and writes each into both CTAs' unit rings.
+// on live in CTA 0 (slot_full, q_full, s_free, p_full, o_empty, unit_empty): both CTAs'
+// copies signal CTA 0's slot_full/q_full (.cta_group::2 copies), and CTA 1's softmax warps
+// arrive on CTA 0's s_free/p_full/o_empty remotely.  Those the producers and softmax warps
+// wait on are signalled in both CTAs at once by the MMA commits (slot_empty, q_empty,
+// s_full, pv_done, o_full).  CTA 0's producer claims units and writes each into both CTAs'
+// unit rings.  The maximum handoff and the epilogue's sum exchange stay inside a CTA.
 #pragma once
 
 #include "fa_fwd_kernel.cuh"
@@ -92,23 +95,25 @@ constexpr int S_KSTEPS = D / 16;
 constexpr int PV_KSTEPS = BN / 16;
 constexpr uint32_t IDESC_S = ptx::make_idesc(1u, 256, BN, 0);
 constexpr uint32_t IDESC_O = ptx::make_idesc(1u, 256, D, 1);
-constexpr uint32_t O_COL0 = 256;            // O_0; O_1 follows at O_COL0 + D
+constexpr uint32_t O_COL0 = 256;            // the accumulator O (128 columns)
+constexpr uint32_t P_COL0 = 384;            // numerator buffers P(b) at P_COL0 + 64 b
 constexpr int UNIT_RING_P = 4;
 // consumers of a published unit: CTA 0's MMA warp and eight softmax warps, CTA 1's eight
 // softmax warps and its producer
 constexpr uint32_t UNIT_CONSUMERS = 1 + 8 + 8 + 1;
 constexpr uint32_t SOFTMAX_WARPS_PAIR = 16;  // softmax warps of both CTAs (o_empty)
+constexpr uint32_t STREAM_WARPS_PAIR = 8;    // one stream's softmax warps, both CTAs
 constexpr uint16_t BOTH = 0x3;              // CTA mask of the pair
 
-// shared memory: two Q buffers (unit parity), the K/V ring, the exchange of the streams'
-// row statistics [2 unit parities][maximum, sum][2 streams][128 rows] (fp32), the mbarriers
-// and the control words
+// shared memory: two Q buffers (unit parity), the K/V ring, the per-row maximum handed
+// between the streams [2 streams][128 rows] and the epilogue's sum exchange [2 streams][128
+// rows] (fp32), the mbarriers and the control words
 constexpr int Q_OFF = 0;
 constexpr int RING_OFF = 2 * Q_TILE_BYTES;
 constexpr int XCH_OFF = RING_OFF + NSLOT * SLOT_BYTES;
-constexpr int XCH_BYTES = 2 * 2 * 2 * BM * 4;
+constexpr int XCH_BYTES = 2 * 2 * BM * 4;
 constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
-constexpr int NUM_BARS = 2 * NSLOT + 18 + 2 * UNIT_RING_P;
+constexpr int NUM_BARS = 2 * NSLOT + 27 + 2 * UNIT_RING_P;
 constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
 // control words: TMEM base, abort flag, 2 spare, then the unit ring
 constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16 + 4 * UNIT_RING_P;
@@ -118,19 +123,22 @@ struct PBars {
   uint32_t base;
   __device__ uint32_t slot_full(int s) const { return base + 8u * s; }
   __device__ uint32_t slot_empty(int s) const { return base + 8u * (NSLOT + s); }
-  __device__ uint32_t q_full(int q) const { return base + 8u * (2 * NSLOT + q); }
-  __device__ uint32_t q_empty(int q) const { return base + 8u * (2 * NSLOT + 2 + q); }
-  __device__ uint32_t s_full(int b) const { return base + 8u * (2 * NSLOT + 4 + b); }
-  __device__ uint32_t p_full(int b) const { return base + 8u * (2 * NSLOT + 6 + b); }
-  __device__ uint32_t o_full() const { return base + 8u * (2 * NSLOT + 8); }
-  __device__ uint32_t o_empty() const { return base + 8u * (2 * NSLOT + 10); }
-  __device__ uint32_t drain() const { return base + 8u * (2 * NSLOT + 13); }
-  // row-statistics exchange of warp pair (wq, wq + 4), wq = 0..3
-  __device__ uint32_t xchg(int wq) const { return base + 8u * (2 * NSLOT + 14 + wq); }
-  __device__ uint32_t unit_full(int s) const { return base + 8u * (2 * NSLOT + 18 + s); }
-  __device__ uint32_t unit_empty(int s) const {
-    return base + 8u * (2 * NSLOT + 18 + UNIT_RING_P + s);
-  }
+  __device__ uint32_t at(int i) const { return base + 8u * (2 * NSLOT + i); }
+  __device__ uint32_t q_full(int q) const { return at(q); }
+  __device__ uint32_t q_empty(int q) const { return at(2 + q); }
+  __device__ uint32_t s_full(int b) const { return at(4 + b); }    // S(b) computed
+  __device__ uint32_t s_free(int b) const { return at(6 + b); }    // S(b) read by the softmax
+  __device__ uint32_t p_full(int b) const { return at(8 + b); }    // P(b) written
+  __device__ uint32_t pv_done(int b) const { return at(10 + b); }  // P(b) V completed
+  __device__ uint32_t o_full() const { return at(12); }
+  __device__ uint32_t o_empty() const { return at(13); }
+  __device__ uint32_t drain() const { return at(14); }
+  // epilogue sum exchange of warp pair (wq, wq + 4), wq = 0..3
+  __device__ uint32_t xchg(int wq) const { return at(15 + wq); }
+  // maximum published by stream s for the rows of lane quarter wq
+  __device__ uint32_t hand(int s, int wq) const { return at(19 + 4 * s + wq); }
+  __device__ uint32_t unit_full(int s) const { return at(27 + s); }
+  __device__ uint32_t unit_empty(int s) const { return at(27 + UNIT_RING_P + s); }
 };
 
 // The CTA's abort flag and its address in the peer CTA: a wait that gives up raises both,
@@ -338,7 +346,10 @@ __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, 
   const uint64_t v_d0 = ptx::smem_desc_sw128(smem + RING_OFF, SLOT_BYTES, 1024);
   constexpr uint32_t SLOT_STEP = SLOT_BYTES >> 4;
   constexpr uint32_t QBUF_STEP = Q_TILE_BYTES >> 4;
-  uint32_t kv_base = 0, pph = 0, unit_it = 0, taken = 0;
+  uint32_t kv_base = 0, unit_it = 0, taken = 0;
+  uint32_t pph = 0;           // phase bits of p_full(b), bit b
+  uint32_t sfph = 0;          // phase bits of s_free(b), bit b
+  uint32_t s_issued = 0;      // bit b: an S product has been issued into buffer b
   auto wait = [&](uint32_t b, uint32_t parity) {
     const bool ok = pwait(b, parity, ab, ERR_WAIT_MMA);
     return __all_sync(0xffffffffu, ok);
@@ -360,38 +371,40 @@ __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, 
     const int n = w.n;
     const int qb = unit_it & 1;
     const uint64_t q_d = q_d0 + qb * QBUF_STEP;
-    auto scores = [&](int j, uint32_t ki) {
-      pair_issue_s(tmem + (j & 1) * BN, q_d, k_d0 + (ki % NSLOT) * SLOT_STEP);
-      ptx::mma2_commit_mc_elect(bar.s_full(j & 1), BOTH);
+    // S(j) into buffer j mod 2, once the softmax has read the buffer's previous scores
+    auto scores = [&](int j) -> bool {
+      const int b = j & 1;
+      if ((s_issued >> b) & 1u) {
+        if (!wait(bar.s_free(b), (sfph >> b) & 1u)) return false;
+        sfph ^= 1u << b;
+      }
+      const uint32_t ki = kv_base + 2 * j;
+      if (!wait_slot(ki)) return false;
+      ptx::tc_fence_after();
+      pair_issue_s(tmem + b * BN, q_d, k_d0 + (ki % NSLOT) * SLOT_STEP);
+      ptx::mma2_commit_mc_elect(bar.s_full(b), BOTH);
       ptx::mma2_commit_mc_elect(bar.slot_empty(ki % NSLOT), BOTH);
       if (j == n - 1) ptx::mma2_commit_mc_elect(bar.q_empty(qb), BOTH);
+      s_issued |= 1u << b;
+      return true;
     };
     if (!wait(bar.q_full(qb), (unit_it >> 1) & 1u)) break;
-    bool ok = true;
-    for (int j = 0; j < 2 && j < n; ++j) {
-      if (!wait_slot(kv_base + 2 * j)) { ok = false; break; }
-      ptx::tc_fence_after();
-      scores(j, kv_base + 2 * j);
-    }
+    bool ok = scores(0) && (n < 2 || scores(1));
     for (int j = 0; j < n && ok; ++j) {
-      const int b = j & 1;  // key stream
+      const int b = j & 1;
+      if (j + 2 < n && !scores(j + 2)) { ok = false; break; }
       const uint32_t vi = kv_base + 2 * j + 1;
       if (!wait_slot(vi)) { ok = false; break; }
       if (!wait(bar.p_full(b), (pph >> b) & 1u)) { ok = false; break; }
       pph ^= 1u << b;
-      // the previous unit's epilogue has read both accumulators
+      // the previous unit's epilogue has read O
       if (j == 0 && !wait(bar.o_empty(), (unit_it & 1u) ^ 1u)) { ok = false; break; }
       ptx::tc_fence_after();
-      pair_issue_pv(tmem + O_COL0 + b * D, tmem + b * BN, v_d0 + (vi % NSLOT) * SLOT_STEP,
-                    j >= 2 ? 1u : 0u);
+      pair_issue_pv(tmem + O_COL0, tmem + P_COL0 + b * 64, v_d0 + (vi % NSLOT) * SLOT_STEP,
+                    j > 0 ? 1u : 0u);
+      ptx::mma2_commit_mc_elect(bar.pv_done(b), BOTH);
       ptx::mma2_commit_mc_elect(bar.slot_empty(vi % NSLOT), BOTH);
       if (j == n - 1) ptx::mma2_commit_mc_elect(bar.o_full(), BOTH);
-      if (j + 2 < n) {
-        const uint32_t ki = kv_base + 2 * (j + 2);
-        if (!wait_slot(ki)) { ok = false; break; }
-        ptx::tc_fence_after();
-        scores(j + 2, ki);
-      }
     }
     if (!ok) break;
     kv_base += 2 * n;
@@ -404,8 +417,29 @@ __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, 
 
 // ---------------------------------------------------------------------------- softmax
 
+// Maximum of a 128-score row: per 32 columns a tree of three-input maxima (depth 4; a
+// chain of them would be 16 deep), then across the four.
+__device__ __forceinline__ float row_max128(const uint32_t (&sr)[4][32]) {
+  float m[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float t[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i)
+      t[i] = ptx::max3(__uint_as_float(sr[c][3 * i]), __uint_as_float(sr[c][3 * i + 1]),
+                       __uint_as_float(sr[c][3 * i + 2]));
+    t[10] = fmaxf(__uint_as_float(sr[c][30]), __uint_as_float(sr[c][31]));
+    const float u0 = ptx::max3(t[0], t[1], t[2]), u1 = ptx::max3(t[3], t[4], t[5]);
+    const float u2 = ptx::max3(t[6], t[7], t[8]), u3 = fmaxf(t[9], t[10]);
+    m[c] = fmaxf(ptx::max3(u0, u1, u2), u3);
+  }
+  return fmaxf(ptx::max3(m[0], m[1], m[2]), m[3]);
+}
+
 // A 128-score row (sr) -> bf16 numerators at t_p (64 columns); adds the sum of the
 // unrounded numerators to le.  NPOLY of every 8 column pairs use the FMA-pipe exponential.
+// Per 32 columns: all arguments first, then all exponentials, then the packing and the
+// sums, so that the exponentials issue back to back.
 template <int NPOLY>
 __device__ __forceinline__ void pair_numerators(const uint32_t (&sr)[4][32], float sl2,
                                                 float neg_m, uint32_t t_p, float &le) {
@@ -414,21 +448,27 @@ __device__ __forceinline__ void pair_numerators(const uint32_t (&sr)[4][32], flo
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    uint32_t pk[16];
+    float x[32], pe[32];
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
       const uint64_t xx = ptx::f2_fma(
           ptx::f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, bias2);
-      float x0, x1, p0, p1;
-      ptx::f2_unpack(xx, x0, x1);
+      ptx::f2_unpack(xx, x[e], x[e + 1]);
+    }
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
       if (((e % 16) / 2) < NPOLY) {
-        exp2_poly_pair(x0, x1, p0, p1);
+        exp2_poly_pair(x[e], x[e + 1], pe[e], pe[e + 1]);
       } else {
-        p0 = ptx::ex2(x0);
-        p1 = ptx::ex2(x1);
+        pe[e] = ptx::ex2(x[e]);
+        pe[e + 1] = ptx::ex2(x[e + 1]);
       }
-      acc[(e / 2) & 3] = ptx::f2_add(acc[(e / 2) & 3], ptx::f2_pack(p0, p1));
-      pk[e / 2] = ptx::pack_bf16x2(p0, p1);
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      pk[e / 2] = ptx::pack_bf16x2(pe[e], pe[e + 1]);
+      acc[(e / 2) & 3] = ptx::f2_add(acc[(e / 2) & 3], ptx::f2_pack(pe[e], pe[e + 1]));
     }
     ptx::tmem_st16(t_p + c * 16, pk);
   }
@@ -447,13 +487,36 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
   const int r_cta = wq * 32 + lane;  // row inside the CTA's 128
   const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
   const uint32_t t_s = tmem + lane_base + h * BN;
-  const uint32_t t_o = tmem + lane_base + O_COL0;  // O_0; O_1 is D columns further
+  const uint32_t t_o = tmem + lane_base + O_COL0;
+  const uint32_t t_p = tmem + lane_base + P_COL0 + h * 64;
   const uint32_t p_full_c = ptx::mapa(bar.p_full(h), 0);
+  const uint32_t s_free_c = ptx::mapa(bar.s_free(h), 0);
   const uint32_t o_empty_c = ptx::mapa(bar.o_empty(), 0);
+  const uint32_t my_hand = bar.hand(h, wq), other_hand = bar.hand(h ^ 1, wq);
   const uint32_t xbar = bar.xchg(wq);
-
+  volatile float *mh = xch;            // [stream][row]: maximum in use after its latest block
+  volatile float *xl = xch + 2 * BM;   // [stream][row]: row sums, for the epilogue
   const float NEG_INF = -__int_as_float(0x7f800000);
-  uint32_t sph = 0, xph = 0, unit_it = 0, taken = 0;
+  uint32_t sph = 0;        // phase bit of s_full(h)
+  uint32_t hph = 0;        // phase bit of the other stream's hand barrier
+  uint32_t xph = 0;        // phase bit of xchg
+  uint32_t pvc0 = 0, pvc1 = 0;  // P V products committed on pv_done(0 / 1) in earlier units
+  uint32_t unit_it = 0, taken = 0;
+  // arrive on one of CTA 0's barriers (local in CTA 0, remote from CTA 1)
+  auto arrive0 = [&](uint32_t local, uint32_t remote) {
+    if (rank == 0)
+      ptx::mbar_arrive_elect(local);
+    else
+      ptx::mbar_arrive_remote_elect(remote);
+  };
+  // the maximum in use after the other stream's latest block
+  auto take_other_max = [&](float &m) {
+    const bool ok = pwait(other_hand, hph, ab, ERR_WAIT_SOFTMAX);
+    hph ^= 1u;
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    m = mh[(h ^ 1) * BM + r_cta];
+    return true;
+  };
 
   for (;;) {
     uint32_t u;
@@ -469,14 +532,16 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
     }
     if (u >= static_cast<uint32_t>(p.num_units)) return;
     const PUnit w = pair_decode<CAUSAL>(p, static_cast<int>(u));
+    const int n = w.n;
     const int row0 = w.r0 + static_cast<int>(rank) * BM;  // first row of this CTA
     const int row = row0 + r_cta;
     const float sl2 = p.scale_log2;
     const int key_lim = CAUSAL ? min(row + w.off, p.Nk - 1) : p.Nk - 1;
-    float m_used = NEG_INF;  // this stream's running maximum (base-2 scaled domain)
-    float l = 0.f;           // this stream's row sum
+    float m_used = NEG_INF;  // maximum in use after the latest block this warp knows of
+    float m_ref = NEG_INF;   // maximum this stream's sum l is relative to
+    float l = 0.f;
 
-    for (int j = h; j < w.n; j += 2) {
+    for (int j = h; j < n; j += 2) {
       bool ok = pwait(bar.s_full(h), sph, ab, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;
       sph ^= 1u;
@@ -487,6 +552,10 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
       ptx::tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) ptx::reg_fence32(sr[c]);
+      // S(h) is read: the tensor core may compute S(j+2) into it
+      ptx::tc_fence_before();
+      __syncwarp();
+      arrive0(bar.s_free(h), s_free_c);
 
       const int kv0 = j * BN;
       const bool need_mask = (CAUSAL && kv0 + BN - 1 > row0 + w.off) || (kv0 + BN > p.Nk);
@@ -498,104 +567,101 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
           for (int e = 0; e < 32; ++e)
             if (c * 32 + e > lim) sr[c][e] = __float_as_uint(NEG_INF);
       }
-      float mx[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float m = ptx::max3(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]),
-                            __uint_as_float(sr[c][2]));
-#pragma unroll
-        for (int e = 3; e < 31; e += 2)
-          m = ptx::max3(m, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
-        mx[c] = fmaxf(m, __uint_as_float(sr[c][31]));
+      const float xmax = row_max128(sr) * sl2;
+      // the maximum in use before this block, then the one after it, handed on to block j+1
+      float m_prev = NEG_INF;
+      if (j > 0 && !take_other_max(m_prev)) return;
+      const float m_new = xmax > m_prev + RESCALE_THRESHOLD ? xmax : m_prev;
+      mh[h * BM + r_cta] = m_new;
+      __syncwarp();
+      ptx::mbar_arrive_elect(my_hand);
+      m_used = m_new;
+      // this stream's sum follows the maximum in use
+      if (m_new != m_ref) {
+        l = (m_ref == NEG_INF) ? 0.f : l * ptx::ex2(m_ref - m_new);
+        m_ref = m_new;
       }
-      const float xmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
-      const bool resc = xmax > m_used + RESCALE_THRESHOLD;
-      const float alpha = resc ? ptx::ex2(m_used - xmax) : 1.f;  // 0 on the stream's first block
-      if (__any_sync(0xffffffffu, resc && j >= 2)) {
-        // O_h is quiescent: the commit that signalled S(j) covered P(j-2) V
-        const uint32_t t_oh = t_o + h * D;
+      if (__any_sync(0xffffffffu, m_new != m_prev && j > 0)) {
+        // rescale O to the new maximum once P(j-1) V (the other stream's, the last product
+        // into O so far) has completed; P(j) V is issued only after this block's p_full
+        const int b1 = (j - 1) & 1;
+        ok = pwait(bar.pv_done(b1), ((b1 ? pvc1 : pvc0) + (j - 1) / 2) & 1u, ab,
+                   ERR_WAIT_SOFTMAX);
+        if (!__all_sync(0xffffffffu, ok)) return;
+        ptx::tc_fence_after();
+        const float alpha = (m_new != m_prev) ? ptx::ex2(m_prev - m_new) : 1.f;
 #pragma unroll 1
         for (int c = 0; c < D / 16; ++c) {
           uint32_t o[16];
-          ptx::tmem_ld16(t_oh + c * 16, o);
+          ptx::tmem_ld16(t_o + c * 16, o);
           ptx::tmem_wait_ld();
           ptx::reg_fence16(o);
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          ptx::tmem_st16(t_oh + c * 16, o);
+          ptx::tmem_st16(t_o + c * 16, o);
         }
       }
-      if (resc) {
-        l *= alpha;
-        m_used = xmax;
+      // P(h) was read by this stream's previous product P(j-2) V
+      if (j >= 2) {
+        ok = pwait(bar.pv_done(h), ((h ? pvc1 : pvc0) + (j - 2) / 2) & 1u, ab, ERR_WAIT_SOFTMAX);
+        if (!__all_sync(0xffffffffu, ok)) return;
+        ptx::tc_fence_after();
       }
-      const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
+      const float neg_m = (m_new == NEG_INF) ? 0.f : -m_new;
       float le = 0.f;
       if (POLY_PAIRS == 0 || need_mask)
-        pair_numerators<0>(sr, sl2, neg_m, t_s, le);
+        pair_numerators<0>(sr, sl2, neg_m, t_p, le);
       else
-        pair_numerators<POLY_PAIRS>(sr, sl2, neg_m, t_s, le);
+        pair_numerators<POLY_PAIRS>(sr, sl2, neg_m, t_p, le);
       l += le;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      ptx::mbar_arrive_remote_elect(p_full_c);
+      arrive0(bar.p_full(h), p_full_c);
     }
 
-    // Epilogue: merge the two streams, O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1) with
-    // a_s = 2^(m_s - m), m = max(m_0, m_1); LSE = ln 2 * (m + log2 l).  A stream without
-    // admissible keys for this row (l_s = 0: no block, or all masked) adds nothing; its
-    // accumulator may hold stale values and is not read into the result.
+    // Epilogue.  m = the maximum in use after block n-1; O and both sums are relative to it
+    // once each stream's sum is brought there: O = O_acc / (l_0 + l_1), LSE = ln 2 (m +
+    // log2(l_0 + l_1)).
     {
-      // [stream][row] maxima and sums of this unit's parity: a stream that finishes its next
-      // unit early cannot overwrite values its partner has not read yet
-      volatile float *xm = xch + (unit_it & 1) * 4 * BM;
-      volatile float *xl = xm + 2 * BM;
-      xm[h * BM + r_cta] = m_used;
-      xl[h * BM + r_cta] = l;
-      __syncwarp();
-      ptx::mbar_arrive_elect(xbar);
-      bool ok = pwait(xbar, xph, ab, ERR_WAIT_SOFTMAX);
-      xph ^= 1u;
-      if (!__all_sync(0xffffffffu, ok)) return;
-      const float m0 = xm[r_cta], m1 = xm[BM + r_cta];
-      const float l0 = xl[r_cta], l1 = xl[BM + r_cta];
-      const float m = fmaxf(m0, m1);
-      const float a0 = l0 > 0.f ? ptx::ex2(m0 - m) : 0.f;
-      const float a1 = l1 > 0.f ? ptx::ex2(m1 - m) : 0.f;
-      const float lt = a0 * l0 + a1 * l1;
-      ok = pwait(bar.o_full(), unit_it & 1u, ab, ERR_WAIT_SOFTMAX);
+      float m = m_used;
+      if (((n - 1) & 1) != h && !take_other_max(m)) return;
+      const float lm = (l > 0.f) ? l * ptx::ex2(m_ref - m) : 0.f;
+      bool ok = pwait(bar.o_full(), unit_it & 1u, ab, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;
       ptx::tc_fence_after();
+      // written only after o_full: the partner has read the previous unit's value, since
+      // this unit's products waited for its o_empty
+      xl[h * BM + r_cta] = lm;
+      __syncwarp();
+      ptx::mbar_arrive_elect(xbar);
+      ok = pwait(xbar, xph, ab, ERR_WAIT_SOFTMAX);
+      xph ^= 1u;
+      if (!__all_sync(0xffffffffu, ok)) return;
+      const float lt = lm + xl[(h ^ 1) * BM + r_cta];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const float f0 = a0 * inv, f1 = a1 * inv;
       const bool valid = row < p.Nq;
       const size_t orow = static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const uint32_t col = h * 64 + c * 32;
-        uint32_t a[32], bq[32];
+        uint32_t a[32];
         ptx::tmem_ld32(t_o + col, a);
-        ptx::tmem_ld32(t_o + D + col, bq);
         ptx::tmem_wait_ld();
         ptx::reg_fence32(a);
-        ptx::reg_fence32(bq);
-        float v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          v[e] = (f0 != 0.f ? __uint_as_float(a[e]) * f0 : 0.f) +
-                 (f1 != 0.f ? __uint_as_float(bq[e]) * f1 : 0.f);
         if (valid) {
           if (OUT_F32) {
             float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + col);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              dst[q] = make_float4(__uint_as_float(a[4 * q]) * inv, __uint_as_float(a[4 * q + 1]) * inv,
+                                   __uint_as_float(a[4 * q + 2]) * inv, __uint_as_float(a[4 * q + 3]) * inv);
           } else {
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + col);
             uint32_t hh[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) hh[e] = ptx::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+            for (int e = 0; e < 16; ++e)
+              hh[e] = ptx::pack_bf16x2(__uint_as_float(a[2 * e]) * inv, __uint_as_float(a[2 * e + 1]) * inv);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               dst[q] = make_uint4(hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
@@ -606,8 +672,10 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
         p.lse[orow] = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994530942f : NEG_INF;
       ptx::tc_fence_before();
       __syncwarp();
-      ptx::mbar_arrive_remote_elect(o_empty_c);
+      arrive0(bar.o_empty(), o_empty_c);
     }
+    pvc0 += (n + 1) / 2;
+    pvc1 += n / 2;
     ++unit_it;
   }
 }
@@ -644,12 +712,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(bar.q_full(b), 1);
       ptx::mbar_init(bar.q_empty(b), 1);
       ptx::mbar_init(bar.s_full(b), 1);
-      ptx::mbar_init(bar.p_full(b), SOFTMAX_WARPS_PAIR / 2);  // one stream's warps, both CTAs
+      ptx::mbar_init(bar.s_free(b), STREAM_WARPS_PAIR);
+      ptx::mbar_init(bar.p_full(b), STREAM_WARPS_PAIR);
+      ptx::mbar_init(bar.pv_done(b), 1);
     }
     ptx::mbar_init(bar.o_full(), 1);
     ptx::mbar_init(bar.o_empty(), SOFTMAX_WARPS_PAIR);
     ptx::mbar_init(bar.drain(), 1);
-    for (int wq = 0; wq < 4; ++wq) ptx::mbar_init(bar.xchg(wq), 2);  // warps wq and wq + 4
+    for (int wq = 0; wq < 4; ++wq) {
+      ptx::mbar_init(bar.xchg(wq), 2);        // warps wq and wq + 4
+      ptx::mbar_init(bar.hand(0, wq), 1);     // one publishing warp per block
+      ptx::mbar_init(bar.hand(1, wq), 1);
+    }
     for (int s = 0; s < UNIT_RING_P; ++s) {
       ptx::mbar_init(bar.unit_full(s), 1);
       ptx::mbar_init(bar.unit_empty(s), UNIT_CONSUMERS);
