@@ -259,31 +259,39 @@ __device__ void pair_load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK,
         ptx::tma_load_3d_pair(smem + Q_OFF + qb * Q_TILE_BYTES + bx * Q_BOX_BYTES, tmQ, qf,
                               bx * 64, w.r0 + static_cast<int>(rank) * BM, w.bh);
       ++q_issued;
-      for (int j = 0; j < w.n; ++j) {
-        // K half: keys j*BN + 64 rank .. + 63, all dimensions (two 64-dimension boxes)
-        {
-          const int sl = issued % NSLOT;
-          if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
-            goto drain;
-          if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
-          const uint32_t sf = ptx::mapa(bar.slot_full(sl), 0);
+      // K and V halves in the order the MMA warp first needs them: K_0, K_1, then per block
+      // j K_(j+2) (its scores are computed early) and V_j
+      auto load_k = [&](int j) -> bool {
+        const int sl = issued % NSLOT;
+        if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
+          return false;
+        if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
+        const uint32_t sf = ptx::mapa(bar.slot_full(sl), 0);
+        // keys j*BN + 64 rank .. + 63, all dimensions (two 64-dimension boxes)
 #pragma unroll
-          for (int bx = 0; bx < 2; ++bx)
-            ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES + bx * K_BOX_BYTES, tmK, sf,
-                                  bx * 64, j * BN + static_cast<int>(rank) * 64, w.bhk);
-          ++issued;
-        }
-        // V half: keys j*BN .. + 127, dimensions 64 rank .. + 63
-        {
-          const int sl = issued % NSLOT;
-          if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
-            goto drain;
-          if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
-          ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES, tmV,
-                                ptx::mapa(bar.slot_full(sl), 0), static_cast<int>(rank) * 64,
-                                j * BN, w.bhk);
-          ++issued;
-        }
+        for (int bx = 0; bx < 2; ++bx)
+          ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES + bx * K_BOX_BYTES, tmK, sf,
+                                bx * 64, j * BN + static_cast<int>(rank) * 64, w.bhk);
+        ++issued;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int sl = issued % NSLOT;
+        if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
+          return false;
+        if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
+        // keys j*BN .. + 127, dimensions 64 rank .. + 63
+        ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES, tmV,
+                              ptx::mapa(bar.slot_full(sl), 0), static_cast<int>(rank) * 64,
+                              j * BN, w.bhk);
+        ++issued;
+        return true;
+      };
+      if (!load_k(0)) goto drain;
+      if (w.n > 1 && !load_k(1)) goto drain;
+      for (int j = 0; j < w.n; ++j) {
+        if (j + 2 < w.n && !load_k(j + 2)) goto drain;
+        if (!load_v(j)) goto drain;
       }
     }
     if (rank == 0) u = ptx::num_clusters_x() + atomicAdd(p.sched, 1u);
@@ -336,8 +344,19 @@ __device__ __forceinline__ void pair_issue_pv(uint32_t tmem_o, uint32_t tmem_s, 
   }
 }
 
+// Ring position, inside a unit of n key blocks, of K_k and V_j in the producer's order
+// K_0, K_1, then per block j: K_(j+2) (while j + 2 < n), V_j.
+__device__ __forceinline__ uint32_t k_pos(int k) { return k < 2 ? k : 2 * k - 2; }
+__device__ __forceinline__ uint32_t v_pos(int j, int n) {
+  return (n > 1 ? 2 : 1) + j + min(j + 1, max(n - 2, 0));
+}
+
 // Warp 8 of CTA 0.  Every commit that frees a resource or signals a result arrives on the
-// barrier in both CTAs.
+// barrier in both CTAs.  Inside a unit it issues, in a loop of non-blocking probes,
+// whichever product can go next: S(k) once its buffer has been read (s_free of block k-2),
+// K_k has landed and P(k-3) V has been issued, or P(j) V_j once the numerators P(j) are
+// written -- so scores for the next blocks never queue behind a product that waits for the
+// softmax.
 template <bool CAUSAL>
 __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, const PBars &bar,
                               volatile uint32_t *ring, const Abort &ab) {
@@ -350,14 +369,19 @@ __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, 
   uint32_t pph = 0;           // phase bits of p_full(b), bit b
   uint32_t sfph = 0;          // phase bits of s_free(b), bit b
   uint32_t s_issued = 0;      // bit b: an S product has been issued into buffer b
+  bool ok = true;
   auto wait = [&](uint32_t b, uint32_t parity) {
-    const bool ok = pwait(b, parity, ab, ERR_WAIT_MMA);
-    return __all_sync(0xffffffffu, ok);
+    const bool r = pwait(b, parity, ab, ERR_WAIT_MMA);
+    return __all_sync(0xffffffffu, r);
   };
-  auto wait_slot = [&](uint32_t idx) {
-    return wait(bar.slot_full(idx % NSLOT), (idx / NSLOT) & 1u);
+  // warp-uniform non-blocking probe
+  auto ready = [&](uint32_t b, uint32_t parity) {
+    return __all_sync(0xffffffffu, ptx::mbar_test_wait(b, parity));
   };
-  for (;;) {
+  auto slot_ready = [&](uint32_t idx) {
+    return ready(bar.slot_full(idx % NSLOT), (idx / NSLOT) & 1u);
+  };
+  while (ok) {
     const int s = taken % UNIT_RING_P;
     if (!__all_sync(0xffffffffu, pwait<true>(bar.unit_full(s), (taken / UNIT_RING_P) & 1u, ab,
                                              ERR_WAIT_MMA)))
@@ -371,40 +395,65 @@ __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, 
     const int n = w.n;
     const int qb = unit_it & 1;
     const uint64_t q_d = q_d0 + qb * QBUF_STEP;
-    // S(j) into buffer j mod 2, once the softmax has read the buffer's previous scores
-    auto scores = [&](int j) -> bool {
-      const int b = j & 1;
-      if ((s_issued >> b) & 1u) {
-        if (!wait(bar.s_free(b), (sfph >> b) & 1u)) return false;
-        sfph ^= 1u << b;
-      }
-      const uint32_t ki = kv_base + 2 * j;
-      if (!wait_slot(ki)) return false;
-      ptx::tc_fence_after();
-      pair_issue_s(tmem + b * BN, q_d, k_d0 + (ki % NSLOT) * SLOT_STEP);
-      ptx::mma2_commit_mc_elect(bar.s_full(b), BOTH);
-      ptx::mma2_commit_mc_elect(bar.slot_empty(ki % NSLOT), BOTH);
-      if (j == n - 1) ptx::mma2_commit_mc_elect(bar.q_empty(qb), BOTH);
-      s_issued |= 1u << b;
-      return true;
-    };
     if (!wait(bar.q_full(qb), (unit_it >> 1) & 1u)) break;
-    bool ok = scores(0) && (n < 2 || scores(1));
-    for (int j = 0; j < n && ok; ++j) {
-      const int b = j & 1;
-      if (j + 2 < n && !scores(j + 2)) { ok = false; break; }
-      const uint32_t vi = kv_base + 2 * j + 1;
-      if (!wait_slot(vi)) { ok = false; break; }
-      if (!wait(bar.p_full(b), (pph >> b) & 1u)) { ok = false; break; }
-      pph ^= 1u << b;
-      // the previous unit's epilogue has read O
-      if (j == 0 && !wait(bar.o_empty(), (unit_it & 1u) ^ 1u)) { ok = false; break; }
-      ptx::tc_fence_after();
-      pair_issue_pv(tmem + O_COL0, tmem + P_COL0 + b * 64, v_d0 + (vi % NSLOT) * SLOT_STEP,
-                    j > 0 ? 1u : 0u);
-      ptx::mma2_commit_mc_elect(bar.pv_done(b), BOTH);
-      ptx::mma2_commit_mc_elect(bar.slot_empty(vi % NSLOT), BOTH);
-      if (j == n - 1) ptx::mma2_commit_mc_elect(bar.o_full(), BOTH);
+    int next_s = 0, next_pv = 0;
+    uint64_t t_idle = 0;  // start of the current run of probes without progress
+    uint32_t spins = 0;
+    while (next_pv < n) {
+      bool progressed = false;
+      // S(k) only after P(k-3) V has been issued: products of one thread complete in
+      // order, so when the softmax sees S(k), every pv_done barrier has at most one pending
+      // phase (P(k-1) V or P(k-2) V), which its parity waits rely on
+      if (next_s < n && next_s <= next_pv + 2) {
+        const int k = next_s, b = k & 1;
+        const bool buf_free = !((s_issued >> b) & 1u) || ready(bar.s_free(b), (sfph >> b) & 1u);
+        const uint32_t ki = kv_base + k_pos(k);
+        if (buf_free && slot_ready(ki)) {
+          if ((s_issued >> b) & 1u) sfph ^= 1u << b;
+          ptx::tc_fence_after();
+          pair_issue_s(tmem + b * BN, q_d, k_d0 + (ki % NSLOT) * SLOT_STEP);
+          ptx::mma2_commit_mc_elect(bar.s_full(b), BOTH);
+          ptx::mma2_commit_mc_elect(bar.slot_empty(ki % NSLOT), BOTH);
+          if (k == n - 1) ptx::mma2_commit_mc_elect(bar.q_empty(qb), BOTH);
+          s_issued |= 1u << b;
+          ++next_s;
+          progressed = true;
+        }
+      }
+      if (next_pv < next_s) {
+        const int j = next_pv, b = j & 1;
+        const uint32_t vi = kv_base + v_pos(j, n);
+        // the previous unit's epilogue has read O before P(0) V overwrites it
+        if (ready(bar.p_full(b), (pph >> b) & 1u) && slot_ready(vi) &&
+            (j > 0 || ready(bar.o_empty(), (unit_it & 1u) ^ 1u))) {
+          pph ^= 1u << b;
+          ptx::tc_fence_after();
+          pair_issue_pv(tmem + O_COL0, tmem + P_COL0 + b * 64, v_d0 + (vi % NSLOT) * SLOT_STEP,
+                        j > 0 ? 1u : 0u);
+          ptx::mma2_commit_mc_elect(bar.pv_done(b), BOTH);
+          ptx::mma2_commit_mc_elect(bar.slot_empty(vi % NSLOT), BOTH);
+          if (j == n - 1) ptx::mma2_commit_mc_elect(bar.o_full(), BOTH);
+          ++next_pv;
+          progressed = true;
+        }
+      }
+      if (progressed) {
+        t_idle = 0;
+        spins = 0;
+      } else if ((++spins & 255u) == 0) {
+        // bounded like every other wait: give up after WAIT_LIMIT_NS without progress
+        const uint64_t now = ptx::globaltimer_ns();
+        if (t_idle == 0) t_idle = now;
+        if (*ab.flag || now - t_idle > WAIT_LIMIT_NS || spins >= WAIT_MAX_ITERS) {
+          if (!*ab.flag) {
+            *ab.flag = 1u;
+            ptx::st_cluster_u32(ab.peer, 1u);
+            atomicOr(&g_fa_error, ERR_WAIT_MMA);
+          }
+          ok = false;
+          break;
+        }
+      }
     }
     if (!ok) break;
     kv_base += 2 * n;
