@@ -38,6 +38,7 @@ DATASHEET_FP8_TFLOPS = 4500.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["exact_attention_101_b200/csrc/fa_fwd_kernel.cuh",
+                  "exact_attention_101_b200/csrc/fa_fwd_pair.cuh",
                   "exact_attention_101_b200/csrc/sm100.cuh",
                   "exact_attention_101_b200/csrc/fa_api.cu"]
 
@@ -563,6 +564,27 @@ def run_ours(args):
                "api": ("fa_fwd_host: pinned host buffers, copies pipelined by head chunks"
                        if host_api else "pinned copies on the stream around the device call")}
 
+    # Lazy-rescale statistics of the d = 128 bf16 forward (its kernel counts them): one more
+    # launch on the workload's inputs and one on scores that drift along the keys (same
+    # shape), each against the eager rule's count on the same rows.
+    rescale = None
+    if (w.kind == "fwd" and not fp8 and not w.dropout and w.d == 128 and w.out_dtype == "bf16"):
+        def counts(qq, kk, vv):
+            fa.rescale_stats(reset=True, stream=stream)
+            fa.forward(qq, kk, vv, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+            steps, lazy, eager = fa.rescale_stats(reset=True, stream=stream)
+            return {"row_block_steps": steps, "lazy_rescales": lazy, "eager_rescales": eager,
+                    "eager_over_lazy": (eager / lazy) if lazy else None}
+        rescale = {"rule": "lazy: move the maximum only when a block exceeds it by more than 8 "
+                           "(log2 units); eager: whenever a block raises it",
+                   w.name: counts(q, k, v)}
+        dr = workloads.drift_inputs(w.B, w.Hq, w.N, w.d, seed=w.seed + 17)
+        dq_, dk_, dv_ = (t.to(dev) for t in (dr.q, dr.k, dr.v))
+        if w.Hkv != w.Hq:
+            dk_, dv_ = dk_[:, :w.Hkv].contiguous(), dv_[:, :w.Hkv].contiguous()
+        rescale["drift (scores ramp along the keys, workloads.drift_inputs)"] = counts(dq_, dk_, dv_)
+        del dq_, dk_, dv_
+
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -595,7 +617,8 @@ def run_ours(args):
             rate, desc, cores, _, _ = oracle_sample_rate(w, inp, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
                "cpu_model": cpu_model(), "nproc": os.cpu_count()}
-    kernel_name = "fa_fwd_kernel"
+    kernel_name = ("fa_fwd_pair_kernel (CTA pairs)" if (w.d == 128 and not fp8 and not w.dropout
+                                                      and w.kind == "fwd") else "fa_fwd_kernel")
     if w.kind == "bwd":
         kernel_name = ("fa_bwd: prep kernel + fa_bwd_kernel + dQ kernel (and the dQ "
                        "accumulator memset), timed together as one call")
@@ -622,6 +645,8 @@ def run_ours(args):
     }
     if quant is not None:
         line["quantise"] = quant
+    if rescale is not None:
+        line["rescale"] = rescale
     print(json.dumps(line))
 
 

@@ -21,8 +21,8 @@ FA_BF16, FA_BF16_OUT_F32, FA_E4M3 = range(3)
 
 # Exported C symbols, in the order of include/fa_b200.h.
 C_SYMBOLS = ("fa_fwd", "fa_fwd_host", "fa_fwd_dropout", "fa_fwd_varlen", "fa_fwd_fp8", "fa_bwd", "fa_bwd_noalloc", "fa_quantize_e4m3",
-             "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_string",
-             "fa_version")
+             "fa_check_device_error", "fa_rescale_stats", "fa_selftest_bounded_wait",
+             "fa_status_string", "fa_version")
 
 _lib = None
 
@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L.fa_quantize_e4m3.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.fa_check_device_error.restype = i
         L.fa_check_device_error.argtypes = [vp]
+        u64p = ctypes.POINTER(ctypes.c_ulonglong)
+        L.fa_rescale_stats.restype = i
+        L.fa_rescale_stats.argtypes = [vp, u64p, u64p, u64p, i]
         L.fa_selftest_bounded_wait.restype = i
         L.fa_selftest_bounded_wait.argtypes = [i, vp]
         L.fa_status_string.restype = ctypes.c_char_p
@@ -129,6 +132,23 @@ def fa_quantize_e4m3(x, signs, x8, descale, B, H, N, d, stream) -> int:
 
 def fa_check_device_error(stream) -> int:
     return lib().fa_check_device_error(stream)
+
+
+def fa_rescale_stats(stream, reset=False):
+    """Raw ``fa_rescale_stats``: returns (status, steps, lazy, eager)."""
+    st, lz, eg = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    r = lib().fa_rescale_stats(stream, ctypes.byref(st), ctypes.byref(lz), ctypes.byref(eg),
+                               int(bool(reset)))
+    return r, st.value, lz.value, eg.value
+
+
+def rescale_stats(reset=False, stream=None):
+    """(steps, lazy rescales, eager rescales) of the d = 128 bf16 forward since the last
+    reset, on the current device; raises on a non-zero status."""
+    r, steps, lazy, eager = fa_rescale_stats(_stream_handle(stream), reset)
+    if r != FA_OK:
+        raise FaError(r, "fa_rescale_stats")
+    return steps, lazy, eager
 
 
 def fa_selftest_bounded_wait(timeout_us, stream) -> int:

@@ -1152,6 +1152,24 @@ fa_status fa_check_device_error(fa_stream_t stream) {
   return FA_OK;
 }
 
+fa_status fa_rescale_stats(fa_stream_t stream, unsigned long long *steps,
+                           unsigned long long *lazy, unsigned long long *eager, int reset) {
+  if (!steps || !lazy || !eager) return FA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  unsigned long long v[3] = {0, 0, 0};
+  if (cudaMemcpyFromSymbol(v, fa::g_fa_rescale_stats, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
+  *steps = v[0];
+  *lazy = v[1];
+  *eager = v[2];
+  if (reset) {
+    const unsigned long long zero[3] = {0, 0, 0};
+    if (cudaMemcpyToSymbol(fa::g_fa_rescale_stats, zero, sizeof(zero)) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 fa_status fa_selftest_bounded_wait(int timeout_us, fa_stream_t stream) {
   if (timeout_us < 1 || timeout_us > 1000000) return FA_ERR_INVALID_ARG;
   fa::fa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(

@@ -263,6 +263,13 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams &p, int u) {
 
 __device__ unsigned int g_fa_error = 0;
 
+// Counters of the online softmax's rescaling, summed over the launches of the CTA-pair
+// forward (read and cleared by fa_rescale_stats): [0] (query row, key block) steps, [1]
+// rescales of the accumulator under the lazy rule the kernel runs, [2] rescales the eager
+// rule -- move the maximum whenever a block raises it -- would have made on the same rows.
+// A rescale is counted only once the row has seen an admissible key.
+__device__ unsigned long long g_fa_rescale_stats[3];
+
 // Bounded wait on an mbarrier phase.  Returns false if another warp of the CTA aborted or
 // if this wait ran out (then it raises the CTA abort flag and the device error word).
 __device__ __forceinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity,

@@ -106,12 +106,13 @@ constexpr uint32_t STREAM_WARPS_PAIR = 8;    // one stream's softmax warps, both
 constexpr uint16_t BOTH = 0x3;              // CTA mask of the pair
 
 // shared memory: two Q buffers (unit parity), the K/V ring, the per-row maximum handed
-// between the streams [2 streams][128 rows] and the epilogue's sum exchange [2 streams][128
-// rows] (fp32), the mbarriers and the control words
+// between the streams [2 streams][128 rows] (and the exact running maximum, for the rescale
+// statistics), the epilogue's sum exchange [2 streams][128 rows] (fp32), the mbarriers and
+// the control words
 constexpr int Q_OFF = 0;
 constexpr int RING_OFF = 2 * Q_TILE_BYTES;
 constexpr int XCH_OFF = RING_OFF + NSLOT * SLOT_BYTES;
-constexpr int XCH_BYTES = 2 * 2 * BM * 4;
+constexpr int XCH_BYTES = 3 * 2 * BM * 4;
 constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
 constexpr int NUM_BARS = 2 * NSLOT + 27 + 2 * UNIT_RING_P;
 constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
@@ -545,6 +546,8 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
   const uint32_t xbar = bar.xchg(wq);
   volatile float *mh = xch;            // [stream][row]: maximum in use after its latest block
   volatile float *xl = xch + 2 * BM;   // [stream][row]: row sums, for the epilogue
+  volatile float *mx = xch + 4 * BM;   // [stream][row]: exact running maximum (statistics)
+  uint32_t n_steps = 0, n_lazy = 0, n_eager = 0;  // rescale statistics of this thread's row
   const float NEG_INF = -__int_as_float(0x7f800000);
   uint32_t sph = 0;        // phase bit of s_full(h)
   uint32_t hph = 0;        // phase bit of the other stream's hand barrier
@@ -558,13 +561,29 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
     else
       ptx::mbar_arrive_remote_elect(remote);
   };
-  // the maximum in use after the other stream's latest block
-  auto take_other_max = [&](float &m) {
+  // the maximum in use (and the exact running maximum) after the other stream's latest
+  // block
+  auto take_other_max = [&](float &m, float &me) {
     const bool ok = pwait(other_hand, hph, ab, ERR_WAIT_SOFTMAX);
     hph ^= 1u;
     if (!__all_sync(0xffffffffu, ok)) return false;
     m = mh[(h ^ 1) * BM + r_cta];
+    me = mx[(h ^ 1) * BM + r_cta];
     return true;
+  };
+  // at the end of the work list: add this warp's rescale statistics to the device counters
+  auto flush_stats = [&]() {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      n_steps += __shfl_xor_sync(0xffffffffu, n_steps, o);
+      n_lazy += __shfl_xor_sync(0xffffffffu, n_lazy, o);
+      n_eager += __shfl_xor_sync(0xffffffffu, n_eager, o);
+    }
+    if (lane == 0) {
+      atomicAdd(&g_fa_rescale_stats[0], static_cast<unsigned long long>(n_steps));
+      atomicAdd(&g_fa_rescale_stats[1], static_cast<unsigned long long>(n_lazy));
+      atomicAdd(&g_fa_rescale_stats[2], static_cast<unsigned long long>(n_eager));
+    }
   };
 
   for (;;) {
@@ -579,7 +598,10 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
       ptx::mbar_arrive_cluster_elect(ptx::mapa(bar.unit_empty(s), 0));
       ++taken;
     }
-    if (u >= static_cast<uint32_t>(p.num_units)) return;
+    if (u >= static_cast<uint32_t>(p.num_units)) {
+      flush_stats();
+      return;
+    }
     const PUnit w = pair_decode<CAUSAL>(p, static_cast<int>(u));
     const int n = w.n;
     const int row0 = w.r0 + static_cast<int>(rank) * BM;  // first row of this CTA
@@ -618,9 +640,13 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
       }
       const float xmax = row_max128(sr) * sl2;
       // the maximum in use before this block, then the one after it, handed on to block j+1
-      float m_prev = NEG_INF;
-      if (j > 0 && !take_other_max(m_prev)) return;
+      float m_prev = NEG_INF, me_prev = NEG_INF;
+      if (j > 0 && !take_other_max(m_prev, me_prev)) return;
       const float m_new = xmax > m_prev + RESCALE_THRESHOLD ? xmax : m_prev;
+      ++n_steps;
+      n_lazy += (m_new != m_prev && m_prev != NEG_INF) ? 1u : 0u;
+      n_eager += (xmax > me_prev && me_prev != NEG_INF) ? 1u : 0u;
+      mx[h * BM + r_cta] = fmaxf(me_prev, xmax);
       mh[h * BM + r_cta] = m_new;
       __syncwarp();
       ptx::mbar_arrive_elect(my_hand);
@@ -673,8 +699,8 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
     // once each stream's sum is brought there: O = O_acc / (l_0 + l_1), LSE = ln 2 (m +
     // log2(l_0 + l_1)).
     {
-      float m = m_used;
-      if (((n - 1) & 1) != h && !take_other_max(m)) return;
+      float m = m_used, me_unused;
+      if (((n - 1) & 1) != h && !take_other_max(m, me_unused)) return;
       const float lm = (l > 0.f) ? l * ptx::ex2(m_ref - m) : 0.f;
       bool ok = pwait(bar.o_full(), unit_it & 1u, ab, ERR_WAIT_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) return;

@@ -302,6 +302,27 @@ fa_status fa_quantize_e4m3(const void *x, const int8_t *signs, void *x8, float *
 fa_status fa_check_device_error(fa_stream_t stream);
 
 /*
+ * Statistics of the online softmax's lazy rescaling.  The page "FlashAttention 4:
+ * Praxisleitfaden ...", section "Intelligenteres Online-Softmax-Rescaling in FA4", states
+ * that rescaling the accumulator only when the running maximum has moved far (here: by
+ * more than 8 in log2 units) needs about ten times fewer rescales than doing so whenever
+ * it moves.  The bf16 head-dimension-128 forward (fa_fwd and fa_fwd_host at d = 128)
+ * counts, per (query row, key block) step, whether it rescaled, and whether the eager rule
+ * would have; the other kernel instances count nothing.  Counters are per device and sum
+ * over all launches (concurrent ones included) since the last reset.
+ *
+ * fa_rescale_stats synchronises `stream`, then writes the counters of the current device:
+ *   steps   (query row, key block) steps processed (rows of the last partial unit
+ *           included: a unit is 256 query rows, a key block 128 keys)
+ *   lazy    rescales made (after the row's first admissible key)
+ *   eager   rescales the eager rule would have made on the same rows
+ * and clears them if `reset` is non-zero.  Returns FA_OK, FA_ERR_INVALID_ARG for a null
+ * pointer, FA_ERR_CUDA if a CUDA call failed.
+ */
+fa_status fa_rescale_stats(fa_stream_t stream, unsigned long long *steps,
+                           unsigned long long *lazy, unsigned long long *eager, int reset);
+
+/*
  * Self-test of the failure path above, without faulting anything: launches one warp that
  * waits on a shared-memory mbarrier nothing ever arrives on, with a limit of timeout_us
  * microseconds (1 .. 1000000).  The wait runs out, the kernel records the time-out in the

@@ -210,3 +210,29 @@ def random_bf16(shape, seed: int) -> torch.Tensor:
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     return torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def drift_inputs(B: int, H: int, N: int, d: int, seed: int, drift: float = 12.0) -> Inputs:
+    """Scores that drift along the keys, so that the running row maximum keeps rising and
+    the online softmax has to rescale again and again: Q i.i.d. N(0, 1); K = 0.2 N(0, 1)
+    plus a ramp from 0 to `drift` along the keys times the sign of Q's mean over the rows
+    (per head and dimension), so each row's scores grow or shrink linearly; V i.i.d.
+    N(0, 1).  Drawn in the order Q, K noise, V; returned in bf16."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn((B, H, N, d), generator=g)
+    k = torch.randn((B, H, N, d), generator=g) * 0.2
+    k += torch.linspace(0, drift, N)[None, None, :, None] * q.mean(dim=2, keepdim=True).sign()
+    v = torch.randn((B, H, N, d), generator=g)
+    return Inputs(q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
+
+
+def quantise_inputs_e4m3(inp: Inputs) -> Inputs:
+    """The fp8 path's per-(batch, head) amax quantisation of bf16 inputs (codes and
+    descales), the recipe of the fp8 workload."""
+    out = {}
+    for name in ("q", "k", "v"):
+        codes, ds = _quantise_e4m3_per_head(getattr(inp, name).float())
+        out[name], out["descale_" + name] = codes, ds
+    return Inputs(out["q"], out["k"], out["v"], out["descale_q"], out["descale_k"],
+                  out["descale_v"])
