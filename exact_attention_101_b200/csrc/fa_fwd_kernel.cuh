@@ -25,7 +25,7 @@
 //
 // Key tiles are BN = 64 keys, and every Q tile has NBUF = 2 score buffers in tensor
 // memory: while the softmax warps of a tile turn S(j) into P(j), the tensor core already
-// computes S(j+1), and S(j+2) as soon as P(j) has been consumed.  So a tile's softmax
+// computes S(j+1), and S(j+NBUF) as soon as P(j) has been consumed.  So a tile's softmax
 // never waits for its own P.V product, and the two tiles' softmax warps -- one of each
 // per SM sub-partition -- can both be busy at once.  This matters on B200 because, at head dim 128, the
 // exponentials of one score tile take the SFU as long as the tensor core takes for that
@@ -50,7 +50,7 @@
 //   slot_full / slot_empty  ring slot loaded (TMA tx bytes) / released by an MMA commit
 //   s_full[x][b]            S(x, b) computed
 //   p_full[x][b]            P(x, b) written by the 128 softmax threads of tile x
-//   pv_done[x]              one P.V product of tile x finished (for the rare rescale)
+//   pv_done[x][n & 1]       P.V product n of tile x finished (for the rare rescale)
 //   o_full[x] / o_empty[x]  O_x final for the unit / read out by the epilogue
 //
 // MMA order of tile x inside a unit (j = key tile): S(x, 0) .. S(x, NBUF-1), then for
@@ -101,6 +101,9 @@ constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units: p <= 256
 // tiles; the rest use the MUFU unit.
 constexpr int EXP2_POLY_PAIRS = FA_EXP2_POLY_PAIRS;
 static_assert(EXP2_POLY_PAIRS >= 0 && EXP2_POLY_PAIRS <= 8, "pairs per 16-column chunk");
+#ifndef FA_D64_SCORE_BUFFERS
+#define FA_D64_SCORE_BUFFERS 2   // score buffers per Q tile at head dim 64 (2 or 3)
+#endif
 
 // Error bits written to the device error word when a bounded wait runs out.
 constexpr uint32_t ERR_WAIT_SOFTMAX = 1u << 0;
@@ -144,12 +147,15 @@ struct TileCfg {
   static constexpr uint32_t AB_FORMAT = FP8 ? 0u : 1u;  // e4m3 : bf16
   static constexpr uint32_t IDESC_S = ptx::make_idesc(AB_FORMAT, BM, BN, 0);
   static constexpr uint32_t IDESC_O = ptx::make_idesc(AB_FORMAT, BM, D, 1);
-  // TMEM column map.  Two score buffers per Q tile.  (At D = 64 tensor memory would hold a
-  // third, but the rescale's wait for the previous P.V product is a parity wait on one
-  // pv_done barrier, exact only while at most one product is outstanding: with S(j)
-  // issued after P.V(j-2), at most P.V(j-1) is.  A third buffer would need one pv_done
-  // barrier per product parity.)
-  static constexpr int NBUF = 2;
+  // TMEM column map.  Score buffers per Q tile: two; at D = 64 tensor memory also holds a
+  // third next to the two O accumulators (FA_D64_SCORE_BUFFERS = 3).  With S(j) issued
+  // after P.V(j-NBUF), up to NBUF-1 products may be outstanding when the softmax of key
+  // tile j rescales, so P.V product n commits to pv_done(x, n & 1): each of the two
+  // barriers then has at most one pending phase at that point, and a parity wait on it is
+  // exact for either count.  The third buffer passes parity but measured 0.7 % (non-causal)
+  // and 1.3 % (causal) slower at B 16, H 12, N 2048 on B200, so two is the default.
+  static constexpr int NBUF = D == 64 ? FA_D64_SCORE_BUFFERS : 2;
+  static_assert(NBUF == 2 || NBUF == 3, "two or three score buffers per Q tile");
   static constexpr uint32_t S_COLS = NBUF * 64;          // score columns of one Q tile
   __host__ __device__ static constexpr uint32_t s_col(int x, int b) { return x * S_COLS + b * 64; }
   static constexpr uint32_t P_OFF = 32;                  // P inside a 64-column S buffer
@@ -159,7 +165,7 @@ struct TileCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NT * Q_TILE_BYTES;
   static constexpr int BAR_OFF = RING_OFF + NSLOT * KV_TILE_BYTES;
-  static constexpr int NUM_BARS = 2 * NSLOT + 22 + 2 * UNIT_RING;
+  static constexpr int NUM_BARS = 2 * NSLOT + 24 + 2 * UNIT_RING;
   static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
   // control words: TMEM base, abort flag, 2 spare, then the ring of published units
   static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16 + 4 * UNIT_RING;
@@ -316,15 +322,16 @@ struct Bars {
   // three score buffers reserved per Q tile (TileCfg::NBUF of them used)
   __device__ uint32_t s_full(int x, int b) const { return base + 8u * (2 * NSLOT + 2 + 3 * x + b); }
   __device__ uint32_t p_full(int x, int b) const { return base + 8u * (2 * NSLOT + 8 + 3 * x + b); }
-  __device__ uint32_t pv_done(int x) const { return base + 8u * (2 * NSLOT + 14 + x); }
-  __device__ uint32_t o_full(int x) const { return base + 8u * (2 * NSLOT + 16 + x); }
-  __device__ uint32_t o_empty(int x) const { return base + 8u * (2 * NSLOT + 18 + x); }
-  __device__ uint32_t drain(int x) const { return base + 8u * (2 * NSLOT + 20 + x); }
+  // P.V product n of tile x commits to pv_done(x, n & 1)
+  __device__ uint32_t pv_done(int x, int q) const { return base + 8u * (2 * NSLOT + 14 + 2 * x + q); }
+  __device__ uint32_t o_full(int x) const { return base + 8u * (2 * NSLOT + 18 + x); }
+  __device__ uint32_t o_empty(int x) const { return base + 8u * (2 * NSLOT + 20 + x); }
+  __device__ uint32_t drain(int x) const { return base + 8u * (2 * NSLOT + 22 + x); }
   // ring of published work units: written (full) by the TMA warp, read (empty) by the
   // MMA and softmax warps
-  __device__ uint32_t unit_full(int s) const { return base + 8u * (2 * NSLOT + 22 + s); }
+  __device__ uint32_t unit_full(int s) const { return base + 8u * (2 * NSLOT + 24 + s); }
   __device__ uint32_t unit_empty(int s) const {
-    return base + 8u * (2 * NSLOT + 22 + UNIT_RING + s);
+    return base + 8u * (2 * NSLOT + 24 + UNIT_RING + s);
   }
 };
 
@@ -475,6 +482,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
   constexpr uint32_t SLOT_STEP = C::KV_TILE_BYTES >> 4;
   const uint32_t t_o = tmem + (x ? C::O_COL1 : C::O_COL0);
   uint32_t kv_base = 0;
+  uint32_t pvn = 0;  // P.V products this warp has issued (all units)
   uint32_t pph = 0;  // phase bits of p_full(x, b), bit b
   uint32_t unit_it = 0;
   auto wait = [&](uint32_t b, uint32_t parity) {
@@ -520,7 +528,8 @@ __device__ void mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
       ptx::tc_fence_after();
       issue_pv<D, FP8>(t_o, tmem + C::s_col(x, b) + C::P_OFF, v_d0 + (vi % C::NSLOT) * SLOT_STEP,
                        j > 0 ? 1u : 0u);
-      ptx::mma_commit_elect(bar.pv_done(x));
+      ptx::mma_commit_elect(bar.pv_done(x, pvn & 1u));
+      ++pvn;
       release(vi, x == 1 && j >= w.n0);
       if (j == nx - 1) ptx::mma_commit_elect(bar.o_full(x));
       if (j + C::NBUF < nx) {
@@ -713,9 +722,10 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       const float alpha = resc ? ptx::ex2(m_used - xmax) : 1.f;  // 0 on the first tile
       if (__any_sync(0xffffffffu, resc && j > 0)) {
         // The accumulator must be quiescent: wait for P(j-1) V(j-1) of this tile (the
-        // earlier products are covered by the commit that signalled S(j)); P(j) V(j) waits
-        // for p_full below.
-        ok = wait_phase(bar.pv_done(x), (pv_base + j - 1) & 1u, abort_flag, ERR_WAIT_SOFTMAX);
+        // products before P(j+1-NBUF) V are covered by the commit that signalled S(j));
+        // P(j) V(j) waits for p_full below.
+        const uint32_t pn = pv_base + j - 1;  // the previous product of this tile
+        ok = wait_phase(bar.pv_done(x, pn & 1u), (pn >> 1) & 1u, abort_flag, ERR_WAIT_SOFTMAX);
         if (!__all_sync(0xffffffffu, ok)) return;
         ptx::tc_fence_after();
 #pragma unroll 1
@@ -859,7 +869,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::mbar_init(bar.s_full(x, b), 1);
         ptx::mbar_init(bar.p_full(x, b), BM);
       }
-      ptx::mbar_init(bar.pv_done(x), 1);
+      ptx::mbar_init(bar.pv_done(x, 0), 1);
+      ptx::mbar_init(bar.pv_done(x, 1), 1);
       ptx::mbar_init(bar.o_full(x), 1);
       ptx::mbar_init(bar.o_empty(x), BM);
     }
