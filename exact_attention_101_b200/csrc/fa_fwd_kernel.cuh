@@ -164,7 +164,10 @@ struct TileCfg {
   // Shared memory map (offsets from a 1024-aligned base).
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NT * Q_TILE_BYTES;
-  static constexpr int BAR_OFF = RING_OFF + NSLOT * KV_TILE_BYTES;
+  // epilogue staging: 32 rows x 32 fp32 columns per softmax warp
+  static constexpr int STAGE_WARP_BYTES = 32 * 32 * 4;
+  static constexpr int STAGE_OFF = RING_OFF + NSLOT * KV_TILE_BYTES;
+  static constexpr int BAR_OFF = STAGE_OFF + 4 * NT * STAGE_WARP_BYTES;
   static constexpr int NUM_BARS = 2 * NSLOT + 24 + 2 * UNIT_RING;
   static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
   // control words: TMEM base, abort flag, 2 spare, then the ring of published units
@@ -647,7 +650,8 @@ __device__ __forceinline__ void softmax_numerators(const uint32_t (&sr)[4][16], 
 // row statistics are carried from tile to tile.
 template <int D, bool CAUSAL, bool OUT_F32, bool FP8, bool VARLEN, bool DROPOUT>
 __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileCfg<D, FP8>::NSLOT> &bar,
-                             volatile uint32_t *unit_ring, volatile uint32_t *abort_flag) {
+                             volatile uint32_t *unit_ring, volatile uint32_t *abort_flag,
+                             uint8_t *stage) {
   using C = TileCfg<D, FP8>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int x = warp / 4;              // Q tile handled by this warpgroup
@@ -791,10 +795,20 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       // the stores inside the tensors whatever the offsets say
       const bool valid = row < w.len_q && (!VARLEN || w.q_tok + row < p.Nq);
       const int hq = w.bh % p.Hq;
-      const size_t orow = VARLEN ? static_cast<size_t>(w.q_tok + (valid ? row : 0)) * p.Hq + hq
-                                 : static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
       const size_t lrow = VARLEN ? static_cast<size_t>(hq) * p.Nq + w.q_tok + (valid ? row : 0)
-                                 : orow;
+                                 : static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
+      // O leaves through this warp's staging buffer in shared memory, 32 columns at a time:
+      // each thread writes its row's 32 values, then the warp stores whole row segments (8
+      // rows of 64 bytes, or 4 rows of 128 bytes, per instruction) instead of 32 scattered
+      // 16-byte pieces.  Chunk positions are XOR-swizzled by row, so that neither the
+      // row-per-thread writes nor the segment reads meet bank conflicts.
+      constexpr int OB = OUT_F32 ? 4 : 2;   // bytes per output element
+      constexpr int SEG = 32 * OB;          // bytes of one row's 32 columns
+      constexpr int CH = SEG / 16;          // 16-byte chunks per segment
+      constexpr int RPI = 32 / CH;          // rows per store instruction
+      auto swz = [](int r) { return CH == 8 ? (r & 7) : ((r >> 1) & 3); };
+      uint8_t *const st = stage + warp * C::STAGE_WARP_BYTES;
+      const int row_w0 = row - lane;        // first row of this warp
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t a[16], bb[16];
@@ -803,30 +817,44 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
         ptx::tmem_wait_ld();
         ptx::reg_fence16(a);
         ptx::reg_fence16(bb);
-        if (valid) {
-          if (OUT_F32) {
-            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + c * 32);
+        uint4 v[CH];
+        if (OUT_F32) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_float4(__uint_as_float(a[4 * v]) * inv, __uint_as_float(a[4 * v + 1]) * inv,
-                                   __uint_as_float(a[4 * v + 2]) * inv, __uint_as_float(a[4 * v + 3]) * inv);
+          for (int q = 0; q < CH; ++q) {
+            const uint32_t *s4 = q < 4 ? a + 4 * q : bb + 4 * (q - 4);
+            v[q] = make_uint4(__float_as_uint(__uint_as_float(s4[0]) * inv),
+                              __float_as_uint(__uint_as_float(s4[1]) * inv),
+                              __float_as_uint(__uint_as_float(s4[2]) * inv),
+                              __float_as_uint(__uint_as_float(s4[3]) * inv));
+          }
+        } else {
+          uint32_t h[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[4 + v] = make_float4(__uint_as_float(bb[4 * v]) * inv, __uint_as_float(bb[4 * v + 1]) * inv,
-                                       __uint_as_float(bb[4 * v + 2]) * inv, __uint_as_float(bb[4 * v + 3]) * inv);
-          } else {
-            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + c * 32);
-            uint32_t h[16];
+          for (int e = 0; e < 8; ++e)
+            h[e] = ptx::pack_bf16x2(__uint_as_float(a[2 * e]) * inv, __uint_as_float(a[2 * e + 1]) * inv);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              h[e] = ptx::pack_bf16x2(__uint_as_float(a[2 * e]) * inv, __uint_as_float(a[2 * e + 1]) * inv);
+          for (int e = 0; e < 8; ++e)
+            h[8 + e] = ptx::pack_bf16x2(__uint_as_float(bb[2 * e]) * inv, __uint_as_float(bb[2 * e + 1]) * inv);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              h[8 + e] = ptx::pack_bf16x2(__uint_as_float(bb[2 * e]) * inv, __uint_as_float(bb[2 * e + 1]) * inv);
+          for (int q = 0; q < CH; ++q) v[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        }
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+        for (int q = 0; q < CH; ++q)
+          *reinterpret_cast<uint4 *>(st + lane * SEG + (q ^ swz(lane)) * 16) = v[q];
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+          const int r = k * RPI + lane / CH, q = lane % CH;
+          const uint4 val = *reinterpret_cast<const uint4 *>(st + r * SEG + (q ^ swz(r)) * 16);
+          const int rr = row_w0 + r;
+          if (rr < w.len_q && (!VARLEN || w.q_tok + rr < p.Nq)) {
+            const size_t orr = VARLEN ? static_cast<size_t>(w.q_tok + rr) * p.Hq + hq
+                                      : static_cast<size_t>(w.bh) * p.Nq + rr;
+            *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.o) + (orr * D + c * 32) * OB +
+                                       q * 16) = val;
           }
         }
+        __syncwarp();
       }
       if (valid)
         p.lse[lrow] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : NEG_INF;
@@ -898,7 +926,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::setmaxnreg_dec<OTHER_REGS>();
 
   if (warp < 4 * C::NT) {
-    softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN, DROPOUT>(p, tmem, bar, unit_ring, abort_flag);
+    softmax_role<D, CAUSAL, OUT_F32, FP8, VARLEN, DROPOUT>(p, tmem, bar, unit_ring, abort_flag,
+                                                          smem_gen + C::STAGE_OFF);
   } else if (warp == MMA_WARP || (C::NT == 2 && warp == MMA_WARP + 2)) {
     mma_role<D, CAUSAL, FP8, VARLEN>(p, smem, tmem, bar, warp == MMA_WARP ? 0 : 1, unit_ring,
                                      abort_flag);
