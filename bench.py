@@ -164,22 +164,61 @@ def profiled_traffic(workload_name):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons with nvidia-smi while the timed region runs."""
+    """SM clock, power and throttle reasons of this rank's GPU while the timed region runs.
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Polls NVML (the library nvidia-smi reads) every ~2 ms on a thread; begin()/end() mark the
+    timed window on the host clock and stop() summarises the samples inside it, so that even a
+    timed region of a few tens of milliseconds is described by samples taken under load.
+    Without NVML it falls back to nvidia-smi at its 100 ms interval (whole run)."""
 
-    def __init__(self, gpu_index):
-        self.gpu = str(gpu_index)
+    SMI_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+    def __init__(self, gpu_index, device=None):
+        self.gpu = gpu_index
+        self.device = device
+        self.samples = []          # (host time, sm MHz, reason bits, power W)
+        self.window = [None, None]
+        self.stop_flag = False
+        self.thread = None
         self.proc = None
         self.lines = []
-        self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.max_mhz = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        handle = None
+        try:  # NVML numbers all GPUs; match this rank's CUDA device by its PCI bus id
+            import torch
+            props = torch.cuda.get_device_properties(self.device if self.device is not None
+                                                     else self.gpu)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id,
+                                        props.pci_device_id)
+            handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            handle = pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu))
+        return pynvml, handle
 
     def start(self):
         try:
+            self.nvml, self.handle = self._nvml_handle()
+            self.max_mhz = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                    self.nvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu, "--query-gpu=" + self.QUERY,
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.SMI_QUERY,
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
@@ -188,11 +227,46 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while not self.stop_flag:
+            try:
+                self.samples.append((time.perf_counter(),
+                                     float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(h)),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1e3))
+            except Exception:
+                return
+            time.sleep(0.002)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def begin(self):
+        self.window[0] = time.perf_counter()
+
+    def end(self):
+        self.window[1] = time.perf_counter()
+
     def stop(self):
+        if self.nvml is not None:
+            time.sleep(0.005)
+            self.stop_flag = True
+            self.thread.join(timeout=2)
+            lo, hi = self.window
+            inside = [x for x in self.samples
+                      if (lo is None or x[0] >= lo) and (hi is None or x[0] <= hi)]
+            if not inside and self.samples and lo is not None:  # window shorter than a poll
+                inside = [min(self.samples, key=lambda x: abs(x[0] - lo))]
+            if not inside:
+                return None
+            reasons = sorted(n for n, bit in self.REASONS if any(x[2] & bit for x in inside))
+            sm = [x[1] for x in inside]
+            return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm),
+                    "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "power_w": round(statistics.median(x[3] for x in inside), 1),
+                    "samples": len(inside), "source": "nvml, 2 ms, timed window only"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -203,7 +277,7 @@ class ClockSampler:
         if self.thread:
             self.thread.join(timeout=2)
         sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _ in self.REASONS]
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
@@ -219,7 +293,8 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvidia-smi, 100 ms, whole run"}
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -438,7 +513,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     fa.check_device_error(stream)
 
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(local_rank, dev)
     clocks.start()
     time.sleep(0.3)
     barrier()
@@ -446,11 +521,13 @@ def run_ours(args):
     # One event at every step boundary: the total is first-to-last, and the per-step
     # times give the median and the best step.
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    clocks.begin()
     evs[0].record(stream)
     for i in range(args.steps):
         step(i)
         evs[i + 1].record(stream)
     torch.cuda.synchronize(dev)
+    clocks.end()
     barrier()
     clk = clocks.stop()
     fa.check_device_error(stream)
