@@ -113,7 +113,10 @@ constexpr int Q_OFF = 0;
 constexpr int RING_OFF = 2 * Q_TILE_BYTES;
 constexpr int XCH_OFF = RING_OFF + NSLOT * SLOT_BYTES;
 constexpr int XCH_BYTES = 3 * 2 * BM * 4;
-constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
+// epilogue staging: 32 rows x 64 bytes per softmax warp
+constexpr int STAGE_WARP_BYTES = 32 * 64;
+constexpr int STAGE_OFF = XCH_OFF + XCH_BYTES;
+constexpr int BAR_OFF = STAGE_OFF + 8 * STAGE_WARP_BYTES;
 constexpr int NUM_BARS = 2 * NSLOT + 27 + 2 * UNIT_RING_P;
 constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
 // control words: TMEM base, abort flag, 2 spare, then the unit ring
@@ -530,7 +533,7 @@ __device__ __forceinline__ void pair_numerators(const uint32_t (&sr)[4][32], flo
 template <bool CAUSAL, bool OUT_F32>
 __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars &bar,
                                   volatile uint32_t *ring, const Abort &ab, uint32_t rank,
-                                  volatile float *xch) {
+                                  volatile float *xch, uint8_t *stage) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = warp / 4;        // key stream (blocks j with j mod 2 == h); O dims [64 h, 64 h + 64)
   const int wq = warp % 4;       // TMEM lane quarter
@@ -717,6 +720,31 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const bool valid = row < p.Nq;
       const size_t orow = static_cast<size_t>(w.bh) * p.Nq + (valid ? row : 0);
+      // O leaves through this warp's staging buffer in shared memory, 64 bytes of each row
+      // (32 bf16 or 16 fp32 columns) at a time: each thread writes its row's four 16-byte
+      // chunks, XOR-swizzled by row so that the writes meet no bank conflicts, then the warp
+      // stores whole 64-byte row segments, 8 rows per instruction, instead of 32 scattered
+      // 16-byte pieces.
+      constexpr int OB = OUT_F32 ? 4 : 2;   // bytes per output element
+      uint8_t *const st = stage + warp * STAGE_WARP_BYTES;
+      const int row_w0 = row - lane;        // first row of this warp
+      auto put = [&](const uint4(&v)[4], int col) {  // col: first column of the segment
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4 *>(st + lane * 64 + (q ^ ((lane >> 1) & 3)) * 16) = v[q];
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = k * 8 + lane / 4, q = lane % 4;
+          const uint4 val = *reinterpret_cast<const uint4 *>(st + r * 64 + (q ^ ((r >> 1) & 3)) * 16);
+          const int rr = row_w0 + r;
+          if (rr < p.Nq)
+            *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.o) +
+                                       ((static_cast<size_t>(w.bh) * p.Nq + rr) * D + col) * OB +
+                                       q * 16) = val;
+        }
+        __syncwarp();
+      };
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const uint32_t col = h * 64 + c * 32;
@@ -724,23 +752,29 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
         ptx::tmem_ld32(t_o + col, a);
         ptx::tmem_wait_ld();
         ptx::reg_fence32(a);
-        if (valid) {
-          if (OUT_F32) {
-            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + col);
+        if (OUT_F32) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(__uint_as_float(a[4 * q]) * inv, __uint_as_float(a[4 * q + 1]) * inv,
-                                   __uint_as_float(a[4 * q + 2]) * inv, __uint_as_float(a[4 * q + 3]) * inv);
-          } else {
-            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + col);
-            uint32_t hh[16];
+          for (int half = 0; half < 2; ++half) {
+            uint4 v[4];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              hh[e] = ptx::pack_bf16x2(__uint_as_float(a[2 * e]) * inv, __uint_as_float(a[2 * e + 1]) * inv);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t *s4 = a + 16 * half + 4 * q;
+              v[q] = make_uint4(__float_as_uint(__uint_as_float(s4[0]) * inv),
+                                __float_as_uint(__uint_as_float(s4[1]) * inv),
+                                __float_as_uint(__uint_as_float(s4[2]) * inv),
+                                __float_as_uint(__uint_as_float(s4[3]) * inv));
+            }
+            put(v, col + 16 * half);
           }
+        } else {
+          uint32_t hh[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            hh[e] = ptx::pack_bf16x2(__uint_as_float(a[2 * e]) * inv, __uint_as_float(a[2 * e + 1]) * inv);
+          uint4 v[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) v[q] = make_uint4(hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
+          put(v, col);
         }
       }
       if (valid && h == 0)
@@ -823,7 +857,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ptx::setmaxnreg_dec<OTHER_REGS>();
 
   if (warp < 8) {
-    pair_softmax_role<CAUSAL, OUT_F32>(p, tmem, bar, ring, ab, rank, xch);
+    pair_softmax_role<CAUSAL, OUT_F32>(p, tmem, bar, ring, ab, rank, xch, smem_gen + STAGE_OFF);
   } else if (rank == 0 && warp == MMA_WARP) {
     pair_mma_role<CAUSAL>(p, smem, tmem, bar, ring, ab);
     __syncwarp();
