@@ -1,5 +1,8 @@
 // fa_fwd_pair.cuh -- the bf16 head-dimension-128 attention forward on CTA pairs (sm_100a).
 //
+// The library runs it without the causal mask; causal work goes to the one-CTA kernel,
+// which measured faster there (its CAUSAL instance is built with FA_PAIR_CAUSAL only).
+//
 // Same method as fa_fwd_kernel.cuh (the IO-aware tiled attention of the page "FlashAttention
 // (DE)", sections "Tiling und blockweise Verarbeitung", "Online-Softmax-Berechnung" and
 // "Zusammenfassen von Operationen in einem CUDA-Kernel"; the warp roles of the page
