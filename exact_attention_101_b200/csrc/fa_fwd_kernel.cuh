@@ -97,10 +97,18 @@ constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units: p <= 256
 #ifndef FA_EXP2_POLY_PAIRS
 #define FA_EXP2_POLY_PAIRS 0
 #endif
+#ifndef FA_EXP2_POLY_PAIRS_FP8
+#define FA_EXP2_POLY_PAIRS_FP8 2
+#endif
 // Column pairs (of every 8) whose exponentials use the FMA-pipe polynomial on unmasked
-// tiles; the rest use the MUFU unit.
+// tiles; the rest use the MUFU unit.  bf16: none (every share measured slower, at d = 64
+// by 13 % and more).  e4m3: its products take half the tensor time of bf16, so the SFU
+// leads by two to one; two pairs of eight measured 2.5 % faster (B8 H16 N4096 d128), and P
+// is rounded to e4m3 anyway, far coarser than the polynomial's 7.5e-5.
 constexpr int EXP2_POLY_PAIRS = FA_EXP2_POLY_PAIRS;
+constexpr int EXP2_POLY_PAIRS_FP8 = FA_EXP2_POLY_PAIRS_FP8;
 static_assert(EXP2_POLY_PAIRS >= 0 && EXP2_POLY_PAIRS <= 8, "pairs per 16-column chunk");
+static_assert(EXP2_POLY_PAIRS_FP8 >= 0 && EXP2_POLY_PAIRS_FP8 <= 8, "pairs per 16-column chunk");
 #ifndef FA_D64_SCORE_BUFFERS
 #define FA_D64_SCORE_BUFFERS 2   // score buffers per Q tile at head dim 64 (2 or 3)
 #endif
@@ -750,8 +758,9 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
       const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
 
       // Numerators p = 2^(s*sl2 - m_used), packed for the P V product.  Tiles without
-      // masked entries send EXP2_POLY_PAIRS of every 8 column pairs to the FMA-pipe
-      // polynomial and the rest to the MUFU unit.
+      // masked entries send NPOLY of every 8 column pairs to the FMA-pipe polynomial and
+      // the rest to the MUFU unit.
+      constexpr int NPOLY = FP8 ? EXP2_POLY_PAIRS_FP8 : EXP2_POLY_PAIRS;
       float le = 0.f;
       const uint32_t t_p = t_s + C::P_OFF;
       if (DROPOUT) {
@@ -765,12 +774,12 @@ __device__ void softmax_role(const FwdParams &p, uint32_t tmem, const Bars<TileC
           keep_bytes(r, p.drop_thr4, keep[h]);
         }
         softmax_numerators<FP8, 0, true>(sr, sl2, neg_m, t_p, le, keep);
-      } else if (EXP2_POLY_PAIRS == 0)   // one copy of the unrolled loop: smaller code, faster
+      } else if (NPOLY == 0)   // one copy of the unrolled loop: smaller code, faster
         softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, le);
       else if (need_mask)
         softmax_numerators<FP8, 0>(sr, sl2, neg_m, t_p, le);
       else
-        softmax_numerators<FP8, EXP2_POLY_PAIRS>(sr, sl2, neg_m, t_p, le);
+        softmax_numerators<FP8, NPOLY>(sr, sl2, neg_m, t_p, le);
       // O is normalised by the sum of the unrounded numerators: the bf16 (e4m3) values the
       // tensor core multiplies with V then sum to 1 within one rounding (2^-9 relative for
       // bf16), and the LSE comes from the same sum
