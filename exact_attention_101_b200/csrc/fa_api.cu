@@ -12,6 +12,7 @@
 #include <map>
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -236,9 +237,9 @@ bool pair_path(int d, bool fp8, int drop_thr, bool causal) {
 #else
 #ifdef FA_PAIR_CAUSAL
   (void)causal;
-  return d == fa::pair::D && !fp8 && drop_thr == 0;
+  return (d == 128 || d == 256) && !fp8 && drop_thr == 0;
 #else
-  return d == fa::pair::D && !fp8 && drop_thr == 0 && !causal;
+  return (d == 128 || d == 256) && !fp8 && drop_thr == 0 && !causal;
 #endif
 #endif
 }
@@ -250,9 +251,10 @@ int fwd_unit_rows(int d, bool pair) {
 
 // Clusters of the pair kernel that fit on device `dev` at once (0 if none), asked once per
 // device and instance.
-template <bool CAUSAL, bool OUT_F32>
+template <int D, bool CAUSAL, bool OUT_F32>
 fa_status pair_setup(int dev, int sms, int *clusters) {
-  auto kern = fa::pair::fa_fwd_pair_kernel<CAUSAL, OUT_F32>;
+  auto kern = fa::pair::fa_fwd_pair_kernel<D, CAUSAL, OUT_F32>;
+  constexpr int SMEM = fa::pair::PCfg<D>::SMEM_BYTES;
   static std::once_flag once[kMaxDevices];
   static fa_status st[kMaxDevices];
   static int n[kMaxDevices];
@@ -260,7 +262,7 @@ fa_status pair_setup(int dev, int sms, int *clusters) {
     st[dev] = FA_ERR_CUDA;
     n[dev] = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fa::pair::SMEM_BYTES) != cudaSuccess) {
+                             SMEM) != cudaSuccess) {
       cudaGetLastError();
       return;
     }
@@ -278,7 +280,7 @@ fa_status pair_setup(int dev, int sms, int *clusters) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2), 1, 1);
     cfg.blockDim = dim3(fa::pair::NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = fa::pair::SMEM_BYTES;
+    cfg.dynamicSmemBytes = SMEM;
     int c = 0;
     if (cudaOccupancyMaxActiveClusters(&c, kern, &cfg) != cudaSuccess) {
       cudaGetLastError();
@@ -291,34 +293,34 @@ fa_status pair_setup(int dev, int sms, int *clusters) {
   return st[dev];
 }
 
-template <bool CAUSAL, bool OUT_F32>
+template <int D, bool CAUSAL, bool OUT_F32>
 fa_status launch_pair(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                       const fa::FwdParams &params, int clusters, int dev, cudaStream_t stream) {
   fa::FwdParams p = params;
   if (sched_slot(dev, &p.sched) != FA_OK) return FA_ERR_CUDA;
   const int n = p.num_units < clusters ? p.num_units : clusters;
-  fa::pair::fa_fwd_pair_kernel<CAUSAL, OUT_F32>
-      <<<2 * n, fa::pair::NUM_THREADS, fa::pair::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  fa::pair::fa_fwd_pair_kernel<D, CAUSAL, OUT_F32>
+      <<<2 * n, fa::pair::NUM_THREADS, fa::pair::PCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <bool CAUSAL, bool OUT_F32>
+template <int D, bool CAUSAL, bool OUT_F32>
 fa_status run_pair(const void *q, const void *k, const void *v, int B, int Hq, int Hkv, int Nq,
                    int Nk, fa::FwdParams &p, const DeviceInfo &info, int dev, cudaStream_t stream,
                    bool *ran) {
   *ran = false;
   int clusters = 0;
-  const fa_status st = pair_setup<CAUSAL, OUT_F32>(dev, info.sms, &clusters);
+  const fa_status st = pair_setup<D, CAUSAL, OUT_F32>(dev, info.sms, &clusters);
   if (st != FA_OK || clusters < 1) return FA_OK;  // not resident here: the one-CTA kernel runs
   CUtensorMap tq, tk, tv;
-  if (!encode_tmap(&tq, q, false, fa::pair::D, Nq, static_cast<uint64_t>(B) * Hq, fa::pair::BM) ||
-      !encode_tmap(&tk, k, false, fa::pair::D, Nk, static_cast<uint64_t>(B) * Hkv, 64) ||
-      !encode_tmap(&tv, v, false, fa::pair::D, Nk, static_cast<uint64_t>(B) * Hkv, fa::pair::BN))
+  if (!encode_tmap(&tq, q, false, D, Nq, static_cast<uint64_t>(B) * Hq, fa::pair::BM) ||
+      !encode_tmap(&tk, k, false, D, Nk, static_cast<uint64_t>(B) * Hkv, 64) ||
+      !encode_tmap(&tv, v, false, D, Nk, static_cast<uint64_t>(B) * Hkv, fa::pair::BN))
     return FA_ERR_INVALID_ARG;
   p.num_qb = (Nq + fa::pair::UNIT_ROWS - 1) / fa::pair::UNIT_ROWS;
   p.num_units = B * Hq * p.num_qb;
   *ran = true;
-  return launch_pair<CAUSAL, OUT_F32>(tq, tk, tv, p, clusters, dev, stream);
+  return launch_pair<D, CAUSAL, OUT_F32>(tq, tk, tv, p, clusters, dev, stream);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -414,16 +416,22 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
   if (pair_path(d, fp8, drop_thr, causal)) {
     bool ran = false;
 #ifdef FA_PAIR_CAUSAL
-    const fa_status ps =
-        causal ? (out_f32 ? run_pair<true, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
-                          : run_pair<true, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran))
-               : (out_f32 ? run_pair<false, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
-                          : run_pair<false, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran));
+    auto run = [&](auto dd) {
+      constexpr int DD = decltype(dd)::value;
+      return causal ? (out_f32 ? run_pair<DD, true, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
+                               : run_pair<DD, true, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran))
+                    : (out_f32 ? run_pair<DD, false, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
+                               : run_pair<DD, false, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran));
+    };
 #else
-    const fa_status ps =
-        out_f32 ? run_pair<false, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
-                : run_pair<false, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran);
+    auto run = [&](auto dd) {
+      constexpr int DD = decltype(dd)::value;
+      return out_f32 ? run_pair<DD, false, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
+                     : run_pair<DD, false, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran);
+    };
 #endif
+    const fa_status ps = d == 128 ? run(std::integral_constant<int, 128>())
+                                  : run(std::integral_constant<int, 256>());
     if (ran || ps != FA_OK) return ps;
     p.num_qb = (Nq + unit_rows - 1) / unit_rows;
     p.num_units = B * Hq * p.num_qb;

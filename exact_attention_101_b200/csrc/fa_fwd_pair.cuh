@@ -68,7 +68,6 @@
 namespace fa {
 namespace pair {
 
-constexpr int D = 128;
 constexpr int BM = 128;                     // query rows of a unit held by one CTA
 constexpr int BN = 128;                     // keys per block (N of S over the pair)
 constexpr int UNIT_ROWS = 2 * BM;           // query rows per unit (MMA M)
@@ -90,16 +89,10 @@ constexpr int POLY_PAIRS = FA_PAIR_POLY_PAIRS;
 static_assert(POLY_PAIRS >= 0 && POLY_PAIRS <= 8, "pairs per 16-column chunk");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int Q_BOX_BYTES = BM * 128;       // 128 rows x 128 bytes (64 dims)
-constexpr int Q_TILE_BYTES = 2 * Q_BOX_BYTES;
-constexpr int K_BOX_BYTES = 64 * 128;       // 64 keys x 128 bytes
-constexpr int SLOT_BYTES = 16384;           // K half: 2 boxes; V half: 128 keys x 64 dims
-constexpr int NSLOT = 8;
-constexpr int S_KSTEPS = D / 16;
+constexpr int K_BOX_BYTES = 64 * 128;       // 64 keys x 128 bytes (64 dims)
+constexpr int V_BOX_BYTES = BN * 128;       // 128 keys x 128 bytes (64 dims)
 constexpr int PV_KSTEPS = BN / 16;
 constexpr uint32_t IDESC_S = ptx::make_idesc(1u, 256, BN, 0);
-constexpr uint32_t IDESC_O = ptx::make_idesc(1u, 256, D, 1);
-constexpr uint32_t O_COL0 = 256;            // the accumulator O (128 columns)
-constexpr uint32_t P_COL0 = 384;            // numerator buffers P(b) at P_COL0 + 64 b
 constexpr int UNIT_RING_P = 4;
 // consumers of a published unit: CTA 0's MMA warp and eight softmax warps, CTA 1's eight
 // softmax warps and its producer
@@ -107,25 +100,60 @@ constexpr uint32_t UNIT_CONSUMERS = 1 + 8 + 8 + 1;
 constexpr uint32_t SOFTMAX_WARPS_PAIR = 16;  // softmax warps of both CTAs (o_empty)
 constexpr uint32_t STREAM_WARPS_PAIR = 8;    // one stream's softmax warps, both CTAs
 constexpr uint16_t BOTH = 0x3;              // CTA mask of the pair
-
-// shared memory: two Q buffers (unit parity), the K/V ring, the per-row maximum handed
-// between the streams [2 streams][128 rows] (and the exact running maximum, for the rescale
-// statistics), the epilogue's sum exchange [2 streams][128 rows] (fp32), the mbarriers and
-// the control words
-constexpr int Q_OFF = 0;
-constexpr int RING_OFF = 2 * Q_TILE_BYTES;
-constexpr int XCH_OFF = RING_OFF + NSLOT * SLOT_BYTES;
+// the per-row maximum handed between the streams [2 streams][128 rows] (and the exact
+// running maximum, for the rescale statistics) and the epilogue's sum exchange [2
+// streams][128 rows], fp32
 constexpr int XCH_BYTES = 3 * 2 * BM * 4;
-// epilogue staging: 32 rows x 64 bytes per softmax warp
-constexpr int STAGE_WARP_BYTES = 32 * 64;
-constexpr int STAGE_OFF = XCH_OFF + XCH_BYTES;
-constexpr int BAR_OFF = STAGE_OFF + 8 * STAGE_WARP_BYTES;
-constexpr int NUM_BARS = 2 * NSLOT + 27 + 2 * UNIT_RING_P;
-constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
-// control words: TMEM base, abort flag, 2 spare, then the unit ring
-constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16 + 4 * UNIT_RING_P;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+constexpr int STAGE_WARP_BYTES = 32 * 64;   // epilogue staging: 32 rows x 64 bytes per warp
 
+// Layout for head dimension D (128 or 256).
+//   Q: this CTA's 128 rows in D/64 boxes of 64 dims; two buffers (unit parity) at D = 128,
+//      one at D = 256 (the next unit's Q then loads after the unit's last S).
+//   Ring slot: a K half (64 keys x D dims, D/64 boxes) or a V half (128 keys x D/2 dims,
+//      D/128 boxes of 64 dims); 128 KB of slots.
+//   Tensor memory: S(b) at 128 b (128 fp32 columns), O at 256 (D columns), and the bf16
+//      numerators P(b): at D = 128 in their own columns (384 + 64 b), so that S(j+2) can be
+//      computed while block j's numerators are still being formed; at D = 256 O takes the
+//      last 256 columns, so P(b) goes over the first 64 columns of S(b), and S(j+2) waits
+//      until P(j) V has been issued (products of one thread run in issue order).
+template <int D>
+struct PCfg {
+  static_assert(D == 128 || D == 256, "head dims of the pair kernel");
+  static constexpr int NQBOX = D / 64;
+  static constexpr int Q_TILE_BYTES = NQBOX * Q_BOX_BYTES;
+  static constexpr int NQBUF = D == 128 ? 2 : 1;
+  static constexpr int NKBOX = D / 64;
+  static constexpr int NVBOX = D / 128;
+  static constexpr int SLOT_BYTES = NKBOX * K_BOX_BYTES;
+  static_assert(NVBOX * V_BOX_BYTES == SLOT_BYTES, "K and V halves fill one slot");
+  static constexpr int NSLOT = 131072 / SLOT_BYTES;
+  static constexpr int S_KSTEPS = D / 16;
+  static constexpr uint32_t IDESC_O = ptx::make_idesc(1u, 256, D, 1);
+  static constexpr bool ALIAS_P = D == 256;
+  static constexpr uint32_t O_COL0 = 256;
+  __host__ __device__ static constexpr uint32_t p_col(int b) {
+    return ALIAS_P ? 128u * b : 384u + 64u * b;
+  }
+  // S(k) may be issued once P(k - 1 - S_LEAD) V has been issued: at D = 128 that keeps every
+  // pv_done barrier at most one phase ahead of the softmax's parity waits; at D = 256 it also
+  // keeps S(k) behind the P V that reads P(k-2) from the same columns
+  static constexpr int S_LEAD = ALIAS_P ? 1 : 2;
+  static_assert(O_COL0 + D <= TMEM_COLS, "TMEM budget");
+  // shared memory: the Q buffers, the K/V ring, the exchange, the epilogue staging, the
+  // mbarriers and the control words
+  static constexpr int Q_OFF = 0;
+  static constexpr int RING_OFF = NQBUF * Q_TILE_BYTES;
+  static constexpr int XCH_OFF = RING_OFF + NSLOT * SLOT_BYTES;
+  static constexpr int STAGE_OFF = XCH_OFF + XCH_BYTES;
+  static constexpr int BAR_OFF = STAGE_OFF + 8 * STAGE_WARP_BYTES;
+  static constexpr int NUM_BARS = 2 * NSLOT + 27 + 2 * UNIT_RING_P;
+  static constexpr int CTL_OFF = BAR_OFF + NUM_BARS * 8;
+  // control words: TMEM base, abort flag, 2 spare, then the unit ring
+  static constexpr int SMEM_BYTES = 1024 + CTL_OFF + 16 + 4 * UNIT_RING_P;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int NSLOT>
 struct PBars {
   uint32_t base;
   __device__ uint32_t slot_full(int s) const { return base + 8u * s; }
@@ -228,11 +256,13 @@ __device__ __forceinline__ PUnit pair_decode(const FwdParams &p, int u) {
 // ring.  Each CTA copies its own 128 rows of Q (into the buffer of the unit's parity) and
 // its halves of every K and V block; all copies complete on CTA 0's barriers, which CTA 0
 // arms with the bytes of both.
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __device__ void pair_load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK,
                                const CUtensorMap *tmV, const FwdParams &p, uint32_t smem,
-                               const PBars &bar, volatile uint32_t *ring, const Abort &ab,
-                               uint32_t rank) {
+                               const PBars<PCfg<D>::NSLOT> &bar, volatile uint32_t *ring,
+                               const Abort &ab, uint32_t rank) {
+  using C = PCfg<D>;
+  constexpr int NSLOT = C::NSLOT;
   ptx::prefetch_tmap(tmQ);
   ptx::prefetch_tmap(tmK);
   ptx::prefetch_tmap(tmV);
@@ -257,14 +287,15 @@ __device__ void pair_load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK,
     if (u >= num_units) break;
     {
       const PUnit w = pair_decode<CAUSAL>(p, static_cast<int>(u));
-      const int qb = q_issued & 1;
-      if (!pwait(bar.q_empty(qb), ((q_issued >> 1) & 1u) ^ 1u, ab, ERR_WAIT_LOAD)) goto drain;
-      if (rank == 0) ptx::mbar_arrive_expect_tx(bar.q_full(qb), 2 * Q_TILE_BYTES);
+      const int qb = q_issued % C::NQBUF;
+      if (!pwait(bar.q_empty(qb), ((q_issued / C::NQBUF) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
+        goto drain;
+      if (rank == 0) ptx::mbar_arrive_expect_tx(bar.q_full(qb), 2 * C::Q_TILE_BYTES);
       const uint32_t qf = ptx::mapa(bar.q_full(qb), 0);
 #pragma unroll
-      for (int bx = 0; bx < 2; ++bx)
-        ptx::tma_load_3d_pair(smem + Q_OFF + qb * Q_TILE_BYTES + bx * Q_BOX_BYTES, tmQ, qf,
-                              bx * 64, w.r0 + static_cast<int>(rank) * BM, w.bh);
+      for (int bx = 0; bx < C::NQBOX; ++bx)
+        ptx::tma_load_3d_pair(smem + C::Q_OFF + qb * C::Q_TILE_BYTES + bx * Q_BOX_BYTES, tmQ,
+                              qf, bx * 64, w.r0 + static_cast<int>(rank) * BM, w.bh);
       ++q_issued;
       // K and V halves in the order the MMA warp first needs them: K_0, K_1, then per block
       // j K_(j+2) (its scores are computed early) and V_j
@@ -272,13 +303,13 @@ __device__ void pair_load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK,
         const int sl = issued % NSLOT;
         if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
           return false;
-        if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
+        if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * C::SLOT_BYTES);
         const uint32_t sf = ptx::mapa(bar.slot_full(sl), 0);
-        // keys j*BN + 64 rank .. + 63, all dimensions (two 64-dimension boxes)
+        // keys j*BN + 64 rank .. + 63, all dimensions (D/64 boxes of 64 dimensions)
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
-          ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES + bx * K_BOX_BYTES, tmK, sf,
-                                bx * 64, j * BN + static_cast<int>(rank) * 64, w.bhk);
+        for (int bx = 0; bx < C::NKBOX; ++bx)
+          ptx::tma_load_3d_pair(smem + C::RING_OFF + sl * C::SLOT_BYTES + bx * K_BOX_BYTES, tmK,
+                                sf, bx * 64, j * BN + static_cast<int>(rank) * 64, w.bhk);
         ++issued;
         return true;
       };
@@ -286,19 +317,26 @@ __device__ void pair_load_role(const CUtensorMap *tmQ, const CUtensorMap *tmK,
         const int sl = issued % NSLOT;
         if (!pwait(bar.slot_empty(sl), ((issued / NSLOT) & 1u) ^ 1u, ab, ERR_WAIT_LOAD))
           return false;
-        if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * SLOT_BYTES);
-        // keys j*BN .. + 127, dimensions 64 rank .. + 63
-        ptx::tma_load_3d_pair(smem + RING_OFF + sl * SLOT_BYTES, tmV,
-                              ptx::mapa(bar.slot_full(sl), 0), static_cast<int>(rank) * 64,
-                              j * BN, w.bhk);
+        if (rank == 0) ptx::mbar_arrive_expect_tx(bar.slot_full(sl), 2 * C::SLOT_BYTES);
+        const uint32_t sf = ptx::mapa(bar.slot_full(sl), 0);
+        // keys j*BN .. + 127, dimensions (D/2) rank .. + D/2 - 1 (D/128 boxes of 64 dimensions)
+#pragma unroll
+        for (int bx = 0; bx < C::NVBOX; ++bx)
+          ptx::tma_load_3d_pair(smem + C::RING_OFF + sl * C::SLOT_BYTES + bx * V_BOX_BYTES, tmV,
+                                sf, static_cast<int>(rank) * (D / 2) + bx * 64, j * BN, w.bhk);
         ++issued;
         return true;
       };
       if (!load_k(0)) goto drain;
       if (w.n > 1 && !load_k(1)) goto drain;
       for (int j = 0; j < w.n; ++j) {
-        if (j + 2 < w.n && !load_k(j + 2)) goto drain;
-        if (!load_v(j)) goto drain;
+        if (C::ALIAS_P) {
+          if (!load_v(j)) goto drain;
+          if (j + 2 < w.n && !load_k(j + 2)) goto drain;
+        } else {
+          if (j + 2 < w.n && !load_k(j + 2)) goto drain;
+          if (!load_v(j)) goto drain;
+        }
       }
     }
     if (rank == 0) u = ptx::num_clusters_x() + atomicAdd(p.sched, 1u);
@@ -312,10 +350,10 @@ drain:
         drain_wait(bar.slot_full(s), (last / NSLOT) & 1u);
       }
     }
-    for (uint32_t qb = 0; qb < 2; ++qb) {
+    for (uint32_t qb = 0; qb < C::NQBUF; ++qb) {
       if (q_issued > qb) {
-        const uint32_t last = qb + 2 * ((q_issued - 1 - qb) / 2);
-        drain_wait(bar.q_full(qb), (last >> 1) & 1u);
+        const uint32_t last = qb + C::NQBUF * ((q_issued - 1 - qb) / C::NQBUF);
+        drain_wait(bar.q_full(qb), (last / C::NQBUF) & 1u);
       }
     }
   } else if (*ab.flag) {
@@ -329,9 +367,10 @@ drain:
 
 // ---------------------------------------------------------------------------- MMA issuer
 
+template <int D>
 __device__ __forceinline__ void pair_issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
 #pragma unroll
-  for (int kk = 0; kk < S_KSTEPS; ++kk) {
+  for (int kk = 0; kk < PCfg<D>::S_KSTEPS; ++kk) {
     const uint32_t kb = kk * 32;  // bytes along the head dimension
     const uint32_t qoff = ((kb / 128) * Q_BOX_BYTES + (kb % 128)) >> 4;
     const uint32_t koff = ((kb / 128) * K_BOX_BYTES + (kb % 128)) >> 4;
@@ -339,23 +378,30 @@ __device__ __forceinline__ void pair_issue_s(uint32_t tmem_s, uint64_t q_desc, u
   }
 }
 
-__device__ __forceinline__ void pair_issue_pv(uint32_t tmem_o, uint32_t tmem_s, uint64_t v_desc,
+template <int D>
+__device__ __forceinline__ void pair_issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t v_desc,
                                               uint32_t accumulate) {
-  // V half is [128 keys x 64 dims], dims contiguous: an MN-major B operand of one 128-byte
-  // swizzle atom across N; 16 key rows of 128 bytes per K-step.
+  // V half is [128 keys x D/2 dims], dims contiguous: an MN-major B operand of D/128 swizzle
+  // atoms (128-byte dimension chunks, one box apart: the LBO of v_desc) across N; 16 key rows
+  // of 128 bytes per K-step.
 #pragma unroll
   for (int kk = 0; kk < PV_KSTEPS; ++kk) {
     const uint32_t off = (kk * 16 * 128) >> 4;
-    ptx::mma2_bf16_ts_elect(tmem_o, tmem_s + kk * 8, v_desc + off, IDESC_O,
+    ptx::mma2_bf16_ts_elect(tmem_o, tmem_p + kk * 8, v_desc + off, PCfg<D>::IDESC_O,
                             kk > 0 ? 1u : accumulate);
   }
 }
 
-// Ring position, inside a unit of n key blocks, of K_k and V_j in the producer's order
-// K_0, K_1, then per block j: K_(j+2) (while j + 2 < n), V_j.
-__device__ __forceinline__ uint32_t k_pos(int k) { return k < 2 ? k : 2 * k - 2; }
+// Ring position, inside a unit of n key blocks, of K_k and V_j in the producer's order, the
+// order in which the MMA warp first needs them: K_0, K_1, then per block j K_(j+2) (while
+// j + 2 < n) and V_j -- or, where S(j+2) follows P(j) V (P over S, D = 256), V_j and K_(j+2).
+template <int D>
+__device__ __forceinline__ uint32_t k_pos(int k) {
+  return k < 2 ? k : (PCfg<D>::ALIAS_P ? 2 * k - 1 : 2 * k - 2);
+}
+template <int D>
 __device__ __forceinline__ uint32_t v_pos(int j, int n) {
-  return (n > 1 ? 2 : 1) + j + min(j + 1, max(n - 2, 0));
+  return (n > 1 ? 2 : 1) + j + min(PCfg<D>::ALIAS_P ? j : j + 1, max(n - 2, 0));
 }
 
 // Warp 8 of CTA 0.  Every commit that frees a resource or signals a result arrives on the
@@ -364,14 +410,17 @@ __device__ __forceinline__ uint32_t v_pos(int j, int n) {
 // K_k has landed and P(k-3) V has been issued, or P(j) V_j once the numerators P(j) are
 // written -- so scores for the next blocks never queue behind a product that waits for the
 // softmax.
-template <bool CAUSAL>
-__device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, const PBars &bar,
-                              volatile uint32_t *ring, const Abort &ab) {
-  const uint64_t q_d0 = ptx::smem_desc_sw128(smem + Q_OFF, 16, 1024);
-  const uint64_t k_d0 = ptx::smem_desc_sw128(smem + RING_OFF, 16, 1024);
-  const uint64_t v_d0 = ptx::smem_desc_sw128(smem + RING_OFF, SLOT_BYTES, 1024);
-  constexpr uint32_t SLOT_STEP = SLOT_BYTES >> 4;
-  constexpr uint32_t QBUF_STEP = Q_TILE_BYTES >> 4;
+template <int D, bool CAUSAL>
+__device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem,
+                              const PBars<PCfg<D>::NSLOT> &bar, volatile uint32_t *ring,
+                              const Abort &ab) {
+  using C = PCfg<D>;
+  constexpr int NSLOT = C::NSLOT;
+  const uint64_t q_d0 = ptx::smem_desc_sw128(smem + C::Q_OFF, 16, 1024);
+  const uint64_t k_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, 16, 1024);
+  const uint64_t v_d0 = ptx::smem_desc_sw128(smem + C::RING_OFF, V_BOX_BYTES, 1024);
+  constexpr uint32_t SLOT_STEP = C::SLOT_BYTES >> 4;
+  constexpr uint32_t QBUF_STEP = C::Q_TILE_BYTES >> 4;
   uint32_t kv_base = 0, unit_it = 0, taken = 0;
   uint32_t pph = 0;           // phase bits of p_full(b), bit b
   uint32_t sfph = 0;          // phase bits of s_free(b), bit b
@@ -400,25 +449,26 @@ __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, 
     if (u >= static_cast<uint32_t>(p.num_units)) break;
     const PUnit w = pair_decode<CAUSAL>(p, static_cast<int>(u));
     const int n = w.n;
-    const int qb = unit_it & 1;
+    const int qb = unit_it % C::NQBUF;
     const uint64_t q_d = q_d0 + qb * QBUF_STEP;
-    if (!wait(bar.q_full(qb), (unit_it >> 1) & 1u)) break;
+    if (!wait(bar.q_full(qb), (unit_it / C::NQBUF) & 1u)) break;
     int next_s = 0, next_pv = 0;
     uint64_t t_idle = 0;  // start of the current run of probes without progress
     uint32_t spins = 0;
     while (next_pv < n) {
       bool progressed = false;
-      // S(k) only after P(k-3) V has been issued: products of one thread complete in
+      // S(k) only after P(k-1-S_LEAD) V has been issued: products of one thread complete in
       // order, so when the softmax sees S(k), every pv_done barrier has at most one pending
-      // phase (P(k-1) V or P(k-2) V), which its parity waits rely on
-      if (next_s < n && next_s <= next_pv + 2) {
+      // phase (P(k-1) V or P(k-2) V), which its parity waits rely on; where P shares S's
+      // columns (S_LEAD 1), S(k) also follows the P(k-2) V that reads them
+      if (next_s < n && next_s <= next_pv + C::S_LEAD) {
         const int k = next_s, b = k & 1;
         const bool buf_free = !((s_issued >> b) & 1u) || ready(bar.s_free(b), (sfph >> b) & 1u);
-        const uint32_t ki = kv_base + k_pos(k);
+        const uint32_t ki = kv_base + k_pos<D>(k);
         if (buf_free && slot_ready(ki)) {
           if ((s_issued >> b) & 1u) sfph ^= 1u << b;
           ptx::tc_fence_after();
-          pair_issue_s(tmem + b * BN, q_d, k_d0 + (ki % NSLOT) * SLOT_STEP);
+          pair_issue_s<D>(tmem + b * BN, q_d, k_d0 + (ki % NSLOT) * SLOT_STEP);
           ptx::mma2_commit_mc_elect(bar.s_full(b), BOTH);
           ptx::mma2_commit_mc_elect(bar.slot_empty(ki % NSLOT), BOTH);
           if (k == n - 1) ptx::mma2_commit_mc_elect(bar.q_empty(qb), BOTH);
@@ -429,14 +479,14 @@ __device__ void pair_mma_role(const FwdParams &p, uint32_t smem, uint32_t tmem, 
       }
       if (next_pv < next_s) {
         const int j = next_pv, b = j & 1;
-        const uint32_t vi = kv_base + v_pos(j, n);
+        const uint32_t vi = kv_base + v_pos<D>(j, n);
         // the previous unit's epilogue has read O before P(0) V overwrites it
         if (ready(bar.p_full(b), (pph >> b) & 1u) && slot_ready(vi) &&
             (j > 0 || ready(bar.o_empty(), (unit_it & 1u) ^ 1u))) {
           pph ^= 1u << b;
           ptx::tc_fence_after();
-          pair_issue_pv(tmem + O_COL0, tmem + P_COL0 + b * 64, v_d0 + (vi % NSLOT) * SLOT_STEP,
-                        j > 0 ? 1u : 0u);
+          pair_issue_pv<D>(tmem + C::O_COL0, tmem + C::p_col(b), v_d0 + (vi % NSLOT) * SLOT_STEP,
+                           j > 0 ? 1u : 0u);
           ptx::mma2_commit_mc_elect(bar.pv_done(b), BOTH);
           ptx::mma2_commit_mc_elect(bar.slot_empty(vi % NSLOT), BOTH);
           if (j == n - 1) ptx::mma2_commit_mc_elect(bar.o_full(), BOTH);
@@ -533,8 +583,9 @@ __device__ __forceinline__ void pair_numerators(const uint32_t (&sr)[4][32], flo
   le += a0 + a1;
 }
 
-template <bool CAUSAL, bool OUT_F32>
-__device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars &bar,
+template <int D, bool CAUSAL, bool OUT_F32>
+__device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem,
+                                  const PBars<PCfg<D>::NSLOT> &bar,
                                   volatile uint32_t *ring, const Abort &ab, uint32_t rank,
                                   volatile float *xch, uint8_t *stage) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -543,8 +594,9 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
   const int r_cta = wq * 32 + lane;  // row inside the CTA's 128
   const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
   const uint32_t t_s = tmem + lane_base + h * BN;
-  const uint32_t t_o = tmem + lane_base + O_COL0;
-  const uint32_t t_p = tmem + lane_base + P_COL0 + h * 64;
+  using C = PCfg<D>;
+  const uint32_t t_o = tmem + lane_base + C::O_COL0;
+  const uint32_t t_p = tmem + lane_base + C::p_col(h);
   const uint32_t p_full_c = ptx::mapa(bar.p_full(h), 0);
   const uint32_t s_free_c = ptx::mapa(bar.s_free(h), 0);
   const uint32_t o_empty_c = ptx::mapa(bar.o_empty(), 0);
@@ -749,8 +801,8 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
         __syncwarp();
       };
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const uint32_t col = h * 64 + c * 32;
+      for (int c = 0; c < D / 64; ++c) {
+        const uint32_t col = h * (D / 2) + c * 32;
         uint32_t a[32];
         ptx::tmem_ld32(t_o + col, a);
         ptx::tmem_wait_ld();
@@ -794,7 +846,7 @@ __device__ void pair_softmax_role(const FwdParams &p, uint32_t tmem, const PBars
 
 // ---------------------------------------------------------------------------- kernel
 
-template <bool CAUSAL, bool OUT_F32>
+template <int D, bool CAUSAL, bool OUT_F32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -803,12 +855,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t smem = (raw + 1023u) & ~1023u;  // 1024-aligned for 128-byte swizzle
   uint8_t *smem_gen = smem_raw + (smem - raw);
-  const PBars bar{smem + BAR_OFF};
-  uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + CTL_OFF);
+  using C = PCfg<D>;
+  const PBars<C::NSLOT> bar{smem + C::BAR_OFF};
+  uint32_t *ctl = reinterpret_cast<uint32_t *>(smem_gen + C::CTL_OFF);
   volatile uint32_t *tmem_slot = ctl;
   volatile uint32_t *abort_flag = ctl + 1;
   volatile uint32_t *ring = ctl + 4;
-  volatile float *xch = reinterpret_cast<volatile float *>(smem_gen + XCH_OFF);
+  volatile float *xch = reinterpret_cast<volatile float *>(smem_gen + C::XCH_OFF);
   const uint32_t rank = ptx::cluster_ctarank();
   const Abort ab{abort_flag, ptx::mapa(ptx::smem_addr(ctl + 1), rank ^ 1u)};
 
@@ -816,7 +869,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NSLOT; ++s) {
+    for (int s = 0; s < C::NSLOT; ++s) {
       ptx::mbar_init(bar.slot_full(s), 1);
       ptx::mbar_init(bar.slot_empty(s), 1);
     }
@@ -860,12 +913,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ptx::setmaxnreg_dec<OTHER_REGS>();
 
   if (warp < 8) {
-    pair_softmax_role<CAUSAL, OUT_F32>(p, tmem, bar, ring, ab, rank, xch, smem_gen + STAGE_OFF);
+    pair_softmax_role<D, CAUSAL, OUT_F32>(p, tmem, bar, ring, ab, rank, xch, smem_gen + C::STAGE_OFF);
   } else if (rank == 0 && warp == MMA_WARP) {
-    pair_mma_role<CAUSAL>(p, smem, tmem, bar, ring, ab);
+    pair_mma_role<D, CAUSAL>(p, smem, tmem, bar, ring, ab);
     __syncwarp();
   } else if (warp == TMA_WARP) {
-    if (lane == 0) pair_load_role<CAUSAL>(&tmQ, &tmK, &tmV, p, smem, bar, ring, ab, rank);
+    if (lane == 0) pair_load_role<D, CAUSAL>(&tmQ, &tmK, &tmV, p, smem, bar, ring, ab, rank);
     __syncwarp();
   }
 

@@ -46,17 +46,19 @@ class MBarrier:
         return self.phase != parity
 
 
-def k_pos(k):
-    return k if k < 2 else 2 * k - 2
+def k_pos(k, alias):
+    return k if k < 2 else (2 * k - 1 if alias else 2 * k - 2)
 
 
-def v_pos(j, n):
-    return (2 if n > 1 else 1) + j + min(j + 1, max(n - 2, 0))
+def v_pos(j, n, alias):
+    return (2 if n > 1 else 1) + j + min(j if alias else j + 1, max(n - 2, 0))
 
 
 class PairModel:
-    def __init__(self, units, seed, nslot=8, rescale_p=0.3, mutant=None):
-        self.units, self.nslot, self.mutant = units, nslot, mutant
+    def __init__(self, units, seed, nslot=8, rescale_p=0.3, mutant=None, alias=False):
+        # alias: the head-dim-256 layout, where P(b) lies over the first columns of S(b), the
+        # producer loads V_j before K_(j+2), and S(k) waits until P(k-2) V has been issued
+        self.units, self.nslot, self.mutant, self.alias = units, nslot, mutant, alias
         self.rng = random.Random(seed)
         self.rescale_p = rescale_p
         self.slot_full = [MBarrier() for _ in range(nslot)]
@@ -86,9 +88,12 @@ class PairModel:
         for u, n in enumerate(self.units):
             order = [("K", 0)] + ([("K", 1)] if n > 1 else [])
             for j in range(n):
+                if self.alias:
+                    order.append(("V", j))
                 if j + 2 < n:
                     order.append(("K", j + 2))
-                order.append(("V", j))
+                if not self.alias:
+                    order.append(("V", j))
             for kind, idx in order:
                 s = issued % self.nslot
                 yield lambda s=s, ph=((issued // self.nslot) & 1) ^ 1: self.slot_empty[s].done(ph)
@@ -103,7 +108,7 @@ class PairModel:
             return False
         k, b = m["next_s"], m["next_s"] & 1
         buf_free = not (m["s_issued"] >> b) & 1 or self.s_free[b].done((m["sfph"] >> b) & 1)
-        ki = m["kv_base"] + k_pos(k)
+        ki = m["kv_base"] + k_pos(k, self.alias)
         return buf_free and self.slot_full[ki % self.nslot].done((ki // self.nslot) & 1)
 
     def _can_values(self, m):
@@ -111,14 +116,19 @@ class PairModel:
         if not m["next_pv"] < m["next_s"]:
             return False
         j, b = m["next_pv"], m["next_pv"] & 1
-        vi = m["kv_base"] + v_pos(j, n)
+        vi = m["kv_base"] + v_pos(j, n, self.alias)
         o_ok = j > 0 or self.mutant == "no_o_empty_wait" or self.o_empty.done((m["unit_it"] & 1) ^ 1)
         return (self.p_full[b].done((m["pph"] >> b) & 1) and o_ok and
                 self.slot_full[vi % self.nslot].done((vi // self.nslot) & 1))
 
     def _mma(self):
+        lead = 1 if self.alias else 2
+        if self.mutant == "scores_four_ahead":
+            lead = 3
+        elif self.mutant == "alias_scores_three_ahead":
+            lead = 2
         m = dict(kv_base=0, pph=0, sfph=0, unit_it=0, u=0, next_s=0, next_pv=0, s_issued=0,
-                 lead=3 if self.mutant == "scores_four_ahead" else 2)
+                 lead=lead)
         for u, n in enumerate(self.units):
             m.update(u=u, next_s=0, next_pv=0)  # s_issued persists across units
             if self.mutant == "buffers_free_at_unit_start":
@@ -127,7 +137,7 @@ class PairModel:
                 progressed = False
                 if self._can_scores(m):
                     k, b = m["next_s"], m["next_s"] & 1
-                    ki = m["kv_base"] + k_pos(k)
+                    ki = m["kv_base"] + k_pos(k, self.alias)
                     if (m["s_issued"] >> b) & 1:
                         m["sfph"] ^= 1 << b
                     self.tc += [("S", u, k, ki % self.nslot),
@@ -137,7 +147,7 @@ class PairModel:
                     progressed = True
                 if self._can_values(m):
                     j, b = m["next_pv"], m["next_pv"] & 1
-                    vi = m["kv_base"] + v_pos(j, n)
+                    vi = m["kv_base"] + v_pos(j, n, self.alias)
                     m["pph"] ^= 1 << b
                     bars = [self.pv_done[b], self.slot_empty[vi % self.nslot]]
                     if j == n - 1:
@@ -178,6 +188,8 @@ class PairModel:
                     yield lambda p=nn & 1: self.pv_done[h].done(p)
                 prev = self.pbuf[h]
                 assert prev is None or prev[2], ("P overwritten before its P V read it", prev, u, j)
+                if self.alias:  # P(j) goes over the columns S(j) came from
+                    assert self.sbuf[h] == ("S", u, j), ("P written over other scores", self.sbuf[h], u, j)
                 self.pbuf[h] = (u, j, False)
                 self.p_full[h].arrive()
             # epilogue
@@ -210,6 +222,9 @@ class PairModel:
         kind, u, j, s = op
         if kind == "S":
             assert self.slot[s] == ("K", u, j), ("S reads K", self.slot[s], u, j)
+            if self.alias:
+                pb = self.pbuf[j & 1]
+                assert pb is None or pb[2], ("S overwrites P before its P V read it", pb, u, j)
             self.sbuf[j & 1] = ("S", u, j)
         else:
             assert self.slot[s] == ("V", u, j), ("P V reads V", self.slot[s], u, j)
@@ -248,10 +263,13 @@ def unit_mix(rng):
     return [rng.randint(1, 9) for _ in range(rng.randint(1, 5))]
 
 
-@pytest.mark.parametrize("nslot", [8, 4])
-def test_pair_handshakes_are_race_free(nslot):
+@pytest.mark.parametrize("alias,nslot", [(False, 8), (False, 4), (True, 4), (True, 2)])
+def test_pair_handshakes_are_race_free(alias, nslot):
+    """Head dim 128 (separate numerator buffers, 8 slots) and 256 (P over S, 4 slots), and
+    smaller rings."""
     for seed in range(250):
-        PairModel(unit_mix(random.Random(seed)), seed, nslot=nslot, rescale_p=0.5).run()
+        PairModel(unit_mix(random.Random(seed)), seed, nslot=nslot, rescale_p=0.5,
+                  alias=alias).run()
 
 
 @pytest.mark.parametrize("mutant", ["scores_four_ahead", "numerators_without_wait",
@@ -265,3 +283,16 @@ def test_model_catches_a_planted_mistake(mutant):
         except AssertionError:
             caught += 1
     assert caught > 0, mutant
+
+
+def test_model_catches_scores_over_unread_numerators():
+    """With P over S, S(k) issued before P(k-2) V (the head-dim-128 lead of two) overwrites
+    numerators the tensor core has not read yet."""
+    caught = 0
+    for seed in range(150):
+        try:
+            PairModel(unit_mix(random.Random(seed)), seed, nslot=4, rescale_p=0.5, alias=True,
+                      mutant="alias_scores_three_ahead").run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0
