@@ -239,7 +239,7 @@ bool pair_path(int d, bool fp8, int drop_thr, bool causal) {
   (void)causal;
   return (d == 128 || d == 256) && !fp8 && drop_thr == 0;
 #else
-  return (d == 128 || d == 256) && !fp8 && drop_thr == 0 && !causal;
+  return (d == 256 || (d == 128 && !causal)) && !fp8 && drop_thr == 0;
 #endif
 #endif
 }
@@ -424,8 +424,12 @@ fa_status fwd_common(const void *q, const void *k, const void *v, void *o, float
                                : run_pair<DD, false, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran));
     };
 #else
+    // head dim 128: without the mask only; head dim 256: both
     auto run = [&](auto dd) {
       constexpr int DD = decltype(dd)::value;
+      if (DD == 256 && causal)
+        return out_f32 ? run_pair<256, true, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
+                       : run_pair<256, true, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran);
       return out_f32 ? run_pair<DD, false, true>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran)
                      : run_pair<DD, false, false>(q, k, v, B, Hq, Hkv, Nq, Nk, p, info, dev, stream, &ran);
     };

@@ -93,9 +93,9 @@ def test_varlen_fp32_output(cuda_ok):
 @pytest.mark.parametrize("d", [64, 128, 256])
 def test_varlen_equal_lengths_equal_fixed_length(cuda_ok, causal, d):
     """Packed sequences of one length against the [B, H, N, d] path.  Where both run the
-    same tiles of the one-CTA kernel (head dim 64, and 128 and 256 under the causal mask):
-    equal bits.  At 128 and 256 without the mask the fixed-length path runs the CTA-pair
-    kernel (another summation order): equal within the bf16 bar."""
+    same tiles of the one-CTA kernel (head dim 64, and 128 under the causal mask): equal
+    bits.  Elsewhere the fixed-length path runs the CTA-pair kernel (another summation
+    order): equal within the bf16 bar."""
     dev = torch.device("cuda", 0)
     B, H, N = 3, 4, 385
     q, k, v = (random_bf16((B, H, N, d), 400 + s) for s in range(3))
@@ -106,7 +106,7 @@ def test_varlen_equal_lengths_equal_fixed_length(cuda_ok, causal, d):
     torch.cuda.synchronize()
     o1 = o1.permute(0, 2, 1, 3).reshape(B * N, H, d)
     l1 = l1.permute(1, 0, 2).reshape(H, B * N)
-    if d == 64 or causal:
+    if d == 64 or (d == 128 and causal):
         assert torch.equal(o1, o2)
         assert torch.equal(l1, l2)
     else:
