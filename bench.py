@@ -641,13 +641,13 @@ def run_ours(args):
                "api": ("fa_fwd_host: pinned host buffers, copies pipelined by head chunks"
                        if host_api else "pinned copies on the stream around the device call")}
 
-    # Lazy-rescale statistics of the d = 128 bf16 forward without the causal mask (its
-    # kernel, the CTA-pair one, counts them): one more launch on the workload's inputs and
-    # one on scores that drift along the keys (same shape), each against the eager rule's
-    # count on the same rows.
+    # Lazy-rescale statistics of the forward instances on the CTA-pair kernel (it counts
+    # them): one more launch on the workload's inputs and one on scores that drift along the
+    # keys (same shape), each against the eager rule's count on the same rows.
+    pair_kernel = (w.kind == "fwd" and not fp8 and not w.dropout
+                   and (w.d == 256 or (w.d == 128 and not w.causal)))
     rescale = None
-    if (w.kind == "fwd" and not fp8 and not w.dropout and w.d == 128 and w.out_dtype == "bf16"
-            and not w.causal):
+    if pair_kernel and w.out_dtype == "bf16":
         def counts(qq, kk, vv):
             fa.rescale_stats(reset=True, stream=stream)
             fa.forward(qq, kk, vv, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
@@ -696,9 +696,7 @@ def run_ours(args):
             rate, desc, cores, _, _ = oracle_sample_rate(w, inp, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
                "cpu_model": cpu_model(), "nproc": os.cpu_count()}
-    kernel_name = ("fa_fwd_pair_kernel (CTA pairs)" if (w.d == 128 and not fp8 and not w.dropout
-                                                      and w.kind == "fwd" and not w.causal)
-                   else "fa_fwd_kernel")
+    kernel_name = "fa_fwd_pair_kernel (CTA pairs)" if pair_kernel else "fa_fwd_kernel"
     if w.kind == "bwd":
         kernel_name = ("fa_bwd: prep kernel + fa_bwd_kernel + dQ kernel (and the dQ "
                        "accumulator memset), timed together as one call")

@@ -225,11 +225,12 @@ fa_status launch(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// The bf16 forward at head dimension 128 without dropout and without the causal mask runs
-// on CTA pairs (fa_fwd_pair.cuh) unless the library is built with FA_NO_PAIR_KERNEL.  Under
-// the causal mask the one-CTA kernel measured faster on B200 (GQA causal B4 Hq32 Hkv8 N8192:
-// 1 205 against 1 167 TFLOP/s; long causal level), so causal work stays there unless the
-// library is built with FA_PAIR_CAUSAL (which sends it to the pair kernel's causal instance).
+// The bf16 forward without dropout runs on CTA pairs (fa_fwd_pair.cuh) at head dimension
+// 256, and at 128 without the causal mask, unless the library is built with
+// FA_NO_PAIR_KERNEL.  Under the causal mask at 128 the one-CTA kernel measured faster on
+// B200 (GQA causal B4 Hq32 Hkv8 N8192: 1 205 against 1 167 TFLOP/s; long causal level), so
+// that work stays there unless the library is built with FA_PAIR_CAUSAL.  At 256 the pair
+// wins either way (long d256: 1 465 against 1 190, causal 1 409 against 1 168).
 bool pair_path(int d, bool fp8, int drop_thr, bool causal) {
 #ifdef FA_NO_PAIR_KERNEL
   (void)d; (void)fp8; (void)drop_thr; (void)causal;

@@ -1,7 +1,11 @@
-// fa_fwd_pair.cuh -- the bf16 head-dimension-128 attention forward on CTA pairs (sm_100a).
+// fa_fwd_pair.cuh -- the bf16 attention forward on CTA pairs, head dims 128 and 256
+// (sm_100a).
 //
-// The library runs it without the causal mask; causal work goes to the one-CTA kernel,
-// which measured faster there (its CAUSAL instance is built with FA_PAIR_CAUSAL only).
+// The library runs it at head dim 128 without the causal mask (causal work there goes to
+// the one-CTA kernel, which measured faster; the pair's causal instance at 128 is built with
+// FA_PAIR_CAUSAL only) and at head dim 256 with or without it.  The text below describes
+// D = 128; PCfg gives what changes at D = 256 (four Q boxes and one Q buffer, 32 KB ring
+// slots, a V half of 128 dimensions, O of 256 columns and P over the first columns of S).
 //
 // Same method as fa_fwd_kernel.cuh (the IO-aware tiled attention of the page "FlashAttention
 // (DE)", sections "Tiling und blockweise Verarbeitung", "Online-Softmax-Berechnung" and

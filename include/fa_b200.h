@@ -306,10 +306,10 @@ fa_status fa_check_device_error(fa_stream_t stream);
  * Praxisleitfaden ...", section "Intelligenteres Online-Softmax-Rescaling in FA4", states
  * that rescaling the accumulator only when the running maximum has moved far (here: by
  * more than 8 in log2 units) needs about ten times fewer rescales than doing so whenever
- * it moves.  The bf16 head-dimension-128 forward without the causal mask (fa_fwd and
- * fa_fwd_host at d = 128, causal = 0: the CTA-pair kernel) counts, per (query row, key
- * block) step, whether it rescaled, and whether the eager rule would have; the other
- * kernel instances count nothing.  Counters are per device and sum
+ * it moves.  The CTA-pair kernel -- fa_fwd and fa_fwd_host in bf16 at d = 128 without
+ * the causal mask and at d = 256 with or without it -- counts, per (query row, key block)
+ * step, whether it rescaled, and whether the eager rule would have; the other kernel
+ * instances count nothing.  Counters are per device and sum
  * over all launches (concurrent ones included) since the last reset.
  *
  * fa_rescale_stats synchronises `stream`, then writes the counters of the current device:
