@@ -38,6 +38,8 @@ def check_lse(lse, Nq, Nk, causal):
     ((2, 6, 3, 385, 385, 64), False, torch.float32),
     ((16, 12, 12, 512, 512, 64), True, torch.bfloat16),     # 384 units
     ((1, 2, 2, 300, 1000, 256), True, torch.bfloat16),
+    ((2, 16, 4, 2048, 2048, 256), False, torch.float32),   # 256 units on CTA pairs
+    ((2, 4, 2, 513, 129, 256), True, torch.bfloat16),      # rows without keys, CTA pairs
     ((3, 4, 1, 513, 129, 128), True, torch.bfloat16),       # rows without keys
     ((1, 3, 3, 1, 1, 64), False, torch.float32),
 ])

@@ -115,10 +115,12 @@ def test_varlen_equal_lengths_equal_fixed_length(cuda_ok, causal, d):
         assert (l1 - l2).abs().max().item() <= 1e-3
 
 
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (129, 513), (513, 129), (1, 700)])
-def test_fixed_length_causal_bottom_right(cuda_ok, nq, nk):
+def test_fixed_length_causal_bottom_right(cuda_ok, nq, nk, d):
+    """Head dim 128 runs the one-CTA kernel under the mask, 256 the CTA-pair kernel."""
     dev = torch.device("cuda", 0)
-    B, Hq, Hkv, d = 1, 4, 2, 128
+    B, Hq, Hkv = 1, 4, 2
     q = random_bf16((B, Hq, nq, d), 500)
     k, v = random_bf16((B, Hkv, nk, d), 501), random_bf16((B, Hkv, nk, d), 502)
     o, lse = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal=True, scale=D_SCALE[d])
