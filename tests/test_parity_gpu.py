@@ -179,7 +179,7 @@ def test_fp8_full_size(cuda_ok):
 @pytest.mark.skipif(os.environ.get("FA_WHOLE_TENSOR") != "1",
                     reason="opt-in whole-tensor comparison (set FA_WHOLE_TENSOR=1)")
 @pytest.mark.parametrize("name", ["gpt2", "gpt2_causal", "long", "long_causal", "gqa_causal",
-                                  "fp8"])
+                                  "fp8", "long_d256", "long_d256_causal"])
 def test_whole_tensor(cuda_ok, name):
     w = W[name]
     inp = workloads.make_inputs(w)
