@@ -33,8 +33,10 @@
  * where the library's kernels are loaded, from the first call on that device until the
  * process exits, whichever entry points are used.
  *
- * Work distribution: the forward and backward kernels run one persistent CTA per SM, and
- * the CTAs claim work units from a counter of their launch.  The counters are 4096 pairs
+ * Work distribution: the forward and backward kernels run one persistent CTA per SM (the
+ * bf16 forward at head dim 256, and at 128 without the causal mask, one cluster of two CTAs
+ * per two SMs, each pair sharing its tensor-core products), and the CTAs claim work units
+ * from a counter of their launch.  The counters are 4096 pairs
  * of 32-bit words per device in the library's static device memory.  Every launch takes
  * the next pair (round-robin per device) and leaves it at zero when it ends.  So at most
  * 4096 of these launches may be in flight on one device at the same time; more, on
