@@ -4,10 +4,9 @@
 Scores that drift along the keys keep raising the running row maximum, so the accumulator
 is rescaled on many key blocks: the results must still match the oracle (head dims 64, 128,
 256 and fp8).  The CTA-pair kernel (head dim 128 without the mask, 256) also counts its
-rescales (fa_rescale_stats): the number of
-(row, key block) steps follows from the shapes, the drift forces lazy rescales, the eager
-rule would have made more, and on i.i.d. normal inputs the lazy rule never fires after a
-row's first key block."""
+rescales (fa_rescale_stats): the number of (row, key block) steps follows from the shapes,
+the drift forces lazy rescales, the eager rule would have made more, and on i.i.d. normal
+inputs the lazy rule never fires after a row's first key block."""
 import math
 
 import numpy as np
