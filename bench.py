@@ -45,6 +45,14 @@ KERNEL_SOURCES = ["exact_attention_101_b200/csrc/fa_fwd_kernel.cuh",
 
 # ------------------------------------------------------------------ host-side helpers
 
+def uses_pair_kernel(w, fp8):
+    """Whether the library runs this forward workload on its CTA-pair kernel (bf16 without
+    dropout at head dim 256, and at 128 without the causal mask), as fa_api.cu's pair_path
+    decides."""
+    return (w.kind == "fwd" and not fp8 and not w.dropout
+            and (w.d == 256 or (w.d == 128 and not w.causal)))
+
+
 def rank_env():
     """(rank, local_rank, world_size) from the torchrun environment (defaults 0, 0, 1)."""
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
@@ -583,10 +591,13 @@ def run_ours(args):
     # kernels per end-to-end step: fa_fwd_host's default chunk count (as many K/V heads per
     # chunk as fit one wave of work units), else the device call's own launches
     if host_api:
-        unit_rows = 128 if w.d > 128 else 256
+        # the library's chunk plan: as many K/V heads per chunk as fit one wave of work
+        # units (CTA pairs: one unit per two SMs; one-CTA kernel at d = 256: 128-row units)
+        pair = uses_pair_kernel(w, fp8)
+        unit_rows = 128 if (w.d > 128 and not pair) else 256
         group_units = (w.Hq // w.Hkv) * (-(-w.N // unit_rows))
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        per = max(1, sms // group_units)
+        per = max(1, (sms // 2 if pair else sms) // group_units)
         e2e_launches = e2e_steps * (-(-(w.B * w.Hkv) // per))
     else:
         e2e_launches = e2e_steps * launches_per_step
@@ -644,8 +655,7 @@ def run_ours(args):
     # Lazy-rescale statistics of the forward instances on the CTA-pair kernel (it counts
     # them): one more launch on the workload's inputs and one on scores that drift along the
     # keys (same shape), each against the eager rule's count on the same rows.
-    pair_kernel = (w.kind == "fwd" and not fp8 and not w.dropout
-                   and (w.d == 256 or (w.d == 128 and not w.causal)))
+    pair_kernel = uses_pair_kernel(w, fp8)
     rescale = None
     if pair_kernel and w.out_dtype == "bf16":
         def counts(qq, kk, vv):
