@@ -34,3 +34,38 @@ def test_fp8_per_head_amax_quantisation():
         assert torch.all(vals.abs().amax(dim=1) == 448.0)
         # outliers (x50) push amax far above the N(0,1) bulk
         assert torch.all(ds * 448.0 > 10.0)
+
+
+def test_drift_inputs_move_the_scores_along_the_keys():
+    """The drifting-score recipe: seeded, bf16, and each row's scores grow or shrink along
+    the keys by far more than their spread within a block, so that on the rows that grow
+    the online softmax's running maximum keeps moving."""
+    a = workloads.drift_inputs(1, 2, 512, 64, seed=3)
+    b = workloads.drift_inputs(1, 2, 512, 64, seed=3)
+    assert torch.equal(a.q, b.q) and torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
+    assert a.q.dtype == torch.bfloat16 and a.k.shape == (1, 2, 512, 64)
+    s = torch.einsum("bhqd,bhkd->bhqk", a.q.float(), a.k.float())
+    first, last = s[..., :64].mean(dim=-1), s[..., -64:].mean(dim=-1)
+    spread = s[..., :64].std(dim=-1)
+    # a trend well above the noise on nearly every row (a row nearly orthogonal to the
+    # ramp's direction has little)
+    assert ((last - first).abs() > 2 * spread).float().mean() > 0.9
+    rising = (last > first).float().mean()
+    assert 0.2 < rising < 0.8                             # both directions occur
+
+
+def test_quantise_inputs_matches_the_fp8_recipe():
+    """quantise_inputs_e4m3 applies the fp8 workload's own per-(batch, head) quantisation:
+    the slice amax maps onto 448 and codes times descale give back the input within half a
+    code step."""
+    x = workloads.drift_inputs(1, 2, 256, 128, seed=4)
+    y = workloads.quantise_inputs_e4m3(x)
+    for src, codes, ds in ((x.q, y.q, y.descale_q), (x.k, y.k, y.descale_k), (x.v, y.v, y.descale_v)):
+        vals = codes.to(torch.float32).reshape(2, -1)
+        assert torch.all(vals.abs().amax(dim=1) == 448.0)
+        back = vals * ds[:, None]
+        err = (back - src.float().reshape(2, -1)).abs()
+        # e4m3 has 3 mantissa bits: half a step is at most 1/16 of the magnitude (plus the
+        # subnormal step near zero)
+        bound = src.float().reshape(2, -1).abs() / 16 + ds[:, None] * 2.0 ** -9
+        assert torch.all(err <= bound + 1e-6)
